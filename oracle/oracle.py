@@ -1,0 +1,212 @@
+"""ctypes front end of the CPU oracle (oracle/svg2_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by __graft_entry__.smoke() and by bench.py's
+cpu_baseline / reference leg.  The product path (the CUDA library and its Python binding) never
+imports this module.
+
+Per-head helpers compose the C functions in the order of the pages' Method section
+("Sparse VideoGen2" wiki summary): k-means on Q and K, centroid scores, top-p, permutation,
+sparse attention, inverse permutation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "svg2_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no FMA contraction, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-std=c11", "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64, i32, f64, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_float
+        L.svg2o_kmeanspp.argtypes = [P, i64, i32, i32, P, P, P]
+        L.svg2o_kmeanspp.restype = i32
+        L.svg2o_assign.argtypes = [P, i64, i32, P, i32, P, P, P]
+        L.svg2o_update.argtypes = [P, i64, i32, P, i32, P, P]
+        L.svg2o_lloyd.argtypes = [P, i64, i32, i32, i32, P, P, P]
+        L.svg2o_select_weights.argtypes = [P, P, P, i32, i32, i32, f64, P]
+        L.svg2o_topp.argtypes = [P, P, i32, i32, f32, P]
+        L.svg2o_permute.argtypes = [P, i64, i32, P, P]
+        L.svg2o_gather_rows.argtypes = [P, P, i64, i32, P]
+        L.svg2o_unpermute.argtypes = [P, P, i64, i32, P]
+        L.svg2o_sparse_attention_rows.argtypes = [P, P, P, i64, i32, P, P, i32, i32, P, f64, P, i64, P]
+        L.svg2o_dense_attention_rows.argtypes = [P, P, P, i64, i32, f64, P, i64, P]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def kmeanspp(X: np.ndarray, k: int, u: np.ndarray):
+    X = _f32(X)
+    N, d = X.shape
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    seeds = np.zeros(k, np.int64)
+    C = np.zeros((k, d), np.float64)
+    rc = lib().svg2o_kmeanspp(_p(X), N, d, k, _p(u), _p(seeds), _p(C))
+    if rc != 0:
+        raise RuntimeError(f"svg2o_kmeanspp failed: {rc}")
+    return seeds, C
+
+
+def assign(X: np.ndarray, C: np.ndarray):
+    X = _f32(X)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    N, d = X.shape
+    labels = np.zeros(N, np.int32)
+    d1 = np.zeros(N, np.float64)
+    d2 = np.zeros(N, np.float64)
+    lib().svg2o_assign(_p(X), N, d, _p(C), C.shape[0], _p(labels), _p(d1), _p(d2))
+    return labels, d1, d2
+
+
+def update(X: np.ndarray, labels: np.ndarray, C: np.ndarray):
+    X = _f32(X)
+    C = np.array(C, dtype=np.float64, copy=True, order="C")
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    counts = np.zeros(C.shape[0], np.int32)
+    lib().svg2o_update(_p(X), X.shape[0], X.shape[1], _p(labels), C.shape[0], _p(C), _p(counts))
+    return C, counts
+
+
+def lloyd(X: np.ndarray, C0: np.ndarray, iters: int):
+    X = _f32(X)
+    C = np.array(C0, dtype=np.float64, copy=True, order="C")
+    N, d = X.shape
+    labels = np.zeros(N, np.int32)
+    counts = np.zeros(C.shape[0], np.int32)
+    lib().svg2o_lloyd(_p(X), N, d, C.shape[0], iters, _p(C), _p(labels), _p(counts))
+    return C, labels, counts
+
+
+def select_weights(cq: np.ndarray, ck: np.ndarray, count_k: np.ndarray, scale: float):
+    cq, ck = _f32(cq), _f32(ck)
+    count_k = np.ascontiguousarray(count_k, dtype=np.int32)
+    nQ, d = cq.shape
+    nK = ck.shape[0]
+    w = np.zeros((nQ, nK), np.float32)
+    lib().svg2o_select_weights(_p(cq), _p(ck), _p(count_k), nQ, nK, d, float(scale), _p(w))
+    return w
+
+
+def topp(w: np.ndarray, count_k: np.ndarray, p: float):
+    w = _f32(w)
+    count_k = np.ascontiguousarray(count_k, dtype=np.int32)
+    nQ, nK = w.shape
+    mask = np.zeros((nQ, nK), np.uint8)
+    lib().svg2o_topp(_p(w), _p(count_k), nQ, nK, float(np.float32(p)), _p(mask))
+    return mask
+
+
+def permute(labels: np.ndarray, k: int):
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    perm = np.zeros(labels.size, np.int32)
+    offsets = np.zeros(k + 1, np.int32)
+    lib().svg2o_permute(_p(labels), labels.size, k, _p(perm), _p(offsets))
+    return perm, offsets
+
+
+def gather_rows(X: np.ndarray, perm: np.ndarray):
+    X = _f32(X)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    out = np.zeros_like(X)
+    lib().svg2o_gather_rows(_p(X), _p(perm), X.shape[0], X.shape[1], _p(out))
+    return out
+
+
+def unpermute(Op: np.ndarray, perm: np.ndarray):
+    Op = np.ascontiguousarray(Op, dtype=np.float64)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    O = np.zeros_like(Op)
+    lib().svg2o_unpermute(_p(Op), _p(perm), Op.shape[0], Op.shape[1], _p(O))
+    return O
+
+
+def sparse_attention_rows(Qp, Kp, Vp, q_off, k_off, mask, scale, rows=None):
+    Qp, Kp, Vp = _f32(Qp), _f32(Kp), _f32(Vp)
+    N, d = Qp.shape
+    q_off = np.ascontiguousarray(q_off, dtype=np.int32)
+    k_off = np.ascontiguousarray(k_off, dtype=np.int32)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.zeros((rows.size, d), np.float64)
+    lib().svg2o_sparse_attention_rows(_p(Qp), _p(Kp), _p(Vp), N, d, _p(q_off), _p(k_off),
+                                      q_off.size - 1, k_off.size - 1, _p(mask), float(scale),
+                                      _p(rows), rows.size, _p(out))
+    return out
+
+
+def dense_attention_rows(Q, K, V, scale, rows=None):
+    Q, K, V = _f32(Q), _f32(K), _f32(V)
+    N, d = Q.shape
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.zeros((rows.size, d), np.float64)
+    lib().svg2o_dense_attention_rows(_p(Q), _p(K), _p(V), N, d, float(scale), _p(rows), rows.size, _p(out))
+    return out
+
+
+def kmeans(X: np.ndarray, k: int, iters: int, u: Optional[np.ndarray] = None,
+           C0: Optional[np.ndarray] = None):
+    """k-means++ seeding (or the given C0), then `iters` Lloyd iterations."""
+    if C0 is None:
+        _, C0 = kmeanspp(X, k, u)
+    return lloyd(X, C0, iters)
+
+
+def layer_head(q, k, v, nQ, nK, iters, top_p, scale, uq=None, uk=None, cq0=None, ck0=None,
+               rows=None) -> Dict[str, np.ndarray]:
+    """The whole layer for one (batch, head), as the Method section orders it.
+
+    `rows` (original token indices) restricts the attention to those output rows.
+    """
+    cq, lq, count_q = kmeans(q, nQ, iters, uq, cq0)
+    ck, lk, count_k = kmeans(k, nK, iters, uk, ck0)
+    w = select_weights(cq.astype(np.float32), ck.astype(np.float32), count_k, scale)
+    mask = topp(w, count_k, top_p)
+    perm_q, q_off = permute(lq, nQ)
+    perm_k, k_off = permute(lk, nK)
+    Qp, Kp, Vp = gather_rows(q, perm_q), gather_rows(k, perm_k), gather_rows(v, perm_k)
+    out = {"cq": cq, "ck": ck, "labels_q": lq, "labels_k": lk, "count_q": count_q, "count_k": count_k,
+           "weights": w, "mask": mask, "perm_q": perm_q, "perm_k": perm_k, "q_off": q_off, "k_off": k_off}
+    if rows is None:
+        Op = sparse_attention_rows(Qp, Kp, Vp, q_off, k_off, mask, scale)
+        out["o"] = unpermute(Op, perm_q)
+    else:
+        inv = np.empty_like(perm_q)
+        inv[perm_q] = np.arange(perm_q.size, dtype=np.int32)
+        out["o_rows"] = sparse_attention_rows(Qp, Kp, Vp, q_off, k_off, mask, scale, inv[np.asarray(rows)])
+    return out
+
+
+def density(mask: np.ndarray, count_q: np.ndarray, count_k: np.ndarray) -> float:
+    """Fraction of the dense score matrix that the selected cluster pairs cover."""
+    cq = count_q.astype(np.float64)
+    ck = count_k.astype(np.float64)
+    n = cq.sum()
+    return float((mask.astype(np.float64) * cq[:, None] * ck[None, :]).sum() / (n * n))

@@ -1,0 +1,328 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix (no GPU needed).
+
+Each test checks an oracle function against something other than itself: a library routine
+(scikit-learn's Lloyd, scipy distances and softmax, numpy's stable argsort, torch's
+scaled_dot_product_attention in float64), a closed form, an invariant, or brute force on tiny
+inputs.  The method is "Sparse VideoGen2" (wiki summary page, Key claims and Method).
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import scipy.spatial.distance as ssd
+import scipy.special
+import torch
+from sklearn.cluster import KMeans
+
+from sparse_attention_video_head_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _mixture(n, d, comps, sigma, seed):
+    rng = np.random.default_rng(seed)
+    centres = rng.standard_normal((comps, d)).astype(np.float32)
+    lab = rng.integers(0, comps, n)
+    return (centres[lab] + sigma * rng.standard_normal((n, d)).astype(np.float32)).astype(np.float32), lab
+
+
+# ---------------------------------------------------------------- k-means (Method (1), section 4.1)
+
+def test_assign_is_brute_force_argmin_with_lowest_index_ties(oracle):
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((300, 8)).astype(np.float32)
+    C = rng.standard_normal((7, 8))
+    C[5] = C[2]                                   # exact duplicate: ties must go to index 2
+    labels, d1, d2 = oracle.assign(X, C)
+    D = ssd.cdist(X.astype(np.float64), C, "sqeuclidean")
+    assert np.array_equal(labels, np.argmin(D, axis=1))   # argmin returns the first minimum
+    assert not np.any(labels == 5)
+    Ds = np.sort(D, axis=1)
+    np.testing.assert_allclose(d1, Ds[:, 0], rtol=1e-12)
+    np.testing.assert_allclose(d2, Ds[:, 1], rtol=1e-12)
+
+
+@pytest.mark.parametrize("iters", [1, 3, 8])
+def test_lloyd_matches_scikit_learn(oracle, iters):
+    X, _ = _mixture(600, 16, 6, 0.4, 2)
+    C0 = X[[0, 50, 100, 150, 200, 250, 300]].astype(np.float64)
+    C, labels, counts = oracle.lloyd(X, C0, iters)
+    km = KMeans(n_clusters=7, init=C0, n_init=1, max_iter=iters, tol=0.0, algorithm="lloyd").fit(
+        X.astype(np.float64))
+    assert counts.min() > 0
+    np.testing.assert_allclose(C, km.cluster_centers_, rtol=1e-12, atol=1e-12)
+    # scikit-learn re-labels against the final centres; the oracle's labels are the ones the
+    # final centres were computed from, so they must average to exactly those centres.
+    for j in range(7):
+        np.testing.assert_allclose(X[labels == j].astype(np.float64).mean(axis=0), C[j], rtol=1e-12, atol=1e-12)
+    assert counts.sum() == X.shape[0]
+    assert np.array_equal(counts, np.bincount(labels, minlength=7))
+
+
+def test_k_equals_one_gives_global_mean(oracle):
+    X, _ = _mixture(257, 12, 3, 0.5, 3)
+    C, labels, counts = oracle.lloyd(X, X[:1].astype(np.float64), 2)
+    np.testing.assert_allclose(C[0], X.astype(np.float64).mean(axis=0), rtol=1e-12, atol=1e-13)
+    assert (labels == 0).all() and counts[0] == 257
+
+
+def test_k_equals_n_from_the_points_has_zero_inertia(oracle):
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((9, 5)).astype(np.float32)
+    C, labels, counts = oracle.lloyd(X, X.astype(np.float64), 3)
+    assert np.array_equal(labels, np.arange(9)) and (counts == 1).all()
+    np.testing.assert_array_equal(C, X.astype(np.float64))
+
+
+def test_lloyd_inertia_is_non_increasing_and_reaches_a_fixed_point(oracle):
+    X, _ = _mixture(800, 8, 10, 0.6, 5)
+    C = X[:12].astype(np.float64)
+    prev = np.inf
+    labels = None
+    for _ in range(60):
+        labels, _, _ = oracle.assign(X, C)
+        inertia = ((X.astype(np.float64) - C[labels]) ** 2).sum()
+        assert inertia <= prev * (1 + 1e-12)
+        prev = inertia
+        C, _ = oracle.update(X, labels, C)
+    # fixed point: assignment is the argmin for every token, centroid is the mean of its members
+    D = ssd.cdist(X.astype(np.float64), C, "sqeuclidean")
+    assert np.array_equal(labels, np.argmin(D, axis=1))
+    for j in np.unique(labels):
+        np.testing.assert_allclose(C[j], X[labels == j].astype(np.float64).mean(0), rtol=1e-12, atol=1e-12)
+
+
+def test_update_keeps_empty_cluster_centroid(oracle):
+    X, _ = _mixture(100, 4, 2, 0.3, 6)
+    C0 = np.vstack([X[:2].astype(np.float64), np.full((1, 4), 1e3)])
+    labels = np.zeros(100, np.int32)
+    labels[50:] = 1
+    C, counts = oracle.update(X, labels, C0)
+    assert counts[2] == 0
+    np.testing.assert_array_equal(C[2], C0[2])
+
+
+def test_well_separated_mixture_recovers_component_means(oracle):
+    X, lab = _mixture(3000, 16, 5, 0.1, 7)
+    seeds, C0 = oracle.kmeanspp(X, 5, np.random.default_rng(8).random(5))
+    C, labels, counts = oracle.lloyd(X, C0, 10)
+    for c in range(5):
+        mu = X[lab == c].astype(np.float64).mean(0)
+        assert np.min(np.linalg.norm(C - mu, axis=1)) < 1e-9 + 0.1 * 4 / np.sqrt((lab == c).sum())
+
+
+# ---------------------------------------------------------------- k-means++ seeding (Method (1), section 4.3)
+
+def test_kmeanspp_first_seed_and_seeds_are_distinct_rows(oracle):
+    X, _ = _mixture(500, 8, 20, 0.3, 9)
+    u = np.random.default_rng(10).random(20)
+    seeds, C = oracle.kmeanspp(X, 20, u)
+    assert seeds[0] == int(np.floor(u[0] * 500))
+    assert len(set(seeds.tolist())) == 20
+    np.testing.assert_array_equal(C, X[seeds].astype(np.float64))
+
+
+def test_kmeanspp_second_seed_follows_d2_distribution(oracle):
+    """Over a uniform grid of u, the second seed's frequency is D^2(t) / sum D^2 (to 2^-32)."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((7, 3)).astype(np.float32)
+    M = 20000
+    grid = (np.arange(M) + 0.5) / M
+    counts = np.zeros(7)
+    for g in grid:
+        s, _ = oracle.kmeanspp(X, 2, np.array([0.0, g]))
+        counts[s[1]] += 1
+    D2 = ssd.cdist(X.astype(np.float64), X[:1].astype(np.float64), "sqeuclidean")[:, 0]
+    np.testing.assert_allclose(counts / M, D2 / D2.sum(), atol=2.0 / M)
+    assert counts[0] == 0                      # the first seed has D^2 = 0
+    # at the bottom edge (u = 0) the zero-weight first seed must still not be drawn again
+    s, _ = oracle.kmeanspp(X, 2, np.array([0.0, 0.0]))
+    assert s.tolist() == [0, 1]
+    s, _ = oracle.kmeanspp(X, 2, np.array([0.0, np.nextafter(1.0, 0.0)]))
+    assert s.tolist() == [0, 6]
+
+
+def test_kmeanspp_third_seed_uses_min_over_seeds(oracle):
+    rng = np.random.default_rng(12)
+    X = rng.standard_normal((6, 2)).astype(np.float32)
+    M = 20000
+    s2, _ = oracle.kmeanspp(X, 2, np.array([0.0, 0.6]))
+    counts = np.zeros(6)
+    for g in (np.arange(M) + 0.5) / M:
+        s, _ = oracle.kmeanspp(X, 3, np.array([0.0, 0.6, g]))
+        assert s[1] == s2[1]
+        counts[s[2]] += 1
+    D2 = ssd.cdist(X.astype(np.float64), X[s2].astype(np.float64), "sqeuclidean").min(axis=1)
+    np.testing.assert_allclose(counts / M, D2 / D2.sum(), atol=2.0 / M)
+
+
+def test_kmeanspp_all_points_equal_falls_back_to_uniform_index(oracle):
+    X = np.ones((10, 4), np.float32)
+    u = np.array([0.05, 0.55, 0.95])
+    seeds, _ = oracle.kmeanspp(X, 3, u)
+    assert seeds.tolist() == [0, 5, 9]
+
+
+# ---------------------------------------------------------------- scores and top-p (section 4.2, Eq. 1-2)
+
+def test_weights_are_size_weighted_centroid_softmax(oracle):
+    rng = np.random.default_rng(13)
+    cq = rng.standard_normal((9, 32)).astype(np.float32)
+    ck = rng.standard_normal((21, 32)).astype(np.float32)
+    count_k = rng.integers(0, 50, 21).astype(np.int32)
+    count_k[[3, 7]] = 0
+    scale = 1 / np.sqrt(32)
+    w = oracle.select_weights(cq, ck, count_k, scale).astype(np.float64)
+    logits = cq.astype(np.float64) @ ck.astype(np.float64).T * scale
+    nz = count_k > 0
+    ref = scipy.special.softmax(logits[:, nz] + np.log(count_k[nz]), axis=1)
+    np.testing.assert_allclose(w[:, nz] / w[:, nz].sum(1, keepdims=True), ref, rtol=1e-6)
+    assert (w[:, ~nz] == 0).all()
+    # the row maximum of the logits gets exp(0) = 1, so its weight equals its cluster size
+    jmax = np.argmax(np.where(nz, logits, -np.inf), axis=1)
+    np.testing.assert_array_equal(w[np.arange(9), jmax], count_k[jmax].astype(np.float64))
+
+
+def _fixed(w, count_k):
+    wmax = max(float(w[j]) for j in range(len(w)) if count_k[j] > 0)
+    return [int(np.floor(float(w[j]) / wmax * 2.0 ** 32)) if count_k[j] > 0 else 0 for j in range(len(w))]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topp_is_the_minimal_greedy_prefix_by_brute_force(oracle, seed):
+    rng = np.random.default_rng(100 + seed)
+    nK = 10
+    w = I.random_weights(4, nK, 200 + seed)
+    count_k = rng.integers(0, 5, nK).astype(np.int32)
+    count_k[0] = 3
+    for p in [1e-6, 0.3, 0.5, 0.8, 0.9, 0.95, 0.999999, 1.0]:
+        mask = oracle.topp(w, count_k, p)
+        for i in range(4):
+            kept = set(np.nonzero(mask[i])[0].tolist())
+            if p >= 1.0:
+                assert kept == set(np.nonzero(count_k)[0].tolist())
+                continue
+            u = _fixed(w[i], count_k)
+            T = int(np.ceil(float(np.float32(p)) * float(sum(u))))
+            assert sum(u[j] for j in kept) >= T
+            assert all(count_k[j] > 0 for j in kept)
+            eligible = [j for j in range(nK) if count_k[j] > 0]
+            best = min(len(S) for r in range(1, len(eligible) + 1)
+                       for S in itertools.combinations(eligible, r) if sum(u[j] for j in S) >= T)
+            assert len(kept) == best
+            # kept is a prefix of the order (u desc, index asc)
+            order = sorted(eligible, key=lambda j: (-u[j], j))
+            assert kept == set(order[:len(kept)])
+
+
+def test_topp_small_p_keeps_exactly_the_argmax_and_is_monotone(oracle):
+    w = I.random_weights(16, 40, 7)
+    count_k = np.ones(40, np.int32)
+    small = oracle.topp(w, count_k, 1e-9)
+    for i in range(16):
+        u = _fixed(w[i], count_k)
+        first = sorted(range(40), key=lambda j: (-u[j], j))[0]
+        assert np.nonzero(small[i])[0].tolist() == [first]
+    prev = small
+    for p in np.linspace(0.05, 1.0, 20):
+        cur = oracle.topp(w, count_k, p)
+        assert (cur >= prev).all()
+        prev = cur
+
+
+def test_topp_handworked_golden(oracle):
+    with open(os.path.join(GOLDEN, "topp_handworked.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        w = np.array([c["weights"]], np.float32)
+        mask = oracle.topp(w, np.array(c["counts"], np.int32), c["p"])
+        assert np.nonzero(mask[0])[0].tolist() == c["kept"], c["note"]
+
+
+# ---------------------------------------------------------------- permutation (Method (2), section 4.1)
+
+@pytest.mark.parametrize("n,k,empty", [(1, 1, 0.0), (1000, 37, 0.3), (4096, 256, 0.5), (5000, 3, 0.0)])
+def test_permute_is_numpy_stable_argsort(oracle, n, k, empty):
+    labels = I.random_labels(n, k, 5 + n, empty)
+    perm, offsets = oracle.permute(labels, k)
+    assert np.array_equal(perm, np.argsort(labels, kind="stable"))
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(np.bincount(labels, minlength=k))]))
+    assert offsets[-1] == n and np.array_equal(np.sort(perm), np.arange(n))
+
+
+def test_unpermute_inverts_the_gather(oracle):
+    rng = np.random.default_rng(14)
+    X = rng.standard_normal((333, 16)).astype(np.float32)
+    labels = I.random_labels(333, 20, 15, 0.2)
+    perm, _ = oracle.permute(labels, 20)
+    Xp = oracle.gather_rows(X, perm)
+    np.testing.assert_array_equal(oracle.unpermute(Xp.astype(np.float64), perm), X.astype(np.float64))
+
+
+# ---------------------------------------------------------------- attention (Method (4), section 4.3)
+
+def _sdpa64(q, k, v, scale, mask=None):
+    q, k, v = (torch.from_numpy(np.asarray(a, np.float64))[None, None] for a in (q, k, v))
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)[0, 0].numpy()
+
+
+def test_sparse_attention_matches_sdpa_with_token_mask(oracle):
+    rng = np.random.default_rng(16)
+    N, d, nQ, nK = 700, 32, 9, 13
+    lq = I.random_labels(N, nQ, 17, 0.2)
+    lk = I.random_labels(N, nK, 18, 0.2)
+    q_off = np.concatenate([[0], np.cumsum(np.bincount(lq, minlength=nQ))]).astype(np.int32)
+    k_off = np.concatenate([[0], np.cumsum(np.bincount(lk, minlength=nK))]).astype(np.int32)
+    Qp = rng.standard_normal((N, d)).astype(np.float32)
+    Kp = rng.standard_normal((N, d)).astype(np.float32)
+    Vp = rng.standard_normal((N, d)).astype(np.float32)
+    mask = (rng.random((nQ, nK)) < 0.4).astype(np.uint8)
+    count_k = np.diff(k_off)
+    for i in range(nQ):
+        if not (mask[i] * (count_k > 0)).any():
+            mask[i, int(np.argmax(count_k))] = 1
+    scale = 1 / np.sqrt(d)
+    out = oracle.sparse_attention_rows(Qp, Kp, Vp, q_off, k_off, mask, scale)
+    cq = np.repeat(np.arange(nQ), np.diff(q_off))
+    ck = np.repeat(np.arange(nK), np.diff(k_off))
+    tok = mask[cq][:, ck].astype(bool)
+    np.testing.assert_allclose(out, _sdpa64(Qp, Kp, Vp, scale, tok), rtol=1e-10, atol=1e-12)
+
+
+def test_dense_attention_matches_sdpa(oracle):
+    rng = np.random.default_rng(19)
+    Q, K, V = (rng.standard_normal((300, 64)).astype(np.float32) for _ in range(3))
+    out = oracle.dense_attention_rows(Q, K, V, 0.125)
+    np.testing.assert_allclose(out, _sdpa64(Q, K, V, 0.125), rtol=1e-10, atol=1e-12)
+
+
+def test_top_p_one_layer_equals_dense_attention(oracle):
+    """With every cluster pair kept, the permutation cancels (section 4.1): output == dense."""
+    cfg = I.CONFIGS["tiny"]
+    hi = I.head_inputs(cfg, 0, 0)
+    q, k, v = hi["q"][:1024], hi["k"][:1024], hi["v"][:1024]
+    out = oracle.layer_head(q, k, v, 8, 16, 3, 1.0, cfg.scale, hi["uq"][:8], hi["uk"][:16])
+    assert out["mask"][:, out["count_k"] > 0].all()
+    dense = oracle.dense_attention_rows(q, k, v, cfg.scale)
+    np.testing.assert_allclose(out["o"], dense, rtol=1e-9, atol=1e-12)
+
+
+def test_single_key_cluster_outputs_that_value_row(oracle):
+    rng = np.random.default_rng(20)
+    N, d = 50, 16
+    q_off = np.array([0, 20, 50], np.int32)
+    k_off = np.array([0, 1, 50], np.int32)           # K cluster 0 holds a single key
+    Qp, Kp, Vp = (rng.standard_normal((N, d)).astype(np.float32) for _ in range(3))
+    mask = np.array([[1, 0], [1, 1]], np.uint8)
+    out = oracle.sparse_attention_rows(Qp, Kp, Vp, q_off, k_off, mask, 0.25)
+    np.testing.assert_array_equal(out[:20], np.broadcast_to(Vp[0].astype(np.float64), (20, d)))
+
+
+def test_density_of_full_mask_is_one(oracle):
+    count_q = np.array([3, 0, 5], np.int32)
+    count_k = np.array([2, 6], np.int32)
+    assert oracle.density(np.ones((3, 2), np.uint8), count_q, count_k) == 1.0
+    assert oracle.density(np.array([[1, 0], [1, 1], [0, 1]], np.uint8), count_q, count_k) == (3 * 2 + 5 * 6) / 64
