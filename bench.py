@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of one SVG2 attention layer on B200.
+
+One step = the whole hot path over one synthetic layer: k-means on Q and on K (k-means++ seeding
+plus Lloyd iterations), centroid scoring and top-p selection, permutation of Q, K, V, and the
+variable-block-size sparse attention with the inverse permutation fused into its epilogue, all
+through the C ABI of libsvg2.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan720p] [--top-p 0.9]
+  python bench.py --impl reference ...     # the CPU oracle, timed on a bounded sample
+
+With N > 1 (torchrun), every rank runs its own layer (replicas, weak scaling: the layer's heads
+are independent and there is no exchange on the path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_video_head_b200 import inputs as I  # noqa: E402
+
+METRIC = "per-layer SVG2 attention ms and sparse-attn TFLOP/s vs BF16 peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="svg2", choices=["svg2", "reference"])
+    ap.add_argument("--config", default="wan720p", choices=sorted(I.CONFIGS))
+    ap.add_argument("--top-p", type=float, default=0.9)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16": j["bf16_tflops"], "bf16_sustained": j["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def gen_inputs(cfg, step=0):
+    import multiprocessing as mp
+    procs = max(1, min(cfg.H, len(os.sched_getaffinity(0))))
+    if procs == 1:
+        return I.layer_inputs(cfg, step)
+    with mp.get_context("spawn").Pool(procs) as pool:
+        parts = pool.starmap(I.head_inputs, [(cfg, 0, h, step) for h in range(cfg.H)])
+    return {k: np.stack([p[k] for p in parts])[None] for k in parts[0]}
+
+
+# ------------------------------------------------------------------------------------------ oracle
+def oracle_sample(cfg, top_p, rows=96, head=0):
+    """The CPU oracle on a bounded sample of the layer: one head's k-means (Q and K), selection and
+    permutation in full, and attention for `rows` query rows; extrapolated to the whole layer."""
+    from oracle import oracle as O
+    hi = I.head_inputs(cfg, 0, head)
+    scale = float(np.float32(cfg.scale))
+    t0 = time.perf_counter()
+    cq, lq, count_q = O.kmeans(hi["q"], cfg.nQ, cfg.iters, hi["uq"])
+    t1 = time.perf_counter()
+    ck, lk, count_k = O.kmeans(hi["k"], cfg.nK, cfg.iters, hi["uk"])
+    t2 = time.perf_counter()
+    w = O.select_weights(cq.astype(np.float32), ck.astype(np.float32), count_k, scale)
+    mask = O.topp(w, count_k, top_p)
+    pq, qo = O.permute(lq, cfg.nQ)
+    pk, ko = O.permute(lk, cfg.nK)
+    Qp, Kp, Vp = O.gather_rows(hi["q"], pq), O.gather_rows(hi["k"], pk), O.gather_rows(hi["v"], pk)
+    t3 = time.perf_counter()
+    sel = np.random.default_rng(1).choice(cfg.N, rows, replace=False)
+    O.sparse_attention_rows(Qp, Kp, Vp, qo, ko, mask, scale, sel)
+    t4 = time.perf_counter()
+    per_head = (t1 - t0) + (t2 - t1) + (t3 - t2) + (t4 - t3) * cfg.N / rows
+    return per_head * cfg.H * 1e3, {"kmeans_q_s": t1 - t0, "kmeans_k_s": t2 - t1, "select_permute_s": t3 - t2,
+                                     "attn_rows_s": t4 - t3, "wall_s": t4 - t0}
+
+
+def run_reference(args, cfg):
+    cores = len(os.sched_getaffinity(0))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, args.top_p, rows=16)
+    vals = []
+    for _ in range(args.steps):
+        v, _ = oracle_sample(cfg, args.top_p)
+        vals.append(v)
+    value = statistics.median(vals)
+    sample = (f"one head of {cfg.H}: full k-means++ + {cfg.iters} Lloyd iterations on Q and K, selection, "
+              f"permutation, and attention for 96 of {cfg.N} query rows; extrapolated x{cfg.N}/96 rows, x{cfg.H} heads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "ms", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(cfg, args.top_p),
+            "cpu_baseline": {"value": value, "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(cfg, top_p):
+    return {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "grid": list(cfg.grid), "d": cfg.d,
+            "nQ": cfg.nQ, "nK": cfg.nK, "iters": cfg.iters, "init": "kmeans++", "top_p": top_p,
+            "components": cfg.components, "sigma": cfg.sigma,
+            "l2": "inputs larger than L2 (each of Q, K, V is %.0f MB)" % (cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6),
+            "parallelism": "replicas"}
+
+
+# ------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.proc = None
+        self.index = index
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ GPU arm
+def main():
+    args = parse()
+    cfg = I.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, cfg)
+        return
+    data = gen_inputs(cfg)  # before CUDA initialisation
+
+    import torch
+    import torch.distributed as dist
+    from sparse_attention_video_head_b200 import svg2
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    P = peaks()
+    B, H, N, d = 1, cfg.H, cfg.N, cfg.d
+    BH = B * H
+    scale = float(np.float32(cfg.scale))
+    Q = torch.from_numpy(data["q"]).to(torch.bfloat16).to(dev)
+    K = torch.from_numpy(data["k"]).to(torch.bfloat16).to(dev)
+    V = torch.from_numpy(data["v"]).to(torch.bfloat16).to(dev)
+    uq = torch.from_numpy(data["uq"]).to(dev)
+    uk = torch.from_numpy(data["uk"]).to(dev)
+    cq = torch.zeros(B, H, cfg.nQ, d, device=dev)
+    ck = torch.zeros(B, H, cfg.nK, d, device=dev)
+    O = torch.empty_like(Q)
+    outs = svg2.layer_output_buffers(B, H, N, cfg.nQ, cfg.nK, device=dev)
+    ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK, device=dev)
+    Qp, Kp, Vp = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    i32 = dict(dtype=torch.int32, device=dev)
+    lab_q, lab_k = torch.empty(B, H, N, **i32), torch.empty(B, H, N, **i32)
+    cnt_q, cnt_k = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nK, **i32)
+    perm_q, perm_k = torch.empty(B, H, N, **i32), torch.empty(B, H, N, **i32)
+    q_off, k_off = torch.empty(B, H, cfg.nQ + 1, **i32), torch.empty(B, H, cfg.nK + 1, **i32)
+    mask = torch.empty(B, H, cfg.nQ, cfg.nK, dtype=torch.uint8, device=dev)
+    sel_count, sel_idx = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nQ, cfg.nK, **i32)
+    stream_len = torch.empty(B, H, cfg.nQ, **i32)
+    KPP = svg2.SVG2_INIT_KMEANSPP
+    stream = torch.cuda.current_stream(dev)
+    names = ["kmeans_q", "kmeans_k", "select", "permute", "sparse_attn"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        svg2.svg2_kmeans(Q, cfg.nQ, cfg.iters, KPP, cq, lab_q, cnt_q, ws, u=uq, perm=perm_q, offsets=q_off)
+        mark(1)
+        svg2.svg2_kmeans(K, cfg.nK, cfg.iters, KPP, ck, lab_k, cnt_k, ws, u=uk, perm=perm_k, offsets=k_off)
+        mark(2)
+        svg2.svg2_select(cq, ck, cnt_k, args.top_p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
+        mark(3)
+        svg2.svg2_gather(Q, perm_q, Qp)
+        svg2.svg2_gather(K, perm_k, Kp)
+        svg2.svg2_gather(V, perm_k, Vp)
+        mark(4)
+        svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
+        mark(5)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    svg2.raise_on_device_error(ws)
+
+    # algorithmic work of the attention (actual = kept pairs only, no padding)
+    cq_h = cnt_q.cpu().numpy().astype(np.float64)
+    sl_h = stream_len.cpu().numpy().astype(np.float64)
+    actual_flops = 4.0 * d * float((cq_h * sl_h).sum())
+    dense_flops = 4.0 * d * N * N * BH
+    density = actual_flops / dense_flops
+    tiles_q = np.ceil(cq_h / 128.0)
+    executed_flops = 4.0 * d * float((tiles_q * 128.0 * np.ceil(sl_h / 128.0) * 128.0).sum())
+    waste128 = fixed128_waste(q_off.cpu().numpy(), k_off.cpu().numpy(), mask.cpu().numpy(), heads=range(min(4, H)))
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    svg2.raise_on_device_error(ws)
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
+    attn_ms = stage_ms["sparse_attn"]
+    achieved_tflops = actual_flops / (attn_ms * 1e-3) / 1e12
+
+    # the same layer through the single public call with host buffers (copies inside the timed region)
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist)
+
+    dense_ms = None
+    if not args.no_dense and rank == 0:
+        dense_ms = time_dense(torch, Q, K, V, scale)
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v, parts = oracle_sample(cfg, args.top_p)
+        cpu = {"value": v, "unit": "ms", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": (f"one head of {cfg.H}: full k-means (Q and K), selection, permutation, attention for 96 "
+                          f"of {cfg.N} rows; extrapolated to the layer"), "parts_s": parts}
+    launches = kernel_launches(cfg)
+    line = {
+        "metric": METRIC, "value": ms_per_step / world, "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.top_p),
+        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel", "achieved": achieved_tflops,
+                     "peak": P["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved_tflops / P["bf16_sustained"],
+                     "peak_source": P["source"] + " bf16 cuBLAS, sustained (kernel timed inside a long step)",
+                     "traffic": None},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(), "stages_ms": stage_ms, "density": density,
+        "attn_tflop_actual": actual_flops / 1e12, "attn_tflop_dense_equiv": dense_flops / 1e12,
+        "attn_tflops_effective": dense_flops / (attn_ms * 1e-3) / 1e12,
+        "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
+        "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
+        "dense_sdpa_ms": dense_ms,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
+    B, H, N, d = 1, cfg.H, cfg.N, cfg.d
+    hq = torch.from_numpy(data["q"]).to(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(data["k"]).to(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(data["v"]).to(torch.bfloat16).pin_memory()
+    huq = torch.from_numpy(data["uq"]).pin_memory()
+    huk = torch.from_numpy(data["uk"]).pin_memory()
+    ho = torch.empty(B, H, N, d, dtype=torch.bfloat16).pin_memory()
+    Q = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    K, V, O = torch.empty_like(Q), torch.empty_like(Q), torch.empty_like(Q)
+    uq = torch.empty(huq.shape, dtype=torch.float64, device=dev)
+    uk = torch.empty(huk.shape, dtype=torch.float64, device=dev)
+    cq = torch.zeros(B, H, cfg.nQ, d, device=dev)
+    ck = torch.zeros(B, H, cfg.nK, d, device=dev)
+    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, args.top_p, float(np.float32(cfg.scale)), 1)
+
+    def one():
+        Q.copy_(hq, non_blocking=True)
+        K.copy_(hk, non_blocking=True)
+        V.copy_(hv, non_blocking=True)
+        uq.copy_(huq, non_blocking=True)
+        uk.copy_(huk, non_blocking=True)
+        svg2.svg2_layer(Q, K, V, prm, cq, ck, O, ws, uq, uk)
+        ho.copy_(O, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 5))
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize(dev)
+    svg2.raise_on_device_error(ws)
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = 3 * hq.numel() * 2 + (huq.numel() + huk.numel()) * 8
+    return {"value": ms / world, "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
+            "steps": steps, "api": "svg2_layer"}
+
+
+def time_dense(torch, Q, K, V, scale, reps=3):
+    try:
+        f = torch.nn.functional.scaled_dot_product_attention
+        f(Q, K, V, scale=scale)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            f(Q, K, V, scale=scale)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+    except Exception as e:  # library baseline only; never part of the product path
+        return f"unavailable: {type(e).__name__}"
+
+
+def fixed128_waste(q_off, k_off, mask, heads):
+    """Fraction of a fixed 128x128 block-sparse kernel's work that would be padding for the same
+    kept cluster pairs (the pages' Fig. 7(b) comparison)."""
+    act, fixed = 0.0, 0.0
+    for h in heads:
+        qo, ko, m = q_off[0, h], k_off[0, h], mask[0, h]
+        nQ, nK = m.shape
+        nb_q = (qo[-1] + 127) // 128
+        nb_k = (ko[-1] + 127) // 128
+        blocks = np.zeros((nb_q, nb_k), bool)
+        for i in range(nQ):
+            if qo[i + 1] == qo[i]:
+                continue
+            js = np.nonzero(m[i])[0]
+            rq = slice(qo[i] // 128, (qo[i + 1] - 1) // 128 + 1)
+            for j in js:
+                if ko[j + 1] == ko[j]:
+                    continue
+                blocks[rq, ko[j] // 128:(ko[j + 1] - 1) // 128 + 1] = True
+                act += float(qo[i + 1] - qo[i]) * float(ko[j + 1] - ko[j])
+        fixed += float(blocks.sum()) * 128.0 * 128.0
+    return 1.0 - act / fixed if fixed > 0 else None
+
+
+def kernel_launches(cfg):
+    per_role = 1 + 1 + cfg.iters * (1 + 3 + 1)   # k-means++, split prep, per iteration: assign, 3 sort, update
+    return 2 * per_role + 1 + 3 + 4               # select, 3 gathers, plan (3) + attention
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+/*
+ * libsvg2 — SVG2 semantic-aware permuted sparse attention for one DiT attention layer,
+ * hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via Semantic-Aware
+ * Permutation" (wiki summary page, sections Key claims and Method; paper sections 4.1-4.3).
+ * Per (batch, head) the layer clusters Q and K with k-means (Method (1)), scores cluster pairs
+ * from centroids and keeps K clusters per Q cluster by top-p (Method (3); section 4.2, Eq. 1-2),
+ * permutes Q, K, V into cluster-contiguous order (Method (2); section 4.1), runs attention over
+ * the kept variable-size blocks only (Method (4); section 4.3, Fig. 7(b)) and scatters the output
+ * rows back to token order (Method (2), "final inverse-permutation of the rows").
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the caller owns all
+ *     memory.  The library never allocates device memory: scratch comes from the caller's
+ *     workspace `ws` of `ws_bytes` bytes (size from svg2_workspace_size), 256-byte aligned.
+ *   - Tensors are contiguous row-major [B, H, N, d] (d innermost); per-head vectors are
+ *     [B, H, n].  d is 64 or 128.  bf16 tensors hold raw bfloat16 values.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous on it:
+ *     arguments are validated on the host first and a bad one returns an error before any launch;
+ *     a failed launch returns SVG2_ERR_CUDA.  Device-side errors (a bounded wait that ran out,
+ *     an out-of-range label) are latched in a status word at the start of `ws` and read with
+ *     svg2_check_status.  No kernel traps or waits without a bound.
+ *   - The library keeps no global state, is reentrant, and never lets a C++ exception cross the
+ *     C boundary.  Return values are svg2_status codes.
+ */
+#ifndef SVG2_H_
+#define SVG2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVG2_API __attribute__((visibility("default")))
+#else
+#define SVG2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVG2_OK = 0,
+  SVG2_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, bad enum value */
+  SVG2_ERR_UNSUPPORTED = 2,   /* d / dtype / cluster count this build does not handle */
+  SVG2_ERR_WORKSPACE = 3,     /* ws too small or misaligned */
+  SVG2_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
+  SVG2_ERR_DEVICE_TIMEOUT = 5,/* a bounded device wait ran out (read via svg2_check_status) */
+  SVG2_ERR_DEVICE_BOUNDS = 6  /* a device index check failed, e.g. a label >= k */
+} svg2_status;
+
+typedef enum { SVG2_BF16 = 0, SVG2_F32 = 1 } svg2_dtype;
+
+/* k-means initialisation.  GIVEN: start from the centroids already in the `centroids` buffer —
+ * this is also the warm start of the pages' centroid cache (section 4.3, Fig. 7(a)): pass the
+ * previous denoising step's centroids.  KMEANSPP: k-means++ seeding from the data (Method (1)). */
+typedef enum { SVG2_INIT_GIVEN = 0, SVG2_INIT_KMEANSPP = 1 } svg2_init;
+
+/* Largest supported sizes of this build. */
+#define SVG2_MAX_CLUSTERS 1024
+#define SVG2_MAX_TOKENS (1 << 24)
+
+/* Human-readable name of a status code (static string, never NULL). */
+SVG2_API const char* svg2_status_string(int status);
+
+/* Bytes of workspace that svg2_layer needs for these sizes; every other entry point needs at
+ * most this much for the same sizes.  Returns SVG2_ERR_INVALID_ARG / UNSUPPORTED on bad sizes. */
+SVG2_API int svg2_workspace_size(int B, int H, int N, int d, int nQ, int nK, size_t* bytes);
+
+/* Reads and clears the device status word in `ws` after synchronising `stream`.
+ * *device_status receives the latched svg2_status (SVG2_OK if none); where/info (optional, may be
+ * NULL) receive a kernel tag and two integers for diagnostics. */
+SVG2_API int svg2_check_status(void* ws, void* stream, int* device_status, uint32_t* where, uint32_t* info);
+
+/*
+ * Batched k-means (Method (1); Key claims section 4.1 and 4.3) on X [B, H, N, d] per (b, h):
+ * `iters` >= 1 Lloyd iterations — assignment label_t = argmin_c ||x_t - c||^2 (ties to the lower
+ * c) as a tensor-core distance GEMM fused with the argmin, then c_j = mean of its members (an empty
+ * cluster keeps its centroid) as a segmented sum divided by the count.
+ *   X          bf16 or f32 per `dtype`.
+ *   init       SVG2_INIT_GIVEN (centroids holds the start, e.g. the previous step's cache) or
+ *              SVG2_INIT_KMEANSPP (seeding from the data; `u` must then hold B*H*k uniforms in
+ *              [0,1), float64, one per seed, and seeds are chosen by fixed-point D^2 sampling).
+ *   centroids  float32 [B, H, k, d], in (GIVEN) and out (final centroids).
+ *   labels     int32 [B, H, N], out: labels of the last assignment (the ones the final centroids
+ *              were computed from).
+ *   counts     int32 [B, H, k], out: cluster sizes under those labels.
+ *   perm       int32 [B, H, N], out (optional, may be NULL): stable sort of the token indices by
+ *              label, perm[j] = token at permuted row j.
+ *   offsets    int32 [B, H, k+1], out (optional): exclusive scan of counts.
+ * 1 <= k <= min(N, SVG2_MAX_CLUSTERS). */
+SVG2_API int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int iters, int init,
+                const double* u, float* centroids, int32_t* labels, int32_t* counts, int32_t* perm,
+                int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Critical-cluster selection (section 4.2, Eq. 1-2; Method (3)).  Per (b, h, Q-cluster i):
+ * l_ij = (cq_i . ck_j) * scale, w_ij = count_k[j] * exp(l_ij - max_j l_ij) over non-empty j
+ * (w = 0 for empty j), then top-p: the shortest prefix of the K clusters ordered by (w desc, j asc)
+ * whose weight reaches p of the row total, in fixed point: u_j = floor(w_j / max w * 2^32),
+ * T = ceil(p * sum u), keep until the running sum >= T.  top_p >= 1 keeps every non-empty cluster.
+ *   cq float32 [B,H,nQ,d]; ck float32 [B,H,nK,d]; count_k int32 [B,H,nK].
+ *   weights   float32 [B,H,nQ,nK], out (optional, may be NULL).
+ *   mask      uint8 [B,H,nQ,nK], out: 1 where the pair is kept.
+ *   sel_count int32 [B,H,nQ], out: number of kept K clusters per Q cluster.
+ *   sel_idx   int32 [B,H,nQ,nK], out: the kept K-cluster indices in ascending order in the first
+ *             sel_count entries of each row (rest unspecified).
+ *   stream_len int32 [B,H,nQ], out (optional): number of keys kept per Q cluster.
+ * nQ, nK in [1, SVG2_MAX_CLUSTERS]; 0 < top_p. */
+SVG2_API int svg2_select(const float* cq, const float* ck, const int32_t* count_k, int B, int H, int nQ, int nK,
+                int d, float top_p, float scale, float* weights, uint8_t* mask, int32_t* sel_count,
+                int32_t* sel_idx, int32_t* stream_len, void* ws, size_t ws_bytes, void* stream);
+
+/* The top-p step of svg2_select alone, on given float32 weights [B,H,nQ,nK] (same outputs). */
+SVG2_API int svg2_select_from_weights(const float* weights, const int32_t* count_k, int B, int H, int nQ, int nK,
+                             float top_p, uint8_t* mask, int32_t* sel_count, int32_t* sel_idx,
+                             int32_t* stream_len, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Stable counting sort of labels (Method (2)): per (b,h), counts [k], offsets [k+1] (exclusive
+ * scan) and perm [N] with perm[j] = original token of permuted row j, in (label asc, token asc).
+ * labels int32 [B,H,N] in [0,k) (a label out of range latches SVG2_ERR_DEVICE_BOUNDS). */
+SVG2_API int svg2_sort(const int32_t* labels, int B, int H, int N, int k, int32_t* perm, int32_t* offsets,
+              int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/* Row gather applying a permutation (Method (2)): Xp[b,h,j,:] = X[b,h,perm[b,h,j],:].
+ * X bf16 or f32 per dtype; Xp is always bf16 (f32 input is rounded to nearest even). */
+SVG2_API int svg2_gather(const void* X, int dtype, const int32_t* perm, int B, int H, int N, int d, void* Xp,
+                void* stream);
+
+/* svg2_sort of `labels` followed by svg2_gather of X: cluster-contiguous bf16 Xp. */
+SVG2_API int svg2_permute(const void* X, int dtype, const int32_t* labels, int B, int H, int N, int d, int k,
+                 void* Xp, int32_t* perm, int32_t* offsets, int32_t* counts, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/*
+ * Variable-block-size sparse attention (Method (4); section 4.3, Fig. 7(b)) on permuted bf16
+ * Qp, Kp, Vp [B,H,N,d] (d = 128): a query row of Q cluster i (rows [q_off[i], q_off[i+1]))
+ * attends, with one softmax, to the keys of every kept K cluster j (rows [k_off[j], k_off[j+1]))
+ * listed in sel_idx[i][0..sel_count[i]).  Online softmax on tcgen05/TMEM tiles; the kept
+ * clusters are gathered into one packed key stream, so ragged cluster edges cost no padding.
+ *   q_off int32 [B,H,nQ+1]; k_off int32 [B,H,nK+1]; sel_count/sel_idx as from svg2_select.
+ *   perm_q   optional int32 [B,H,N]: if given, output row r is written to token perm_q[r]
+ *            (the inverse permutation fused into the epilogue); if NULL, O is in permuted order.
+ *   O        bf16 [B,H,N,d], out.  scale multiplies q.k (usually 1/sqrt(d)). */
+SVG2_API int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
+                     const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int B, int H,
+                     int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Inverse permutation of output rows (Method (2)): O[b,h,perm[b,h,j],:] = Op[b,h,j,:], bf16. */
+SVG2_API int svg2_unpermute(const void* Op, const int32_t* perm, int B, int H, int N, int d, void* O, void* stream);
+
+/* Parameters of one layer call. */
+typedef struct {
+  int nQ, nK;          /* clusters for Q and for K */
+  int iters;           /* Lloyd iterations per call (>= 1) */
+  int init;            /* svg2_init: GIVEN = warm start from cq/ck, KMEANSPP = cold start */
+  float top_p;         /* (0, 1]; >= 1 keeps every pair */
+  float scale;         /* softmax scale, usually 1/sqrt(d) */
+  int fuse_unpermute;  /* 1: write O in token order from the attention epilogue (default path);
+                          0: write permuted rows, then run svg2_unpermute */
+} svg2_params;
+
+/* Optional device buffers for the layer's intermediate results.  Any NULL field is kept inside
+ * the workspace instead.  Shapes as in the per-stage calls above. */
+typedef struct {
+  int32_t *labels_q, *labels_k, *count_q, *count_k, *perm_q, *perm_k, *q_off, *k_off;
+  float* weights;
+  uint8_t* mask;
+  int32_t *sel_count, *sel_idx, *stream_len;
+} svg2_layer_outputs;
+
+/*
+ * One SVG2 attention layer (Method (1)-(4)): k-means on Q (nQ) and on K (nK), selection, permute,
+ * sparse attention and inverse permutation, all enqueued on `stream` with no host synchronisation.
+ *   Q, K, V   [B,H,N,d] bf16 or f32 (dtype), d = 128 for the tensor-core attention.
+ *   uq, uk    float64 uniforms [B,H,nQ] / [B,H,nK] for k-means++ (ignored for GIVEN; may be NULL).
+ *   cq, ck    float32 centroid caches [B,H,nQ,d] / [B,H,nK,d]: in for GIVEN (warm start), out always.
+ *   O         bf16 [B,H,N,d], out, in token order.
+ *   outs      optional (may be NULL), see svg2_layer_outputs. */
+SVG2_API int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, int H, int N, int d,
+               const svg2_params* params, const double* uq, const double* uk, float* cq, float* ck, void* O,
+               const svg2_layer_outputs* outs, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Self-test of the tensor-core building blocks (not part of the method): C = A * B^T for
+ * bf16 A [128, 128] and B [n, 128] (n in {64, 128, 256}), loaded by TMA with 128-byte swizzle,
+ * multiplied by tcgen05.mma into TMEM (float32); then P = bf16(C[:, :128]) is written back to
+ * TMEM and multiplied by V [128, 128] (bf16, row-major: keys x d) from shared memory as
+ * O = P * V, exercising the TMEM-operand form used by the attention.  Outputs C float32
+ * [128, n] and O float32 [128, 128].  ws holds the status word. */
+SVG2_API int svg2_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O, void* ws,
+                      size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVG2_H_ */

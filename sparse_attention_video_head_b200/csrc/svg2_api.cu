@@ -1,0 +1,395 @@
+// C-ABI entry points of libsvg2 (declared in include/svg2.h): argument validation, workspace
+// carving, tensor-map encoding and the launch sequence of each stage and of the whole layer.
+// Host code only; every step of the method runs in the kernels of the other .cu files.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <new>
+
+#include "svg2.h"
+#include "svg2_internal.h"
+
+namespace svg2 {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? SVG2_OK : SVG2_ERR_CUDA; }
+
+bool valid_dtype(int dt) { return dt == SVG2_BF16 || dt == SVG2_F32; }
+
+// Sizes shared by all stages.
+int check_sizes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return SVG2_ERR_INVALID_ARG;
+  if (N > SVG2_MAX_TOKENS) return SVG2_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > (1 << 20)) return SVG2_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return SVG2_ERR_UNSUPPORTED;
+  return SVG2_OK;
+}
+
+int check_k(int k, int N) {
+  if (k < 1 || k > N) return SVG2_ERR_INVALID_ARG;
+  if (k > SVG2_MAX_CLUSTERS) return SVG2_ERR_UNSUPPORTED;
+  return SVG2_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr) return SVG2_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return SVG2_ERR_WORKSPACE;
+  if (ws_bytes < need) return SVG2_ERR_WORKSPACE;
+  return SVG2_OK;
+}
+
+struct LayerCarve {
+  DeviceStatus* st;
+  KmeansScratch kq, kk;
+  int32_t *labels_q, *labels_k, *count_q, *count_k, *perm_q, *perm_k, *q_off, *k_off;
+  float* weights;
+  uint8_t* mask;
+  int32_t *sel_count, *sel_idx, *stream_len;
+  void *Qp, *Kp, *Vp, *Op;
+  AttnScratch attn;
+};
+
+void carve_layer(Carve& c, int BH, int N, int d, int nQ, int nK, const svg2_layer_outputs* o, LayerCarve& L) {
+  L.st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+  carve_kmeans(c, BH, N, d, nQ, L.kq, false);
+  carve_kmeans(c, BH, N, d, nK, L.kk, false);
+  auto pick = [&](int32_t* user, size_t n) { return user != nullptr ? user : c.take<int32_t>(n); };
+  const size_t BHN = static_cast<size_t>(BH) * N;
+  L.labels_q = pick(o ? o->labels_q : nullptr, BHN);
+  L.labels_k = pick(o ? o->labels_k : nullptr, BHN);
+  L.count_q = pick(o ? o->count_q : nullptr, static_cast<size_t>(BH) * nQ);
+  L.count_k = pick(o ? o->count_k : nullptr, static_cast<size_t>(BH) * nK);
+  L.perm_q = pick(o ? o->perm_q : nullptr, BHN);
+  L.perm_k = pick(o ? o->perm_k : nullptr, BHN);
+  L.q_off = pick(o ? o->q_off : nullptr, static_cast<size_t>(BH) * (nQ + 1));
+  L.k_off = pick(o ? o->k_off : nullptr, static_cast<size_t>(BH) * (nK + 1));
+  L.weights = o ? o->weights : nullptr;  // optional output only
+  L.mask = (o && o->mask) ? o->mask : c.take<uint8_t>(static_cast<size_t>(BH) * nQ * nK);
+  L.sel_count = pick(o ? o->sel_count : nullptr, static_cast<size_t>(BH) * nQ);
+  L.sel_idx = pick(o ? o->sel_idx : nullptr, static_cast<size_t>(BH) * nQ * nK);
+  L.stream_len = pick(o ? o->stream_len : nullptr, static_cast<size_t>(BH) * nQ);
+  L.Qp = c.take<uint16_t>(BHN * d);
+  L.Kp = c.take<uint16_t>(BHN * d);
+  L.Vp = c.take<uint16_t>(BHN * d);
+  L.Op = c.take<uint16_t>(BHN * d);
+  carve_attn(c, BH, N, nQ, L.attn);
+}
+
+cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int iters, int init, const double* u,
+                       float* C, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets,
+                       const KmeansScratch& s, DeviceStatus* st, cudaStream_t stream) {
+  cudaError_t e = cudaSuccess;
+  if (init == SVG2_INIT_KMEANSPP) e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, stream);
+  if (e == cudaSuccess) e = launch_centroid_prep(C, BH, k, d, s.c_hi, s.c_lo, s.c_norm, stream);
+  for (int it = 0; it < iters && e == cudaSuccess; ++it) {
+    e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, st, stream);
+    if (e == cudaSuccess) e = launch_sort(labels, BH, N, k, perm, offsets, counts, s.chunk_hist, st, stream);
+    if (e == cudaSuccess) e = launch_update(X, f32, BH, N, d, k, perm, offsets, C, s.c_hi, s.c_lo, s.c_norm, stream);
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t make_tmap_bf16_rows(void* map, const void* base, uint64_t rows, uint32_t d, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  if (!aligned(base, 16) || rows == 0 || box_rows == 0 || box_rows > 256) return cudaErrorInvalidValue;
+  const cuuint64_t dims[2] = {d, rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                        dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace svg2
+
+using namespace svg2;
+
+extern "C" {
+
+const char* svg2_status_string(int status) {
+  switch (status) {
+    case SVG2_OK: return "SVG2_OK";
+    case SVG2_ERR_INVALID_ARG: return "SVG2_ERR_INVALID_ARG: invalid argument";
+    case SVG2_ERR_UNSUPPORTED: return "SVG2_ERR_UNSUPPORTED: size or type not supported by this build";
+    case SVG2_ERR_WORKSPACE: return "SVG2_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case SVG2_ERR_CUDA: return "SVG2_ERR_CUDA: a CUDA call failed";
+    case SVG2_ERR_DEVICE_TIMEOUT: return "SVG2_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+    case SVG2_ERR_DEVICE_BOUNDS: return "SVG2_ERR_DEVICE_BOUNDS: a device index check failed";
+    default: return "SVG2: unknown status";
+  }
+}
+
+int svg2_workspace_size(int B, int H, int N, int d, int nQ, int nK, size_t* bytes) {
+  if (bytes == nullptr) return SVG2_ERR_INVALID_ARG;
+  int r = check_sizes(B, H, N, d);
+  if (r == SVG2_OK) r = check_k(nQ, N);
+  if (r == SVG2_OK) r = check_k(nK, N);
+  if (r != SVG2_OK) return r;
+  Carve c(nullptr);
+  LayerCarve L;
+  carve_layer(c, B * H, N, d, nQ, nK, nullptr, L);
+  *bytes = align_up(c.off, 256);
+  return SVG2_OK;
+}
+
+int svg2_check_status(void* ws, void* stream, int* device_status, uint32_t* where, uint32_t* info) {
+  if (ws == nullptr || device_status == nullptr) return SVG2_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceStatus h{};
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return SVG2_ERR_CUDA;
+  *device_status = static_cast<int>(h.code);
+  if (where) *where = h.where;
+  if (info) {
+    info[0] = h.info0;
+    info[1] = h.info1;
+  }
+  return SVG2_OK;
+}
+
+int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int iters, int init, const double* u,
+                float* centroids, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets, void* ws,
+                size_t ws_bytes, void* stream) {
+  try {
+    int r = check_sizes(B, H, N, d);
+    if (r == SVG2_OK) r = check_k(k, N);
+    if (r != SVG2_OK) return r;
+    if (!valid_dtype(dtype) || iters < 1 || (init != SVG2_INIT_GIVEN && init != SVG2_INIT_KMEANSPP))
+      return SVG2_ERR_INVALID_ARG;
+    if (X == nullptr || centroids == nullptr || labels == nullptr || counts == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (init == SVG2_INIT_KMEANSPP && u == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(centroids, 16)) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+    KmeansScratch s;
+    carve_kmeans(c, BH, N, d, k, s, perm == nullptr);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    if (perm == nullptr) perm = s.perm;
+    if (offsets == nullptr) offsets = s.offsets;
+    return to_status(run_kmeans(X, dtype == SVG2_F32, BH, N, d, k, iters, init, u, centroids, labels, counts, perm,
+                                offsets, s, st, static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+static int select_common(const float* cq, const float* ck, const float* w_in, const int32_t* count_k, int B, int H,
+                         int nQ, int nK, int d, float top_p, float scale, float* weights, uint8_t* mask,
+                         int32_t* sel_count, int32_t* sel_idx, int32_t* stream_len, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (B < 1 || H < 1 || nQ < 1 || nK < 1) return SVG2_ERR_INVALID_ARG;
+  if (nQ > SVG2_MAX_CLUSTERS || nK > SVG2_MAX_CLUSTERS) return SVG2_ERR_UNSUPPORTED;
+  if (w_in == nullptr && d != 64 && d != 128) return SVG2_ERR_UNSUPPORTED;
+  if (!(top_p > 0.f) || top_p != top_p) return SVG2_ERR_INVALID_ARG;
+  if (count_k == nullptr || mask == nullptr || sel_count == nullptr || sel_idx == nullptr) return SVG2_ERR_INVALID_ARG;
+  if (w_in == nullptr && (cq == nullptr || ck == nullptr)) return SVG2_ERR_INVALID_ARG;
+  int r = check_ws(ws, ws_bytes, kStatusBytes);
+  if (r != SVG2_OK) return r;
+  return to_status(launch_select(cq, ck, w_in, count_k, B * H, nQ, nK, d, top_p, scale, weights, mask, sel_count,
+                                 sel_idx, stream_len, static_cast<cudaStream_t>(stream)));
+}
+
+int svg2_select(const float* cq, const float* ck, const int32_t* count_k, int B, int H, int nQ, int nK, int d,
+                float top_p, float scale, float* weights, uint8_t* mask, int32_t* sel_count, int32_t* sel_idx,
+                int32_t* stream_len, void* ws, size_t ws_bytes, void* stream) {
+  try {
+    return select_common(cq, ck, nullptr, count_k, B, H, nQ, nK, d, top_p, scale, weights, mask, sel_count, sel_idx,
+                         stream_len, ws, ws_bytes, stream);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_select_from_weights(const float* weights, const int32_t* count_k, int B, int H, int nQ, int nK, float top_p,
+                             uint8_t* mask, int32_t* sel_count, int32_t* sel_idx, int32_t* stream_len, void* ws,
+                             size_t ws_bytes, void* stream) {
+  try {
+    if (weights == nullptr) return SVG2_ERR_INVALID_ARG;
+    return select_common(nullptr, nullptr, weights, count_k, B, H, nQ, nK, 0, top_p, 1.f, nullptr, mask, sel_count,
+                         sel_idx, stream_len, ws, ws_bytes, stream);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_sort(const int32_t* labels, int B, int H, int N, int k, int32_t* perm, int32_t* offsets, int32_t* counts,
+              void* ws, size_t ws_bytes, void* stream) {
+  try {
+    if (B < 1 || H < 1 || N < 1) return SVG2_ERR_INVALID_ARG;
+    if (N > SVG2_MAX_TOKENS) return SVG2_ERR_UNSUPPORTED;
+    if (k < 1) return SVG2_ERR_INVALID_ARG;
+    if (k > SVG2_MAX_CLUSTERS) return SVG2_ERR_UNSUPPORTED;  // (a sort may have more clusters than tokens)
+    int r = SVG2_OK;
+    if (labels == nullptr || perm == nullptr || offsets == nullptr) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+    int32_t* ch = c.take<int32_t>(static_cast<size_t>(BH) * kSortChunks * k);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    return to_status(launch_sort(labels, BH, N, k, perm, offsets, counts, ch, st, static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_gather(const void* X, int dtype, const int32_t* perm, int B, int H, int N, int d, void* Xp, void* stream) {
+  try {
+    const int r = check_sizes(B, H, N, d);
+    if (r != SVG2_OK) return r;
+    if (!valid_dtype(dtype) || X == nullptr || perm == nullptr || Xp == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(Xp, 16)) return SVG2_ERR_INVALID_ARG;
+    return to_status(launch_gather(X, dtype == SVG2_F32, perm, B * H, N, d, Xp, static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_permute(const void* X, int dtype, const int32_t* labels, int B, int H, int N, int d, int k, void* Xp,
+                 int32_t* perm, int32_t* offsets, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  try {
+    int r = svg2_sort(labels, B, H, N, k, perm, offsets, counts, ws, ws_bytes, stream);
+    if (r != SVG2_OK) return r;
+    return svg2_gather(X, dtype, perm, B, H, N, d, Xp, stream);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off, const int32_t* k_off,
+                     const int32_t* sel_count, const int32_t* sel_idx, int B, int H, int N, int d, int nQ, int nK,
+                     float scale, const int32_t* perm_q, void* O, void* ws, size_t ws_bytes, void* stream) {
+  try {
+    int r = check_sizes(B, H, N, d);
+    if (r == SVG2_OK) r = check_k(nQ, N);
+    if (r == SVG2_OK) r = check_k(nK, N);
+    if (r != SVG2_OK) return r;
+    if (Qp == nullptr || Kp == nullptr || Vp == nullptr || q_off == nullptr || k_off == nullptr ||
+        sel_count == nullptr || sel_idx == nullptr || O == nullptr)
+      return SVG2_ERR_INVALID_ARG;
+    if (!aligned(Qp, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(O, 16)) return SVG2_ERR_INVALID_ARG;
+    if (scale != scale) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+    AttnScratch a;
+    carve_attn(c, BH, N, nQ, a);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    return to_status(launch_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, BH, N, d, nQ, nK, scale, perm_q,
+                                        O, a, st, static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_unpermute(const void* Op, const int32_t* perm, int B, int H, int N, int d, void* O, void* stream) {
+  try {
+    const int r = check_sizes(B, H, N, d);
+    if (r != SVG2_OK) return r;
+    if (Op == nullptr || perm == nullptr || O == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (!aligned(Op, 16) || !aligned(O, 16)) return SVG2_ERR_INVALID_ARG;
+    return to_status(launch_unpermute(Op, perm, B * H, N, d, O, static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, int H, int N, int d,
+               const svg2_params* p, const double* uq, const double* uk, float* cq, float* ck, void* O,
+               const svg2_layer_outputs* outs, void* ws, size_t ws_bytes, void* stream) {
+  try {
+    if (p == nullptr) return SVG2_ERR_INVALID_ARG;
+    int r = check_sizes(B, H, N, d);
+    if (r == SVG2_OK) r = check_k(p->nQ, N);
+    if (r == SVG2_OK) r = check_k(p->nK, N);
+    if (r != SVG2_OK) return r;
+    if (!valid_dtype(dtype) || p->iters < 1 || (p->init != SVG2_INIT_GIVEN && p->init != SVG2_INIT_KMEANSPP))
+      return SVG2_ERR_INVALID_ARG;
+    if (!(p->top_p > 0.f) || p->scale != p->scale) return SVG2_ERR_INVALID_ARG;
+    if (Q == nullptr || K == nullptr || V == nullptr || cq == nullptr || ck == nullptr || O == nullptr)
+      return SVG2_ERR_INVALID_ARG;
+    if (p->init == SVG2_INIT_KMEANSPP && (uq == nullptr || uk == nullptr)) return SVG2_ERR_INVALID_ARG;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(cq, 16) ||
+        !aligned(ck, 16))
+      return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    LayerCarve L;
+    carve_layer(c, BH, N, d, p->nQ, p->nK, outs, L);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool f32 = dtype == SVG2_F32;
+    cudaError_t e = run_kmeans(Q, f32, BH, N, d, p->nQ, p->iters, p->init, uq, cq, L.labels_q, L.count_q, L.perm_q,
+                               L.q_off, L.kq, L.st, s);
+    if (e == cudaSuccess)
+      e = run_kmeans(K, f32, BH, N, d, p->nK, p->iters, p->init, uk, ck, L.labels_k, L.count_k, L.perm_k, L.k_off,
+                     L.kk, L.st, s);
+    if (e == cudaSuccess)
+      e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, L.weights, L.mask,
+                        L.sel_count, L.sel_idx, L.stream_len, s);
+    if (e == cudaSuccess) e = launch_gather(Q, f32, L.perm_q, BH, N, d, L.Qp, s);
+    if (e == cudaSuccess) e = launch_gather2(K, V, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s);
+    if (e == cudaSuccess) {
+      if (p->fuse_unpermute) {
+        e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
+                               p->scale, L.perm_q, O, L.attn, L.st, s);
+      } else {
+        e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
+                               p->scale, nullptr, L.Op, L.attn, L.st, s);
+        if (e == cudaSuccess) e = launch_unpermute(L.Op, L.perm_q, BH, N, d, O, s);
+      }
+    }
+    return to_status(e);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O, void* ws,
+                      size_t ws_bytes, void* stream) {
+  try {
+    if (A == nullptr || Bm == nullptr || V == nullptr || C == nullptr || O == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (n != 64 && n != 128 && n != 256) return SVG2_ERR_UNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(Bm, 16) || !aligned(V, 16)) return SVG2_ERR_INVALID_ARG;
+    const int r = check_ws(ws, ws_bytes, kStatusBytes);
+    if (r != SVG2_OK) return r;
+    return to_status(launch_selftest_mma(A, Bm, n, V, C, O, static_cast<DeviceStatus*>(ws),
+                                         static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+}  // extern "C"

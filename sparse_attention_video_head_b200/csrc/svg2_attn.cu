@@ -1,0 +1,599 @@
+// Variable-block-size sparse attention ("Sparse VideoGen2" wiki summary, Method (4); Key claims
+// section 4.3, Fig. 7(b)) on tcgen05 tensor cores with TMEM accumulators.
+//
+// Work unit = up to two 128-row Q tiles (A, B) of one Q cluster.  Their keys are the rows of the
+// kept K clusters, concatenated into one packed key stream and cut into 128-key tiles, so a
+// cluster boundary costs nothing; only the stream's last tile is masked.  The design follows the
+// Blackwell execution model rather than the pages' FlashInfer-derived kernel:
+//   warps 0-3   softmax + correction + epilogue for Q tile A (TMEM lanes = query rows)
+//   warps 4-7   the same for Q tile B
+//   warps 8-11  key/value producer: thread r gathers row r of each key tile with cp.async into
+//               the 128-byte-swizzled layout the tensor core reads (two stages)
+//   warp 12     Q tiles by TMA, then the single-thread MMA issuer
+//   warp 13     TMEM allocator (512 columns: S_A, S_B, O_A, O_B; P overwrites S as bf16)
+// MMA order per key tile j: PV_A(j-1) -> S_A(j) -> PV_B(j-1) -> S_B(j).  Because tcgen05 ops of
+// one thread complete in order, "S_X(j) done" also means "O_X holds every PV up to j-1", so the
+// softmax warps rescale O_X in TMEM (only when the row max grows by more than 2^8) before
+// releasing P_X(j).  Softmax is exact: p = 2^(s*scale*log2e - m), O / l at the end, with l summed
+// over the bf16-rounded p that the PV product uses.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "svg2_device.cuh"
+#include "svg2_internal.h"
+
+namespace svg2 {
+
+namespace {
+
+constexpr int kAttnThreads = 512;
+constexpr int kMaxRanges = 1024;
+// bytes of one 128-row tile of d bf16 values (d/64 swizzled 16 KB halves)
+template <int D>
+constexpr uint32_t tile_bytes() { return 128u * D * 2u; }
+template <int D>
+constexpr uint32_t attn_smem() { return 6 * tile_bytes<D>() + 1024 /*align*/ + 4096 /*ranges*/ + 4096 + 64 /*cum*/ + 256; }
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct AttnBars {
+  uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], o_full, mma_done;
+  uint32_t tmem_base;
+  int32_t L;
+  int32_t nranges;
+};
+
+__global__ void plan_count_kernel(const int32_t* __restrict__ q_off, int nQ, int N,
+                                  int32_t* __restrict__ head_units) {
+  __shared__ int32_t part[32];
+  const int bh = blockIdx.x;
+  int acc = 0;
+  for (int i = threadIdx.x; i < nQ; i += blockDim.x) {
+    const int r0 = q_off[static_cast<size_t>(bh) * (nQ + 1) + i];
+    const int n = q_off[static_cast<size_t>(bh) * (nQ + 1) + i + 1] - r0;
+    if (r0 < 0 || n <= 0 || r0 + n > N) continue;
+    acc += (n + 255) / 256;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += part[w];
+    head_units[bh] = t;
+  }
+}
+
+__global__ void plan_scan_kernel(const int32_t* __restrict__ head_units, int BH, int32_t* __restrict__ head_base) {
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int b = 0; b < BH; ++b) {
+      head_base[b] = run;
+      run += head_units[b];
+    }
+    head_base[BH] = run;
+  }
+}
+
+__global__ void plan_write_kernel(const int32_t* __restrict__ q_off, int nQ, int N,
+                                  const int32_t* __restrict__ head_base, AttnUnit* __restrict__ units) {
+  const int bh = blockIdx.x;
+  if (threadIdx.x != 0) return;
+  int pos = head_base[bh];
+  const int32_t* qo = q_off + static_cast<size_t>(bh) * (nQ + 1);
+  for (int i = 0; i < nQ; ++i) {
+    const int r0 = qo[i], n = qo[i + 1] - qo[i];
+    if (r0 < 0 || n <= 0 || r0 + n > N) continue;  // malformed offsets produce no work
+    for (int u = 0; u < n; u += 256) {
+      AttnUnit un;
+      un.bh = bh;
+      un.cluster = i;
+      un.row0 = r0 + u;
+      un.nrows = min(256, n - u);
+      units[pos++] = un;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ Kp,
+                       const __nv_bfloat16* __restrict__ Vp, const int32_t* __restrict__ k_off,
+                       const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_idx, int N, int nQ,
+                       int nK, float scale, const int32_t* __restrict__ perm_q, __nv_bfloat16* __restrict__ O,
+                       const AttnUnit* __restrict__ units, const int32_t* __restrict__ head_base, int BH,
+                       DeviceStatus* st) {
+  const int total_units = head_base[BH];
+  if (static_cast<int>(blockIdx.x) >= total_units) return;
+  if (status_set(st)) return;
+  const AttnUnit un = units[blockIdx.x];
+
+  constexpr uint32_t kTile = tile_bytes<D>();
+  constexpr int kHalves = D / 64;   // 128-byte swizzle atoms across d
+  constexpr int kSteps = D / 16;    // K=16 MMA steps across d
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem;                 // Q_A, Q_B
+  uint8_t* k_s = smem + 2 * kTile;     // K stage 0, 1
+  uint8_t* v_s = smem + 4 * kTile;     // V stage 0, 1
+  int32_t* r_start = reinterpret_cast<int32_t*>(smem + 6 * kTile);
+  int32_t* r_cum = r_start + kMaxRanges;  // kMaxRanges + 1 entries
+  AttnBars* bars = reinterpret_cast<AttnBars*>(r_cum + kMaxRanges + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = un.bh;
+  const bool has_b = un.nrows > 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->k_full[i]), 128);
+      mbar_init(smem_u32(&bars->v_full[i]), 128);
+      mbar_init(smem_u32(&bars->kv_empty[i]), 1);
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->p_full[i]), 4);
+    }
+    mbar_init(smem_u32(&bars->o_full), 1);
+    mbar_init(smem_u32(&bars->mma_done), 1);
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp >= 8 && warp < 12) {
+    // key-stream range table: start row and stream offset of every kept K cluster
+    const int pt = threadIdx.x - 256;
+    const size_t row = static_cast<size_t>(bh) * nQ + un.cluster;
+    int cnt = sel_count[row];
+    cnt = cnt < 0 ? 0 : (cnt > nK ? nK : cnt);
+    const int32_t* ko = k_off + static_cast<size_t>(bh) * (nK + 1);
+    // each thread handles a contiguous block of entries, then a scan over the 128 block sums
+    const int per = (cnt + 127) / 128;
+    const int e0 = min(cnt, pt * per), e1 = min(cnt, e0 + per);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) {
+      int j = sel_idx[row * nK + e];
+      j = j < 0 ? 0 : (j >= nK ? nK - 1 : j);
+      const int s0 = ko[j], len = ko[j + 1] - s0;
+      r_start[e] = s0;
+      r_cum[e] = len;  // temporarily the length
+      local += len;
+    }
+    // scan of `local` across the 128 producer threads (4 warps) via shuffles + shared
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int32_t* wsum = r_cum + kMaxRanges + 1;  // 4 scratch ints (inside the 16-int gap)
+    if (lane == 31) wsum[warp - 8] = incl;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int wbase = 0;
+    for (int w = 0; w < warp - 8; ++w) wbase += wsum[w];
+    int run = wbase + incl - local;
+    for (int e = e0; e < e1; ++e) {
+      const int len = r_cum[e];
+      r_cum[e] = run;
+      run += len;
+    }
+    if (pt == 127) {
+      bars->L = run;  // thread 127 holds the last block
+      bars->nranges = cnt;
+      r_cum[cnt] = run;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int L = bars->L;
+  const int nranges = bars->nranges;
+  const int nt = (L + 127) / 128;
+
+  if (warp == 12) {
+    // ---------------- Q by TMA, then MMA issue ----------------
+    if (elect_one()) {
+      prefetch_tensormap(&tm_q);
+      const uint32_t qbar = smem_u32(&bars->q_full);
+      const uint32_t qa = smem_u32(q_s), qb = smem_u32(q_s + kTile);
+      mbar_arrive_expect_tx(qbar, has_b ? 2 * kTile : kTile);
+      const int y = bh * N + un.row0;
+#pragma unroll
+      for (int hf = 0; hf < kHalves; ++hf) {
+        tma_load_2d(qa + hf * 16384, &tm_q, hf * 64, y, qbar);
+        if (has_b) tma_load_2d(qb + hf * 16384, &tm_q, hf * 64, y + 128, qbar);
+      }
+      bool ok = mbar_wait(qbar, 0, st, kWhereAttnMma);
+      const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
+      const uint32_t id_o = idesc_bf16_f32(128, D, 1);
+      const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
+      auto issue_s = [&](int x, int stage) {
+        const uint32_t qbase = x == 0 ? qa : qb;
+        const uint32_t kbase = kb + stage * kTile;
+        const uint32_t d_tmem = tmem + x * 128;
+#pragma unroll
+        for (int ks = 0; ks < kSteps; ++ks) {
+          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_ss(d_tmem, sdesc_sw128(qbase + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024), id_s,
+                 ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int x, int stage, int j) {
+        const uint32_t vbase = vb + stage * kTile;
+        const uint32_t d_tmem = tmem + 256 + x * 128;
+        const uint32_t p_tmem = tmem + x * 128;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          mma_ts(d_tmem, p_tmem + ks * 8, sdesc_sw128(vbase + ks * 2048, 16384, 1024), id_o,
+                 (j > 0 || ks > 0) ? 1u : 0u);
+        }
+      };
+      if (ok && nt > 0) {
+        ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          mma_commit(smem_u32(&bars->s_full[0]));
+          if (has_b) {
+            issue_s(1, 0);
+            mma_commit(smem_u32(&bars->s_full[1]));
+          }
+        }
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        const int stage = j & 1;
+        ok = mbar_wait(smem_u32(&bars->p_full[0]), j & 1, st, kWhereAttnMma);
+        if (ok) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, stage, j);
+        const bool more = j + 1 < nt;
+        if (more) {
+          ok = mbar_wait(smem_u32(&bars->k_full[stage ^ 1]), ((j + 1) >> 1) & 1, st, kWhereAttnMma);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, stage ^ 1);
+          mma_commit(smem_u32(&bars->s_full[0]));
+        }
+        if (has_b) {
+          ok = mbar_wait(smem_u32(&bars->p_full[1]), j & 1, st, kWhereAttnMma);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, stage, j);
+        }
+        mma_commit(smem_u32(&bars->kv_empty[stage]));
+        if (has_b && more) {
+          issue_s(1, stage ^ 1);
+          mma_commit(smem_u32(&bars->s_full[1]));
+        }
+      }
+      if (ok) mma_commit(smem_u32(&bars->o_full));
+      mma_commit(smem_u32(&bars->mma_done));
+      mbar_wait(smem_u32(&bars->mma_done), 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
+      if (!ok) mbar_wait(qbar, 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------- key/value gather producer ----------------
+    const int r = threadIdx.x - 256;
+    const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
+    const size_t head_row0 = static_cast<size_t>(bh) * N;
+    for (int j = 0; j < nt; ++j) {
+      const int stage = j & 1;
+      if (j >= 2) {
+        if (!mbar_wait(smem_u32(&bars->kv_empty[stage]), ((j >> 1) - 1) & 1, st, kWhereAttnProducer)) break;
+      }
+      int p = j * 128 + r;
+      if (p >= L) p = L - 1;
+      // largest e with r_cum[e] <= p
+      int lo = 0, hi = nranges - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (r_cum[mid] <= p) lo = mid; else hi = mid - 1;
+      }
+      int krow = r_start[lo] + (p - r_cum[lo]);
+      krow = krow < 0 ? 0 : (krow >= N ? N - 1 : krow);
+      const __nv_bfloat16* ksrc = Kp + (head_row0 + krow) * D;
+      const __nv_bfloat16* vsrc = Vp + (head_row0 + krow) * D;
+      const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cp_async16(kdst + h * 16384 + sw128_offset(r, c), ksrc + h * 64 + c * 8);
+      cp_async_commit();
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cp_async16(vdst + h * 16384 + sw128_offset(r, c), vsrc + h * 64 + c * 8);
+      cp_async_commit();
+      cp_async_wait<1>();
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&bars->k_full[stage]));
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&bars->v_full[stage]));
+    }
+    cp_async_wait<0>();
+  } else if (warp < 8) {
+    // ---------------- softmax / correction / epilogue for tile X ----------------
+    const int x = warp >> 2;
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int nrows_x = x == 0 ? min(128, un.nrows) : un.nrows - 128;
+    if (x == 1 && !has_b) {
+      // nothing to do
+    } else {
+      const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+      const uint32_t t_s = tmem + lane_off + x * 128;
+      const uint32_t t_o = tmem + lane_off + 256 + x * 128;
+      const float sl2 = scale * kLog2e;
+      // Every tcgen05.ld/st below is a warp-collective (.sync.aligned) instruction, so all of it
+      // runs under warp-uniform control flow; per-row decisions only select values.
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nt; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x]), j & 1, st, kWhereAttnSoftmax));
+        if (!ok) break;
+        tc_fence_after();
+        const int valid = min(128, L - j * 128);
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_s + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+        }
+        const float m_new = fmaxf(m_used, mx * sl2);
+        const bool grow = m_new > m_used + kRescaleThreshold;
+        float f = 1.f;
+        if (grow) {
+          if (j > 0) f = fast_exp2(m_used - m_new);
+          l *= f;
+          m_used = m_new;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O holds every PV product up to tile j-1 (S_X(j) completing implies it); rows that keep
+          // their max multiply by 1.
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(t_o + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+            tmem_st32(t_o + c * 32, v);
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_s + c * 32, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = c * 32 + 2 * e;
+            const float p0 = col < valid ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), sl2, -m_used)) : 0.f;
+            const float p1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), sl2, -m_used)) : 0.f;
+            pk[e] = pack_bf16x2(p0, p1);
+            l += bf16lo_to_f32(pk[e]) + bf16hi_to_f32(pk[e]);
+          }
+          tmem_st16(t_s + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x]));
+      }
+      if (ok && nt > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0, st, kWhereAttnSoftmax));
+      if (ok) {
+        tc_fence_after();
+        const int prow = un.row0 + x * 128 + row;
+        int tk = -1;
+        if (row < nrows_x) {
+          tk = perm_q != nullptr ? __ldg(perm_q + static_cast<size_t>(bh) * N + prow) : prow;
+          if (tk < 0 || tk >= N) tk = -1;  // an invalid permutation entry is skipped
+        }
+        uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<size_t>(bh) * N + (tk < 0 ? 0 : tk)) * D);
+        const float inv = (nt > 0 && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (nt > 0) {
+            tmem_ld32(t_o + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (tk >= 0) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv, __uint_as_float(v[8 * e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv);
+              dst[c * 4 + e] = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Self-test of the tensor-core path: C = A B^T, then O = bf16(C[:, :128]) V with P from TMEM.
+// ------------------------------------------------------------------------------------------------
+struct TestBars {
+  uint64_t full, mma1, mma2;
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(128, 1)
+    selftest_mma_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_v, int n, float* __restrict__ C,
+                        float* __restrict__ Out, DeviceStatus* st) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_s = smem;                  // 32 KB
+  uint8_t* b_s = smem + 32768;          // up to 64 KB (256 rows)
+  uint8_t* v_s = smem + 32768 + 65536;  // 32 KB
+  TestBars* bars = reinterpret_cast<TestBars*>(v_s + 32768);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->full), 1);
+    mbar_init(smem_u32(&bars->mma1), 1);
+    mbar_init(smem_u32(&bars->mma2), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t bhalf = static_cast<uint32_t>(n) * 128u;  // bytes per 64-column half of B
+  bool ok = true;
+  if (warp == 0 && elect_one()) {
+    const uint32_t bar = smem_u32(&bars->full);
+    mbar_arrive_expect_tx(bar, 32768 + 2 * bhalf + 32768);
+    tma_load_2d(smem_u32(a_s), &tm_a, 0, 0, bar);
+    tma_load_2d(smem_u32(a_s) + 16384, &tm_a, 64, 0, bar);
+    tma_load_2d(smem_u32(b_s), &tm_b, 0, 0, bar);
+    tma_load_2d(smem_u32(b_s) + bhalf, &tm_b, 64, 0, bar);
+    tma_load_2d(smem_u32(v_s), &tm_v, 0, 0, bar);
+    tma_load_2d(smem_u32(v_s) + 16384, &tm_v, 64, 0, bar);
+    ok = mbar_wait(bar, 0, st, kWhereSelftest);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, static_cast<uint32_t>(n), 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
+        const uint32_t kob = (ks >> 2) * bhalf + (ks & 3) * 32;
+        mma_ss(tmem, sdesc_sw128(smem_u32(a_s) + ko, 16, 1024), sdesc_sw128(smem_u32(b_s) + kob, 16, 1024), idesc,
+               ks > 0 ? 1u : 0u);
+      }
+    }
+    mma_commit(smem_u32(&bars->mma1));
+  }
+  __syncwarp();
+  ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->mma1), 0, st, kWhereSelftest));
+  tc_fence_after();
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const int row = warp * 32 + lane;
+  if (ok) {
+    for (int c = 0; c < n / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + c * 32, v);
+      tmem_wait_ld();
+      for (int e = 0; e < 32; ++e) C[static_cast<size_t>(row) * n + c * 32 + e] = __uint_as_float(v[e]);
+      if (c < 4) {
+        uint32_t pk[16];
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        tmem_st16(tmem + lane_off + 256 + c * 16, pk);
+      }
+    }
+    if (n < 128) {
+      uint32_t pk[16];
+      for (int e = 0; e < 16; ++e) pk[e] = 0u;
+      for (int c = n / 32; c < 4; ++c) tmem_st16(tmem + lane_off + 256 + c * 16, pk);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0 && elect_one()) {
+    if (ok) {
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts(tmem + 384, tmem + 256 + ks * 8, sdesc_sw128(smem_u32(v_s) + ks * 2048, 16384, 1024), idesc,
+               ks > 0 ? 1u : 0u);
+    }
+    mma_commit(smem_u32(&bars->mma2));
+  }
+  __syncwarp();
+  ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->mma2), 0, st, kWhereSelftest) && ok);
+  tc_fence_after();
+  if (ok) {
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + 384 + c * 32, v);
+      tmem_wait_ld();
+      for (int e = 0; e < 32; ++e) Out[static_cast<size_t>(row) * 128 + c * 32 + e] = __uint_as_float(v[e]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
+                               const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int BH,
+                               int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
+                               const AttnScratch& sc, DeviceStatus* st, cudaStream_t s) {
+  plan_count_kernel<<<BH, 256, 0, s>>>(q_off, nQ, N, sc.head_units);
+  plan_scan_kernel<<<1, 32, 0, s>>>(sc.head_units, BH, sc.head_base);
+  plan_write_kernel<<<BH, 32, 0, s>>>(q_off, nQ, N, sc.head_base, sc.units);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  alignas(64) CUtensorMap tq;
+  e = make_tmap_bf16_rows(&tq, Qp, static_cast<uint64_t>(BH) * N, static_cast<uint32_t>(d), 128);
+  if (e != cudaSuccess) return e;
+  const long long grid = static_cast<long long>(BH) * attn_max_units_per_head(N, nQ);
+  if (d == 128) {
+    e = cudaFuncSetAttribute(sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<128>());
+    if (e != cudaSuccess) return e;
+    sparse_attn_kernel<128><<<static_cast<unsigned>(grid), kAttnThreads, attn_smem<128>(), s>>>(
+        tq, static_cast<const __nv_bfloat16*>(Kp), static_cast<const __nv_bfloat16*>(Vp), k_off, sel_count, sel_idx,
+        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st);
+  } else {
+    e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<64>());
+    if (e != cudaSuccess) return e;
+    sparse_attn_kernel<64><<<static_cast<unsigned>(grid), kAttnThreads, attn_smem<64>(), s>>>(
+        tq, static_cast<const __nv_bfloat16*>(Kp), static_cast<const __nv_bfloat16*>(Vp), k_off, sel_count, sel_idx,
+        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O,
+                                DeviceStatus* st, cudaStream_t s) {
+  alignas(64) CUtensorMap ta, tb, tv;
+  cudaError_t e = make_tmap_bf16_rows(&ta, A, 128, 128, 128);
+  if (e == cudaSuccess) e = make_tmap_bf16_rows(&tb, Bm, static_cast<uint64_t>(n), 128, static_cast<uint32_t>(n));
+  if (e == cudaSuccess) e = make_tmap_bf16_rows(&tv, V, 128, 128, 128);
+  if (e != cudaSuccess) return e;
+  const uint32_t smem = 32768 + 65536 + 32768 + 1024 + 256;
+  e = cudaFuncSetAttribute(selftest_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  selftest_mma_kernel<<<1, 128, smem, s>>>(ta, tb, tv, n, C, O, st);
+  return cudaGetLastError();
+}
+
+}  // namespace svg2

@@ -1,0 +1,142 @@
+// Internal declarations shared by the .cu files of libsvg2 (not part of the public C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace svg2 {
+
+// Device status word, at offset 0 of every workspace.
+struct DeviceStatus {
+  uint32_t code;   // svg2_status of the first device error, 0 if none
+  uint32_t where;  // kernel tag (kWhere*)
+  uint32_t info0;
+  uint32_t info1;
+};
+
+constexpr uint32_t kStatusDeviceTimeout = 5;  // == SVG2_ERR_DEVICE_TIMEOUT
+constexpr uint32_t kStatusDeviceBounds = 6;   // == SVG2_ERR_DEVICE_BOUNDS
+
+// About 0.5 s at the B200's boost clock: far above any legitimate wait inside one tile step.
+constexpr long long kWaitBudgetCycles = 1000LL * 1000LL * 1000LL;
+
+// Kernel tags for DeviceStatus::where.
+enum : uint32_t {
+  kWhereSort = 1,
+  kWhereAssign = 2,
+  kWhereAttnProducer = 3,
+  kWhereAttnMma = 4,
+  kWhereAttnSoftmax = 5,
+  kWhereSelftest = 6,
+  kWhereAssignTail = 7,
+  kWhereAttnDrain = 8,
+};
+
+constexpr int kStatusBytes = 256;
+constexpr int kSortChunks = 32;  // token chunks per (b,h) in the stable counting sort
+constexpr int kAssignTileM = 128;
+constexpr int kAssignChunkN = 128;  // centroids per MMA chunk
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int kpad_of(int k) { return (k + kAssignChunkN - 1) / kAssignChunkN * kAssignChunkN; }
+
+// Bump allocator over the caller's workspace; with base == nullptr it only measures.
+struct Carve {
+  char* base;
+  size_t off;
+  explicit Carve(void* b) : base(static_cast<char*>(b)), off(0) {}
+  template <class T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+// Scratch of one k-means call (one role).
+struct KmeansScratch {
+  uint16_t* c_hi;     // [BH, kpad, d] bf16 high part of the centroids
+  uint16_t* c_lo;     // [BH, kpad, d] bf16 residual part
+  float* c_norm;      // [BH, kpad] squared norms of the centroids
+  double* pp_dist;    // [BH, N] k-means++ current D^2
+  int32_t* pp_near;   // [BH, N] k-means++ nearest seed
+  int32_t* chunk_hist;// [BH, kSortChunks, k]
+  int32_t* perm;      // [BH, N] (if the caller passes none)
+  int32_t* offsets;   // [BH, k+1]
+};
+
+inline void carve_kmeans(Carve& c, int BH, int N, int d, int k, KmeansScratch& s, bool need_perm) {
+  const int kp = kpad_of(k);
+  s.c_hi = c.take<uint16_t>(static_cast<size_t>(BH) * kp * d);
+  s.c_lo = c.take<uint16_t>(static_cast<size_t>(BH) * kp * d);
+  s.c_norm = c.take<float>(static_cast<size_t>(BH) * kp);
+  s.pp_dist = c.take<double>(static_cast<size_t>(BH) * N);
+  s.pp_near = c.take<int32_t>(static_cast<size_t>(BH) * N);
+  s.chunk_hist = c.take<int32_t>(static_cast<size_t>(BH) * kSortChunks * k);
+  s.perm = need_perm ? c.take<int32_t>(static_cast<size_t>(BH) * N) : nullptr;
+  s.offsets = c.take<int32_t>(static_cast<size_t>(BH) * (k + 1));
+}
+
+// Attention work plan: one unit = up to two 128-row Q tiles of one Q cluster.
+struct AttnUnit {
+  int32_t bh;
+  int32_t cluster;
+  int32_t row0;   // first permuted row of the unit
+  int32_t nrows;  // 1..256
+};
+
+inline int attn_max_units_per_head(int N, int nQ) { return (N + 255) / 256 + nQ; }
+
+struct AttnScratch {
+  AttnUnit* units;     // [BH * max_units_per_head] compacted
+  int32_t* head_units; // [BH]
+  int32_t* head_base;  // [BH + 1]
+};
+
+inline void carve_attn(Carve& c, int BH, int N, int nQ, AttnScratch& s) {
+  s.units = c.take<AttnUnit>(static_cast<size_t>(BH) * attn_max_units_per_head(N, nQ));
+  s.head_units = c.take<int32_t>(BH);
+  s.head_base = c.take<int32_t>(BH + 1);
+}
+
+// ---- launchers (host functions defined in the .cu files); all return cudaError_t ----
+cudaError_t launch_sort(const int32_t* labels, int BH, int N, int k, int32_t* perm, int32_t* offsets,
+                        int32_t* counts, int32_t* chunk_hist, DeviceStatus* st, cudaStream_t s);
+cudaError_t launch_gather(const void* X, bool x_f32, const int32_t* perm, int BH, int N, int d, void* Xp,
+                          cudaStream_t s);
+cudaError_t launch_gather2(const void* X0, const void* X1, bool x_f32, const int32_t* perm, int BH, int N,
+                           int d, void* Xp0, void* Xp1, cudaStream_t s);
+cudaError_t launch_unpermute(const void* Op, const int32_t* perm, int BH, int N, int d, void* O,
+                             cudaStream_t s);
+
+cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
+                            float* centroids, double* dist, int32_t* near, cudaStream_t s);
+cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, uint16_t* c_hi, uint16_t* c_lo,
+                                 float* c_norm, cudaStream_t s);
+cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,
+                          const uint16_t* c_hi, const uint16_t* c_lo, const float* c_norm, int32_t* labels,
+                          DeviceStatus* st, cudaStream_t s);
+cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
+                          const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
+                          float* c_norm, cudaStream_t s);
+
+cudaError_t launch_select(const float* cq, const float* ck, const float* weights_in, const int32_t* count_k,
+                          int BH, int nQ, int nK, int d, float top_p, float scale, float* weights_out,
+                          uint8_t* mask, int32_t* sel_count, int32_t* sel_idx, int32_t* stream_len,
+                          cudaStream_t s);
+
+cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
+                               const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int BH,
+                               int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
+                               const AttnScratch& scratch, DeviceStatus* st, cudaStream_t s);
+
+cudaError_t launch_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O,
+                                DeviceStatus* st, cudaStream_t s);
+
+// Tensor map over a [rows, d] bf16 matrix with a box of 64 columns x box_rows rows, 128B swizzle.
+cudaError_t make_tmap_bf16_rows(void* map /* CUtensorMap* */, const void* base, uint64_t rows, uint32_t d,
+                                uint32_t box_rows);
+
+}  // namespace svg2

@@ -1,0 +1,247 @@
+"""Thin Python binding of libsvg2 (include/svg2.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  PyTorch supplies device memory
+and the current CUDA stream; all of the method's steps run in the library's sm_100a kernels.
+There is no fallback: if libsvg2.so is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsvg2.so")
+
+SVG2_BF16, SVG2_F32 = 0, 1
+SVG2_INIT_GIVEN, SVG2_INIT_KMEANSPP = 0, 1
+MAX_CLUSTERS = 1024
+
+_EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeans", "svg2_select",
+            "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
+            "svg2_unpermute", "svg2_layer", "svg2_selftest_mma")
+
+_lib = None
+
+
+class Svg2Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+class SvgParams(ctypes.Structure):
+    _fields_ = [("nQ", ctypes.c_int), ("nK", ctypes.c_int), ("iters", ctypes.c_int), ("init", ctypes.c_int),
+                ("top_p", ctypes.c_float), ("scale", ctypes.c_float), ("fuse_unpermute", ctypes.c_int)]
+
+
+class SvgLayerOutputs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "labels_q", "labels_k", "count_q", "count_k", "perm_q", "perm_k", "q_off", "k_off", "weights", "mask",
+        "sel_count", "sel_idx", "stream_len")]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsvg2.so (built in-tree by sparse_attention_video_head_b200/build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python sparse_attention_video_head_b200/build.py`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.svg2_status_string.argtypes = [I]
+        L.svg2_status_string.restype = ctypes.c_char_p
+        L.svg2_workspace_size.argtypes = [I, I, I, I, I, I, ctypes.POINTER(S)]
+        L.svg2_check_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_uint32),
+                                        ctypes.POINTER(ctypes.c_uint32)]
+        L.svg2_kmeans.argtypes = [P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, S, P]
+        L.svg2_select.argtypes = [P, P, P, I, I, I, I, I, F, F, P, P, P, P, P, P, S, P]
+        L.svg2_select_from_weights.argtypes = [P, P, I, I, I, I, F, P, P, P, P, P, S, P]
+        L.svg2_sort.argtypes = [P, I, I, I, I, P, P, P, P, S, P]
+        L.svg2_gather.argtypes = [P, I, P, I, I, I, I, P, P]
+        L.svg2_permute.argtypes = [P, I, P, I, I, I, I, I, P, P, P, P, P, S, P]
+        L.svg2_sparse_attn.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, S, P]
+        L.svg2_unpermute.argtypes = [P, P, I, I, I, I, P, P]
+        L.svg2_layer.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(SvgParams), P, P, P, P, P,
+                                 ctypes.POINTER(SvgLayerOutputs), P, S, P]
+        L.svg2_selftest_mma.argtypes = [P, P, I, P, P, P, P, S, P]
+        for name in _EXPORTS:
+            if name != "svg2_status_string":
+                getattr(L, name).restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().svg2_status_string(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise Svg2Error(rc, what)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libsvg2 takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libsvg2 takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SVG2_BF16
+    if t.dtype == torch.float32:
+        return SVG2_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def svg2_workspace_size(B: int, H: int, N: int, d: int, nQ: int, nK: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().svg2_workspace_size(B, H, N, d, nQ, nK, ctypes.byref(out)), "svg2_workspace_size")
+    return int(out.value)
+
+
+def workspace(B: int, H: int, N: int, d: int, nQ: int, nK: int, device=None) -> torch.Tensor:
+    """A workspace tensor for these sizes (device memory from torch; the status word starts at 0)."""
+    return torch.zeros(svg2_workspace_size(B, H, N, d, nQ, nK), dtype=torch.uint8, device=device or "cuda")
+
+
+def svg2_check_status(ws: torch.Tensor, stream=None):
+    code = ctypes.c_int(0)
+    where = ctypes.c_uint32(0)
+    info = (ctypes.c_uint32 * 2)()
+    _check(lib().svg2_check_status(_p(ws), _stream(stream), ctypes.byref(code), ctypes.byref(where), info),
+           "svg2_check_status")
+    return int(code.value), int(where.value), (int(info[0]), int(info[1]))
+
+
+def raise_on_device_error(ws: torch.Tensor, stream=None):
+    code, where, info = svg2_check_status(ws, stream)
+    if code != 0:
+        raise Svg2Error(code, f"device status (kernel tag {where}, info {info})")
+
+
+def svg2_kmeans(X: torch.Tensor, k: int, iters: int, init: int, centroids: torch.Tensor, labels: torch.Tensor,
+                counts: torch.Tensor, ws: torch.Tensor, u: Optional[torch.Tensor] = None,
+                perm: Optional[torch.Tensor] = None, offsets: Optional[torch.Tensor] = None, stream=None):
+    B, H, N, d = X.shape
+    _check(lib().svg2_kmeans(_p(X), _dtype(X), B, H, N, d, k, iters, init, _p(u), _p(centroids), _p(labels),
+                             _p(counts), _p(perm), _p(offsets), _p(ws), ws.numel(), _stream(stream)), "svg2_kmeans")
+
+
+def svg2_select(cq: torch.Tensor, ck: torch.Tensor, count_k: torch.Tensor, top_p: float, scale: float,
+                mask: torch.Tensor, sel_count: torch.Tensor, sel_idx: torch.Tensor, ws: torch.Tensor,
+                weights: Optional[torch.Tensor] = None, stream_len: Optional[torch.Tensor] = None, stream=None):
+    B, H, nQ, d = cq.shape
+    nK = ck.shape[2]
+    _check(lib().svg2_select(_p(cq), _p(ck), _p(count_k), B, H, nQ, nK, d, float(top_p), float(scale), _p(weights),
+                             _p(mask), _p(sel_count), _p(sel_idx), _p(stream_len), _p(ws), ws.numel(),
+                             _stream(stream)), "svg2_select")
+
+
+def svg2_select_from_weights(weights: torch.Tensor, count_k: torch.Tensor, top_p: float, mask: torch.Tensor,
+                             sel_count: torch.Tensor, sel_idx: torch.Tensor, ws: torch.Tensor,
+                             stream_len: Optional[torch.Tensor] = None, stream=None):
+    B, H, nQ, nK = weights.shape
+    _check(lib().svg2_select_from_weights(_p(weights), _p(count_k), B, H, nQ, nK, float(top_p), _p(mask),
+                                          _p(sel_count), _p(sel_idx), _p(stream_len), _p(ws), ws.numel(),
+                                          _stream(stream)), "svg2_select_from_weights")
+
+
+def svg2_sort(labels: torch.Tensor, k: int, perm: torch.Tensor, offsets: torch.Tensor, counts: Optional[torch.Tensor],
+              ws: torch.Tensor, stream=None):
+    B, H, N = labels.shape
+    _check(lib().svg2_sort(_p(labels), B, H, N, k, _p(perm), _p(offsets), _p(counts), _p(ws), ws.numel(),
+                           _stream(stream)), "svg2_sort")
+
+
+def svg2_gather(X: torch.Tensor, perm: torch.Tensor, Xp: torch.Tensor, stream=None):
+    B, H, N, d = X.shape
+    _check(lib().svg2_gather(_p(X), _dtype(X), _p(perm), B, H, N, d, _p(Xp), _stream(stream)), "svg2_gather")
+
+
+def svg2_permute(X: torch.Tensor, labels: torch.Tensor, k: int, Xp: torch.Tensor, perm: torch.Tensor,
+                 offsets: torch.Tensor, counts: Optional[torch.Tensor], ws: torch.Tensor, stream=None):
+    B, H, N, d = X.shape
+    _check(lib().svg2_permute(_p(X), _dtype(X), _p(labels), B, H, N, d, k, _p(Xp), _p(perm), _p(offsets),
+                              _p(counts), _p(ws), ws.numel(), _stream(stream)), "svg2_permute")
+
+
+def svg2_sparse_attn(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off: torch.Tensor, k_off: torch.Tensor,
+                     sel_count: torch.Tensor, sel_idx: torch.Tensor, scale: float, O: torch.Tensor, ws: torch.Tensor,
+                     perm_q: Optional[torch.Tensor] = None, stream=None):
+    B, H, N, d = Qp.shape
+    nQ = q_off.shape[-1] - 1
+    nK = k_off.shape[-1] - 1
+    _check(lib().svg2_sparse_attn(_p(Qp), _p(Kp), _p(Vp), _p(q_off), _p(k_off), _p(sel_count), _p(sel_idx), B, H, N,
+                                  d, nQ, nK, float(scale), _p(perm_q), _p(O), _p(ws), ws.numel(), _stream(stream)),
+           "svg2_sparse_attn")
+
+
+def svg2_unpermute(Op: torch.Tensor, perm: torch.Tensor, O: torch.Tensor, stream=None):
+    B, H, N, d = Op.shape
+    _check(lib().svg2_unpermute(_p(Op), _p(perm), B, H, N, d, _p(O), _stream(stream)), "svg2_unpermute")
+
+
+@dataclass
+class LayerParams:
+    nQ: int
+    nK: int
+    iters: int
+    init: int = SVG2_INIT_KMEANSPP
+    top_p: float = 0.9
+    scale: float = 1.0 / 128 ** 0.5
+    fuse_unpermute: int = 1
+
+    def c(self) -> SvgParams:
+        return SvgParams(self.nQ, self.nK, self.iters, self.init, self.top_p, self.scale, self.fuse_unpermute)
+
+
+def layer_output_buffers(B: int, H: int, N: int, nQ: int, nK: int, device="cuda") -> Dict[str, torch.Tensor]:
+    """Device buffers for every intermediate result the layer can expose (see svg2_layer_outputs)."""
+    i32 = dict(dtype=torch.int32, device=device)
+    return {
+        "labels_q": torch.empty(B, H, N, **i32), "labels_k": torch.empty(B, H, N, **i32),
+        "count_q": torch.empty(B, H, nQ, **i32), "count_k": torch.empty(B, H, nK, **i32),
+        "perm_q": torch.empty(B, H, N, **i32), "perm_k": torch.empty(B, H, N, **i32),
+        "q_off": torch.empty(B, H, nQ + 1, **i32), "k_off": torch.empty(B, H, nK + 1, **i32),
+        "weights": torch.empty(B, H, nQ, nK, dtype=torch.float32, device=device),
+        "mask": torch.empty(B, H, nQ, nK, dtype=torch.uint8, device=device),
+        "sel_count": torch.empty(B, H, nQ, **i32), "sel_idx": torch.empty(B, H, nQ, nK, **i32),
+        "stream_len": torch.empty(B, H, nQ, **i32),
+    }
+
+
+def svg2_layer(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, params: LayerParams, cq: torch.Tensor,
+               ck: torch.Tensor, O: torch.Tensor, ws: torch.Tensor, uq: Optional[torch.Tensor] = None,
+               uk: Optional[torch.Tensor] = None, outs: Optional[Dict[str, torch.Tensor]] = None, stream=None):
+    B, H, N, d = Q.shape
+    prm = params.c()
+    c_outs = None
+    if outs is not None:
+        c_outs = SvgLayerOutputs(*[(_p(outs[n]).value if outs.get(n) is not None else None)
+                                   for n, _ in SvgLayerOutputs._fields_])
+    _check(lib().svg2_layer(_p(Q), _p(K), _p(V), _dtype(Q), B, H, N, d, ctypes.byref(prm), _p(uq), _p(uk), _p(cq),
+                            _p(ck), _p(O), ctypes.byref(c_outs) if c_outs is not None else None, _p(ws), ws.numel(),
+                            _stream(stream)), "svg2_layer")
+
+
+def svg2_selftest_mma(A: torch.Tensor, Bm: torch.Tensor, V: torch.Tensor, ws: torch.Tensor, stream=None):
+    n = Bm.shape[0]
+    C = torch.empty(128, n, dtype=torch.float32, device=A.device)
+    O = torch.empty(128, 128, dtype=torch.float32, device=A.device)
+    _check(lib().svg2_selftest_mma(_p(A), _p(Bm), n, _p(V), _p(C), _p(O), _p(ws), ws.numel(), _stream(stream)),
+           "svg2_selftest_mma")
+    return C, O

@@ -1,0 +1,142 @@
+"""The C-ABI boundary on the host (no GPU): the library loads, exports every entry point that
+include/svg2.h declares, and rejects bad arguments with the documented status codes before it
+touches the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_video_head_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "svg2.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    from sparse_attention_video_head_b200 import svg2
+    return svg2.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SVG2_API\s+(?:const\s+)?\w+\*?\s+\**(svg2_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("svg2_kmeans", "svg2_select", "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute",
+              "svg2_sparse_attn", "svg2_unpermute", "svg2_layer", "svg2_workspace_size", "svg2_check_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_library_has_no_driver_or_torch_link_dependency():
+    B.build()
+    import subprocess
+    out = subprocess.run(["ldd", B.LIB], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out and "not found" not in out
+
+
+def test_status_strings(L):
+    from sparse_attention_video_head_b200 import svg2
+    assert svg2.status_string(0) == "SVG2_OK"
+    for c in range(1, 7):
+        assert svg2.status_string(c).startswith("SVG2_ERR")
+
+
+def test_workspace_size_is_monotone_and_validates(L):
+    from sparse_attention_video_head_b200 import svg2
+    small = svg2.svg2_workspace_size(1, 8, 12480, 128, 64, 256)
+    big = svg2.svg2_workspace_size(1, 40, 75600, 128, 100, 500)
+    assert 0 < small < big
+    # Wan-720p: Q, K, V permuted copies plus the un-fused output copy dominate (4 x 774 MB)
+    assert big > 4 * 40 * 75600 * 128 * 2
+    out = ctypes.c_size_t(0)
+    assert L.svg2_workspace_size(1, 1, 100, 96, 4, 4, ctypes.byref(out)) == UNSUPPORTED
+    assert L.svg2_workspace_size(1, 1, 100, 128, 0, 4, ctypes.byref(out)) == INVALID
+    assert L.svg2_workspace_size(1, 1, 100, 128, 101, 4, ctypes.byref(out)) == INVALID
+    assert L.svg2_workspace_size(1, 1, 5000, 128, 2000, 4, ctypes.byref(out)) == UNSUPPORTED
+    assert L.svg2_workspace_size(0, 1, 100, 128, 4, 4, ctypes.byref(out)) == INVALID
+    assert L.svg2_workspace_size(1, 1, 100, 128, 4, 4, None) == INVALID
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation first
+
+
+def test_kmeans_rejects_bad_arguments(L):
+    P = None
+    args = lambda **kw: dict(dict(X=FAKE, dt=0, B=1, H=1, N=100, d=128, k=4, it=1, init=0, u=P, C=FAKE, lab=FAKE,
+                                  cnt=FAKE, perm=P, off=P, ws=FAKE, wsb=1 << 30), **kw)
+    def call(**kw):
+        a = args(**kw)
+        return L.svg2_kmeans(a["X"], a["dt"], a["B"], a["H"], a["N"], a["d"], a["k"], a["it"], a["init"], a["u"],
+                             a["C"], a["lab"], a["cnt"], a["perm"], a["off"], a["ws"], a["wsb"], None)
+    assert call(X=None) == INVALID
+    assert call(dt=7) == INVALID
+    assert call(k=0) == INVALID
+    assert call(k=101) == INVALID
+    assert call(d=96) == UNSUPPORTED
+    assert call(it=0) == INVALID
+    assert call(init=5) == INVALID
+    assert call(init=1, u=None) == INVALID           # k-means++ needs its uniforms
+    assert call(ws=None) == WORKSPACE
+    assert call(wsb=16) == WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x10010)) == WORKSPACE   # not 256-byte aligned
+
+
+def test_select_and_topp_reject_bad_arguments(L):
+    F = ctypes.c_float
+    assert L.svg2_select(FAKE, FAKE, FAKE, 1, 1, 4, 8, 128, F(0.0), F(0.1), None, FAKE, FAKE, FAKE, None, FAKE,
+                         1 << 20, None) == INVALID
+    assert L.svg2_select(FAKE, FAKE, FAKE, 1, 1, 4, 2000, 128, F(0.9), F(0.1), None, FAKE, FAKE, FAKE, None, FAKE,
+                         1 << 20, None) == UNSUPPORTED
+    assert L.svg2_select(FAKE, FAKE, None, 1, 1, 4, 8, 128, F(0.9), F(0.1), None, FAKE, FAKE, FAKE, None, FAKE,
+                         1 << 20, None) == INVALID
+    assert L.svg2_select_from_weights(None, FAKE, 1, 1, 4, 8, F(0.9), FAKE, FAKE, FAKE, None, FAKE, 1 << 20,
+                                      None) == INVALID
+    assert L.svg2_select_from_weights(FAKE, FAKE, 1, 1, 4, 8, F(float("nan")), FAKE, FAKE, FAKE, None, FAKE, 1 << 20,
+                                      None) == INVALID
+    assert L.svg2_select_from_weights(FAKE, FAKE, 1, 1, 4, 8, F(0.9), FAKE, FAKE, FAKE, None, None, 0,
+                                      None) == WORKSPACE
+
+
+def test_permutation_calls_reject_bad_arguments(L):
+    assert L.svg2_sort(None, 1, 1, 10, 4, FAKE, FAKE, None, FAKE, 1 << 20, None) == INVALID
+    assert L.svg2_sort(FAKE, 1, 1, 10, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == INVALID
+    assert L.svg2_sort(FAKE, 1, 1, 10, 4096, FAKE, FAKE, None, FAKE, 1 << 20, None) == UNSUPPORTED
+    assert L.svg2_sort(FAKE, 1, 1, 10, 4, FAKE, FAKE, None, FAKE, 8, None) == WORKSPACE
+    assert L.svg2_gather(FAKE, 3, FAKE, 1, 1, 10, 128, FAKE, None) == INVALID
+    assert L.svg2_gather(FAKE, 0, FAKE, 1, 1, 10, 32, FAKE, None) == UNSUPPORTED
+    assert L.svg2_gather(ctypes.c_void_p(0x10002), 0, FAKE, 1, 1, 10, 128, FAKE, None) == INVALID
+    assert L.svg2_unpermute(FAKE, None, 1, 1, 10, 128, FAKE, None) == INVALID
+
+
+def test_attention_and_layer_reject_bad_arguments(L):
+    from sparse_attention_video_head_b200.svg2 import SvgParams
+    F = ctypes.c_float
+    assert L.svg2_sparse_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1000, 96, 4, 4, F(0.1), None, FAKE,
+                              FAKE, 1 << 30, None) == UNSUPPORTED   # the attention kernel is built for d = 64, 128
+    assert L.svg2_sparse_attn(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 1000, 128, 4, 4, F(0.1), None, FAKE,
+                              FAKE, 1 << 30, None) == INVALID
+    assert L.svg2_sparse_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1000, 128, 4, 4, F(0.1), None, FAKE,
+                              FAKE, 64, None) == WORKSPACE
+    p = SvgParams(4, 8, 2, 1, 0.9, 0.1, 1)
+    args = [FAKE, FAKE, FAKE, 0, 1, 1, 1000, 128, ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 34,
+            None]
+    bad = SvgParams(4, 8, 2, 1, 0.9, 0.1, 1)
+    bad.top_p = -1.0
+    assert L.svg2_layer(*args[:8], ctypes.byref(bad), *args[9:]) == INVALID
+    bad = SvgParams(4, 8, 0, 1, 0.9, 0.1, 1)
+    assert L.svg2_layer(*args[:8], ctypes.byref(bad), *args[9:]) == INVALID
+    assert L.svg2_layer(*args[:9], None, *args[10:]) == INVALID          # k-means++ without uniforms
+    assert L.svg2_layer(*args[:16], 1024, None) == WORKSPACE
+    assert L.svg2_layer(*args[:8], None, *args[9:]) == INVALID

@@ -1,0 +1,156 @@
+"""The whole layer through the C ABI (svg2_layer) vs the oracle, on the configured workloads.
+
+Per head, each stage is checked against the oracle given the GPU's own upstream results (so a
+near-tie label difference in k-means does not leak into the attention check):
+  permutation/offsets from the GPU labels: bit-exact; selection from the GPU centroids: mask equal
+  except where a float32 weight rounds differently (counted); attention on the GPU's permuted
+  inputs and mask: max-abs 2e-2, mean-abs 2e-3 (sampled rows at full size).  The independent
+  end-to-end agreement (labels, density, output error vs the oracle's own layer) is reported.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_attention_video_head_b200 import inputs as I
+from tests.gpu_helpers import bf16_dev, host, pool_layer_inputs, require_gpu, to_dev
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+
+
+def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1):
+    B, H, N, d = data["q"].shape
+    conv = to_dev if cfg.dtype == "f32" else bf16_dev
+    Q, K, V = conv(data["q"]), conv(data["k"]), conv(data["v"])
+    cq = torch.zeros(B, H, cfg.nQ, d, device="cuda") if cq is None else cq
+    ck = torch.zeros(B, H, cfg.nK, d, device="cuda") if ck is None else ck
+    O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device="cuda")
+    outs = svg2.layer_output_buffers(B, H, N, cfg.nQ, cfg.nK)
+    ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK)
+    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP if init is None else init, top_p,
+                           float(np.float32(cfg.scale)), fuse)
+    svg2.svg2_layer(Q, K, V, prm, cq, ck, O, ws, to_dev(data["uq"]), to_dev(data["uk"]), outs)
+    torch.cuda.synchronize()
+    svg2.raise_on_device_error(ws)
+    res = {k: host(v) for k, v in outs.items()}
+    res.update(o=host(O), cq=host(cq), ck=host(ck))
+    return res
+
+
+def check_head(oracle, cfg, data, res, h, top_p, rows=None):
+    scale = float(np.float32(cfg.scale))
+    q, k, v = data["q"][0, h], data["k"][0, h], data["v"][0, h]
+    g = {key: val[0, h] for key, val in res.items()}
+    # permutation of the GPU labels: bit-exact
+    pq, qo = oracle.permute(g["labels_q"], cfg.nQ)
+    pk, ko = oracle.permute(g["labels_k"], cfg.nK)
+    assert np.array_equal(g["perm_q"], pq) and np.array_equal(g["q_off"], qo)
+    assert np.array_equal(g["perm_k"], pk) and np.array_equal(g["k_off"], ko)
+    assert np.array_equal(g["count_q"], np.diff(qo)) and np.array_equal(g["count_k"], np.diff(ko))
+    # centroids are the means of the GPU's final labels (float64 sums rounded to float32)
+    for C, X, lab, kk in ((g["cq"], q, g["labels_q"], cfg.nQ), (g["ck"], k, g["labels_k"], cfg.nK)):
+        Cref, cnt = oracle.update(X, lab, C.astype(np.float64))
+        np.testing.assert_array_equal(C, Cref.astype(np.float32))
+    # selection from the GPU centroids
+    w_ref = oracle.select_weights(g["cq"], g["ck"], g["count_k"], scale)
+    np.testing.assert_allclose(g["weights"], w_ref, rtol=1e-6)
+    mask_ref = oracle.topp(w_ref, g["count_k"], top_p)
+    mism = int((g["mask"] != mask_ref).sum())
+    assert mism <= 2, mism
+    # attention on the GPU's permuted inputs and mask, compared in token order
+    Qp, Kp, Vp = oracle.gather_rows(q, pq), oracle.gather_rows(k, pk), oracle.gather_rows(v, pk)
+    if cfg.dtype == "f32":   # the kernels compute in bf16: the permuted copies are rounded
+        Qp, Kp, Vp = I.round_to_bf16(Qp), I.round_to_bf16(Kp), I.round_to_bf16(Vp)
+    inv = np.empty_like(pq)
+    inv[pq] = np.arange(pq.size, dtype=np.int32)
+    tok = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    ref = oracle.sparse_attention_rows(Qp, Kp, Vp, qo, ko, g["mask"], scale, inv[tok])
+    err = np.abs(g["o"][tok] - ref)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    dens = oracle.density(g["mask"], g["count_q"], g["count_k"])
+    return dict(mask_mismatch=mism, max_abs=float(err.max()), mean_abs=float(err.mean()), density=dens)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg_name", ["tiny", "small"])
+def test_layer_small_configs_every_head(oracle, cfg_name):
+    svg2 = require_gpu()
+    cfg = I.CONFIGS[cfg_name]
+    data = pool_layer_inputs(cfg, range(cfg.H))
+    top_p = cfg.top_p[0]
+    res = run_layer(svg2, cfg, data, top_p)
+    for h in range(cfg.H):
+        st = check_head(oracle, cfg, data, res, h, top_p)
+        e2e = oracle.layer_head(data["q"][0, h], data["k"][0, h], data["v"][0, h], cfg.nQ, cfg.nK, cfg.iters, top_p,
+                                float(np.float32(cfg.scale)), data["uq"][0, h], data["uk"][0, h])
+        agree_q = float((res["labels_q"][0, h] == e2e["labels_q"]).mean())
+        agree_k = float((res["labels_k"][0, h] == e2e["labels_k"]).mean())
+        o_rel = float(np.linalg.norm(res["o"][0, h] - e2e["o"]) / np.linalg.norm(e2e["o"]))
+        print(f"{cfg_name} head {h}: {st}; e2e label agreement q {agree_q:.5f} k {agree_k:.5f}, O rel-L2 {o_rel:.2e}")
+        assert agree_q >= 0.99 and agree_k >= 0.99
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg_name", ["wan720p", "hunyuan720p"])
+def test_layer_full_size_sampled_heads(oracle, cfg_name):
+    svg2 = require_gpu()
+    cfg = I.CONFIGS[cfg_name]
+    data = pool_layer_inputs(cfg, range(cfg.H))
+    top_p = 0.9
+    res = run_layer(svg2, cfg, data, top_p)
+    rng = np.random.default_rng(cfg.cfg_id)
+    for h in (0, cfg.H // 2, cfg.H - 1):
+        rows = np.sort(rng.choice(cfg.N, 384, replace=False))
+        st = check_head(oracle, cfg, data, res, h, top_p, rows)
+        print(f"{cfg_name} head {h}: {st}")
+
+
+@pytest.mark.gpu
+def test_top_p_one_equals_dense_attention():
+    """With every pair kept the permutation cancels (section 4.1): the layer equals dense attention."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS["small"]
+    data = pool_layer_inputs(cfg, range(2))
+    res = run_layer(svg2, cfg, data, 1.0)
+    q, k, v = (torch.from_numpy(data[n]).cuda() for n in ("q", "k", "v"))
+    dense = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=float(np.float32(cfg.scale)))
+    err = np.abs(res["o"] - dense.cpu().numpy())
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+
+
+@pytest.mark.gpu
+def test_unfused_and_fused_inverse_permutation_agree():
+    svg2 = require_gpu()
+    cfg = I.CONFIGS["small"]
+    data = pool_layer_inputs(cfg, range(2))
+    a = run_layer(svg2, cfg, data, 0.9, fuse=1)
+    b = run_layer(svg2, cfg, data, 0.9, fuse=0)
+    np.testing.assert_array_equal(a["o"], b["o"])
+
+
+@pytest.mark.gpu
+def test_warm_start_sequence_tracks_cold_start(oracle):
+    """Centroid cache across denoising steps (section 4.3, Fig. 7(a)): warm start from the previous
+    step's centroids with 2 iterations stays close to dense attention like a cold start does."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS["small"]
+    heads = range(2)
+    d0 = pool_layer_inputs(cfg, heads, 0)
+    r0 = run_layer(svg2, cfg, d0, 0.9)
+    cq, ck = torch.from_numpy(r0["cq"]).cuda(), torch.from_numpy(r0["ck"]).cuda()
+    warm_cfg = I.LayerConfig(**{**cfg.__dict__, "iters": 2, "drift": 0.05})
+    for step in (1, 2):
+        ds = pool_layer_inputs(I.CONFIGS["small"], heads, 0)
+        eps = np.random.default_rng(step).standard_normal(ds["q"].shape, dtype=np.float32)
+        ds["q"] = I.round_to_bf16(ds["q"] + 0.05 * step * eps)
+        ds["k"] = I.round_to_bf16(ds["k"] + 0.05 * step * eps[:, :, ::-1])
+        warm = run_layer(svg2, warm_cfg, ds, 0.9, init=svg2.SVG2_INIT_GIVEN, cq=cq.clone(), ck=ck.clone())
+        cold = run_layer(svg2, cfg, ds, 0.9)
+        for h in heads:
+            check_head(oracle, warm_cfg, ds, warm, h, 0.9, rows=np.arange(0, cfg.N, 97))
+        q, k, v = (torch.from_numpy(ds[n]).cuda() for n in ("q", "k", "v"))
+        dense = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=float(np.float32(cfg.scale))).cpu().numpy()
+        e_w = np.linalg.norm(warm["o"] - dense) / np.linalg.norm(dense)
+        e_c = np.linalg.norm(cold["o"] - dense) / np.linalg.norm(dense)
+        print(f"step {step}: rel-L2 vs dense warm {e_w:.4f} cold {e_c:.4f}")
+        assert e_w <= 1.5 * e_c + 0.02
+        cq, ck = torch.from_numpy(warm["cq"]).cuda(), torch.from_numpy(warm["ck"]).cuda()
