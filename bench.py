@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="run only this many heads of the layer (profiling cases)")
     return ap.parse_args()
 
 
@@ -172,6 +173,9 @@ class ClockSampler:
 def main():
     args = parse()
     cfg = I.CONFIGS[args.config]
+    if args.heads:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, H=args.heads)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -186,6 +186,278 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// k-means++ on a cluster of kPpCtas CTAs per (b,h): each CTA keeps D^2 (float64) and the nearest
+// seed (uint16) of its token range in shared memory; warps read token rows cooperatively (each lane
+// d/32 consecutive values, so one warp load covers a row); per seed, the CTAs exchange their
+// fixed-point weight totals through distributed shared memory and the CTA holding the sampling
+// target finds the token.  The float64 D^2 of a token is summed per lane over its values and then
+// across lanes in a fixed butterfly order; it can differ from a sequential sum in the last bit,
+// which moves the fixed-point weight floor(D^2 / M0 * 2^32) only when D^2 / M0 * 2^32 lies within
+// ~1e-6 of an integer, and changes a pick only if the sampling target sits exactly on that step.
+// ------------------------------------------------------------------------------------------------
+constexpr int kPpCtas = 8;
+constexpr int kPpThreads = 1024;
+constexpr int kPpWarps = kPpThreads / 32;
+constexpr int kPpMaxTokensPerCta = 15360;   // 10 bytes of state per token: 150 KB of shared memory
+
+__host__ __device__ constexpr size_t pp_smem_bytes(int per_cta) {
+  return static_cast<size_t>(per_cta) * 10 + 16;
+}
+
+template <int E, bool F32>
+__device__ __forceinline__ void pp_load_row(const void* X, size_t row_elem, int lane, float (&v)[E]) {
+  if constexpr (F32) {
+    const float* p = static_cast<const float*>(X) + row_elem + lane * E;
+    if constexpr (E == 4) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else {
+      const float2 a = __ldg(reinterpret_cast<const float2*>(p));
+      v[0] = a.x; v[1] = a.y;
+    }
+  } else {
+    const unsigned short* p = static_cast<const unsigned short*>(X) + row_elem + lane * E;
+    if constexpr (E == 4) {
+      const uint2 a = __ldg(reinterpret_cast<const uint2*>(p));
+      v[0] = bf16lo_to_f32(a.x); v[1] = bf16hi_to_f32(a.x); v[2] = bf16lo_to_f32(a.y); v[3] = bf16hi_to_f32(a.y);
+    } else {
+      const uint32_t a = __ldg(reinterpret_cast<const uint32_t*>(p));
+      v[0] = bf16lo_to_f32(a); v[1] = bf16hi_to_f32(a);
+    }
+  }
+}
+
+template <int E>
+__device__ __forceinline__ double pp_exact(const float (&v)[E], const float* cs, int lane) {
+  double acc = 0.0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const double df = __dsub_rn(static_cast<double>(v[e]), static_cast<double>(cs[lane * E + e]));
+    acc = __dadd_rn(acc, __dmul_rn(df, df));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+  return __shfl_sync(0xffffffffu, acc, 0);  // lane 0's summation order decides
+}
+
+template <int E, bool F32>
+__global__ void __cluster_dims__(kPpCtas, 1, 1) __launch_bounds__(kPpThreads, 1)
+    kmeanspp_cluster_kernel(const void* __restrict__ X, int N, int k, const double* __restrict__ u,
+                            float* __restrict__ C) {
+  constexpr int D = E * 32;
+  constexpr int kBatch = 8;  // token rows in flight per warp
+  extern __shared__ uint8_t pp_smem[];
+  __shared__ float cs[D];
+  __shared__ float ss[1024];
+  __shared__ unsigned long long wsum[kPpWarps];
+  __shared__ unsigned long long cta_tot[kPpCtas];
+  __shared__ double cta_max[kPpCtas];
+  __shared__ unsigned long long pick_bcast;
+  __shared__ unsigned long long hit_base;
+  __shared__ int hit_warp;
+  const uint32_t rank = cluster_rank();
+  const int bh = blockIdx.x / kPpCtas;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_cta = (N + kPpCtas - 1) / kPpCtas;
+  const int lo = min(N, static_cast<int>(rank) * per_cta), hi = min(N, lo + per_cta);
+  const int per_warp = (hi - lo + kPpWarps - 1) / kPpWarps;
+  const int wlo = min(hi, lo + warp * per_warp), whi = min(hi, wlo + per_warp);
+  double* Ds = reinterpret_cast<double*>(pp_smem);
+  uint16_t* As = reinterpret_cast<uint16_t*>(pp_smem + static_cast<size_t>(per_cta) * 8);
+  const size_t xbase = static_cast<size_t>(bh) * N * D;
+  float* Ch = C + static_cast<size_t>(bh) * k * D;
+  const double* uh = u + static_cast<size_t>(bh) * k;
+
+  auto load_seed = [&](int p, int s) {
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      float v;
+      if constexpr (F32) v = static_cast<const float*>(X)[xbase + static_cast<size_t>(p) * D + i];
+      else v = bf16lo_to_f32(static_cast<const unsigned short*>(X)[xbase + static_cast<size_t>(p) * D + i]);
+      cs[i] = v;
+      if (rank == 0) Ch[static_cast<size_t>(s) * D + i] = v;
+    }
+  };
+
+  unsigned long long qsum = 0ull;  // this warp's total fixed-point weight (held by lane 0)
+  double M0 = 0.0;
+
+  // Lower D^2 of this warp's tokens with seed s (already in cs; ss holds seed-to-seed distances).
+  auto update_pass = [&](int s, bool first) {
+    for (int tb = wlo; tb < whi; tb += 32) {
+      const int t = tb + lane;
+      double Dt = INFINITY;
+      bool cand = false;
+      if (t < whi) {
+        if (first) {
+          cand = true;
+        } else {
+          Dt = Ds[t - lo];
+          cand = static_cast<double>(ss[As[t - lo]]) < 4.0001 * Dt;  // else provably not closer
+        }
+      }
+      unsigned m = __ballot_sync(0xffffffffu, cand);
+      while (m) {
+        int tl[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          tl[i] = m ? __ffs(m) - 1 : -1;
+          if (m) m &= m - 1;
+        }
+        float part[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          part[i] = 0.f;
+          if (tl[i] >= 0) {
+            float v[E];
+            pp_load_row<E, F32>(X, xbase + static_cast<size_t>(tb + tl[i]) * D, lane, v);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              const float df = v[e] - cs[lane * E + e];
+              part[i] = fmaf(df, df, part[i]);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          if (tl[i] < 0) continue;                                        // warp-uniform
+          const float f = __shfl_sync(0xffffffffu, part[i], 0);            // one value for the warp
+          const double Di = __shfl_sync(0xffffffffu, Dt, tl[i]);
+          if (!first && static_cast<double>(f) > Di * (1.0 + 1e-3)) continue;  // float32 error << 1e-3
+          float v[E];
+          pp_load_row<E, F32>(X, xbase + static_cast<size_t>(tb + tl[i]) * D, lane, v);
+          const double nd = pp_exact<E>(v, cs, lane);
+          if (nd < Di && lane == 0) {
+            if (!first) {
+              qsum -= fixed_weight(Di, M0);
+              qsum += fixed_weight(nd, M0);
+            }
+            Ds[tb + tl[i] - lo] = nd;
+            As[tb + tl[i] - lo] = static_cast<uint16_t>(s);
+          }
+        }
+      }
+    }
+  };
+
+  // ---- seed 0, the initial D^2 and the fixed-point scale M0 (cluster-wide maximum)
+  long long p0 = static_cast<long long>(floor(uh[0] * static_cast<double>(N)));
+  if (p0 >= N) p0 = N - 1;
+  if (p0 < 0) p0 = 0;
+  load_seed(static_cast<int>(p0), 0);
+  __syncthreads();
+  update_pass(0, true);
+  __syncwarp();
+  double lmax = 0.0;
+  for (int t = wlo + lane; t < whi; t += 32) lmax = fmax(lmax, Ds[t - lo]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  if (lane == 0) wsum[warp] = static_cast<unsigned long long>(__double_as_longlong(lmax));
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double mx = 0.0;
+    for (int w = 0; w < kPpWarps; ++w) mx = fmax(mx, __longlong_as_double(static_cast<long long>(wsum[w])));
+    for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_f64(&cta_max[rank], r, mx);
+  }
+  cluster_sync();
+  for (int r = 0; r < kPpCtas; ++r) M0 = fmax(M0, cta_max[r]);
+  if (lane == 0)
+    for (int t = wlo; t < whi; ++t) qsum += fixed_weight(Ds[t - lo], M0);
+
+  for (int s = 1; s < k; ++s) {
+    // ---- totals: warps -> CTA -> every CTA of the cluster
+    if (lane == 0) wsum[warp] = qsum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned long long t = 0;
+      for (int w = 0; w < kPpWarps; ++w) t += wsum[w];
+      for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_u64(&cta_tot[rank], r, t);
+    }
+    cluster_sync();
+    unsigned long long U = 0, base = 0;
+    for (int r = 0; r < kPpCtas; ++r) {
+      if (r < static_cast<int>(rank)) base += cta_tot[r];
+      U += cta_tot[r];
+    }
+    if (U == 0ull) {
+      if (threadIdx.x == 0 && rank == 0) {
+        const long long p = static_cast<long long>(floor(uh[s] * static_cast<double>(N)));
+        const unsigned long long pk = static_cast<unsigned long long>(p >= N ? N - 1 : p);
+        for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_u64(&pick_bcast, r, pk);
+      }
+    } else {
+      unsigned long long target = static_cast<unsigned long long>(floor(uh[s] * static_cast<double>(U)));
+      if (target > U - 1ull) target = U - 1ull;
+      const unsigned long long mine = cta_tot[rank];
+      if (mine > 0ull && base <= target && target < base + mine) {  // block-uniform
+        if (threadIdx.x == 0) {
+          unsigned long long run = base;
+          int w = 0;
+          for (; w < kPpWarps - 1; ++w) {
+            if (target < run + wsum[w]) break;
+            run += wsum[w];
+          }
+          hit_warp = w;
+          hit_base = run;
+        }
+        __syncthreads();
+        if (warp == hit_warp) {
+          // lanes split the warp's tokens into contiguous pieces; scan the piece sums
+          const int piece = (whi - wlo + 31) / 32;
+          const int plo = min(whi, wlo + lane * piece), phi = min(whi, plo + piece);
+          unsigned long long ps = 0;
+          for (int t = plo; t < phi; ++t) ps += fixed_weight(Ds[t - lo], M0);
+          unsigned long long incl = ps;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          unsigned long long run = hit_base + incl - ps;
+          if (ps > 0ull && run <= target && target < run + ps) {
+            int pk = phi - 1;
+            for (int t = plo; t < phi; ++t) {
+              run += fixed_weight(Ds[t - lo], M0);
+              if (run > target) {
+                pk = t;
+                break;
+              }
+            }
+            for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_u64(&pick_bcast, r, static_cast<unsigned long long>(pk));
+          }
+        }
+      }
+    }
+    cluster_sync();
+    const int p = static_cast<int>(pick_bcast);
+    load_seed(p, s);
+    __syncthreads();
+    // ---- squared distances from the new seed to every earlier seed (float32, for pruning)
+    for (int a = threadIdx.x; a < s; a += blockDim.x) {
+      const float* ca = Ch + static_cast<size_t>(a) * D;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < D; i += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(ca + i);
+        const float d0 = cs[i] - c4.x, d1 = cs[i + 1] - c4.y, d2 = cs[i + 2] - c4.z, d3 = cs[i + 3] - c4.w;
+        acc = fmaf(d0, d0, acc);
+        acc = fmaf(d1, d1, acc);
+        acc = fmaf(d2, d2, acc);
+        acc = fmaf(d3, d3, acc);
+      }
+      ss[a] = acc;
+    }
+    __syncthreads();
+    update_pass(s, false);
+    __syncthreads();
+  }
+  cluster_sync();  // no CTA leaves while another may still write into its shared memory
+}
+
 // Split float32 centroids into bf16 hi + lo parts, zero the padding rows, compute ||c||^2.
 __global__ void centroid_prep_kernel(const float* __restrict__ C, int BH, int k, int kpad, int d,
                                      uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
@@ -254,7 +526,8 @@ __global__ void __launch_bounds__(128) assign_exact_kernel(const void* __restric
 constexpr int kAsgThreads = 256;
 constexpr uint32_t kAsgXStage = 32768;   // 128 tokens x 128 d bf16 (two 16 KB halves)
 constexpr uint32_t kAsgCStage = 65536;   // 128 centroids x 128 d x {hi, lo}
-constexpr uint32_t kAsgSmem = 2 * kAsgXStage + 2 * kAsgCStage + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t kAsgSmem = 2 * kAsgXStage + 2 * kAsgCStage + 1024 /*align*/ + 256 /*barriers*/ +
+                               4 * 128 * 4 /*norms*/ + 128 * 33 * 4 /*scratch*/;
 constexpr uint32_t kAsgTmemCols = 512;   // 4 accumulators of 128 columns
 
 struct AsgBars {
@@ -445,34 +718,80 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: argmin over centroids ----------------
+    // Per 32-column group: scores s = ||c||^2 - 2 x.c (no branches), the group minimum, then a bit
+    // mask of the columns within tau of the running minimum; columns in the mask (rare: the
+    // minimum itself and near-ties) go through shared scratch into a 4-entry candidate list.
+    // tau = 2^-11 (||x||^2 + max(d_min, 0)) is >= 3x the bound on the split-bf16 score error
+    // 2^-15 (5 ||x||^2 + 2 d_min), so the true argmin is always among the candidates; when more
+    // than one candidate survives, exact float32 ||x - c||^2 decides (ties to the lower index).
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int et = threadIdx.x - 128;  // 0..127
+    float* cn_s = reinterpret_cast<float*>(bars + 1);          // [4][128] staged norms
+    float* scr = cn_s + 4 * 128 + et * 33;                     // per-thread scratch, 32 scores
     long long g = 0;
     int it = 0;
     bool ok = true;
     for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
       const int bh = static_cast<int>(w / ntiles), tile = static_cast<int>(w % ntiles);
       const int xsI = it & 1;
-      float s1 = INFINITY, s2 = INFINITY, s3 = INFINITY;
-      int i1 = 0, i2 = -1, i3 = -1;
       const float* cn = c_norm + static_cast<size_t>(bh) * kpad;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssignTail));
+      if (!ok) break;
+      const uint8_t* xt = xs + xsI * kAsgXStage;
+      const float xn = tile_row_norm(xt, row);
+      float gmin = INFINITY;
+      float cv[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+      int ci[4] = {-1, -1, -1, -1};
       for (int c = 0; c < nchunks; ++c, ++g) {
         const int a = static_cast<int>(g & 3);
+        cn_s[a * 128 + et] = __ldg(cn + c * kAssignChunkN + et);
+        asm volatile("bar.sync 2, 128;" ::: "memory");
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full[a]), (g >> 2) & 1, st, kWhereAssign));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
         for (int qq = 0; qq < 4; ++qq) {
+          const int jb = c * kAssignChunkN + qq * 32;
+          if (jb >= k) break;  // uniform
           uint32_t v[32];
           tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kAssignChunkN + qq * 32, v);
           tmem_wait_ld();
-          const int jb = c * kAssignChunkN + qq * 32;
+          const float* cnq = cn_s + a * 128 + qq * 32;
+          float sc[32];
+          float mloc = INFINITY;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int j = jb + e;
-            if (j < k) {
-              const float s = fmaf(-2.f, __uint_as_float(v[e]), __ldg(cn + j));
-              top3_insert(s, j, s1, i1, s2, i2, s3, i3);
+            sc[e] = fmaf(-2.f, __uint_as_float(v[e]), cnq[e]);
+            if (jb + 32 > k && jb + e >= k) sc[e] = INFINITY;
+            mloc = fminf(mloc, sc[e]);
+          }
+          gmin = fminf(gmin, mloc);
+          const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
+          unsigned hits = 0;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) hits |= (sc[e] <= thr ? 1u : 0u) << e;
+          if (hits) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) scr[e] = sc[e];
+            while (hits) {
+              const int e = __ffs(hits) - 1;
+              hits &= hits - 1;
+              const float val = scr[e];
+              // replace the worst candidate if this one is better (strictly: ties keep the earlier,
+              // i.e. lower, index)
+              int wi = 0;
+#pragma unroll
+              for (int r = 1; r < 4; ++r)
+                if (cv[r] > cv[wi]) wi = r;
+              if (val < cv[wi]) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                  if (r == wi) {
+                    cv[r] = val;
+                    ci[r] = jb + e;
+                  }
+              }
             }
           }
         }
@@ -481,34 +800,36 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[a]));
       }
       if (!ok) break;
-      // the X tile is still resident (its stage is released only after this epilogue arrives)
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssignTail));
-      if (!ok) break;
       const int n = tile * kAssignTileM + row;
       if (n < N) {
-        int best = i1;
-        if (i2 >= 0) {
-          const uint8_t* xt = xs + xsI * kAsgXStage;
-          const float xn = tile_row_norm(xt, row);
-          const float tau = ldexpf(xn + fmaxf(__ldg(cn + i1), __ldg(cn + i2)), -10);
-          if (s2 - s1 < tau) {
-            const float* Cb = C + static_cast<size_t>(bh) * k * 128;
-            float bd = tile_row_dist(xt, row, Cb + static_cast<size_t>(i1) * 128);
-            const float d2 = tile_row_dist(xt, row, Cb + static_cast<size_t>(i2) * 128);
-            if (d2 < bd || (d2 == bd && i2 < best)) {
-              bd = d2;
-              best = i2;
-            }
-            if (i3 >= 0 && s3 - s1 < tau) {
-              const float d3 = tile_row_dist(xt, row, Cb + static_cast<size_t>(i3) * 128);
-              if (d3 < bd || (d3 == bd && i3 < best)) {
-                bd = d3;
-                best = i3;
-              }
+        const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
+        int best = -1, nc = 0;
+        float bv = INFINITY;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if (ci[r] >= 0 && cv[r] <= thr) {
+            ++nc;
+            if (cv[r] < bv || (cv[r] == bv && ci[r] < best)) {
+              bv = cv[r];
+              best = ci[r];
             }
           }
         }
-        labels[static_cast<size_t>(bh) * N + n] = best;
+        if (nc > 1) {
+          const float* Cb = C + static_cast<size_t>(bh) * k * 128;
+          float bd = INFINITY;
+          best = -1;
+#pragma unroll 1
+          for (int r = 0; r < 4; ++r) {
+            if (ci[r] < 0 || cv[r] > thr) continue;
+            const float dd = tile_row_dist(xt, row, Cb + static_cast<size_t>(ci[r]) * 128);
+            if (dd < bd || (dd == bd && ci[r] < best)) {
+              bd = dd;
+              best = ci[r];
+            }
+          }
+        }
+        labels[static_cast<size_t>(bh) * N + n] = best < 0 ? 0 : best;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->x_empty[xsI]));
@@ -526,70 +847,91 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
 // ------------------------------------------------------------------------------------------------
 // Update: centroid = mean of members (float64, ascending token order)
 // ------------------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) update_kernel(const void* __restrict__ X, bool f32, int BH, int N, int k,
-                                                      int kpad, const int32_t* __restrict__ perm,
-                                                      const int32_t* __restrict__ offsets,
-                                                      float* __restrict__ C, uint16_t* __restrict__ hi,
-                                                      uint16_t* __restrict__ lo, float* __restrict__ norm) {
-  constexpr int E = D / 32;  // dims per lane
-  const int lane = threadIdx.x & 31;
-  const long long wid = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
-  if (wid >= static_cast<long long>(BH) * k) return;
-  const int bh = static_cast<int>(wid / k), j = static_cast<int>(wid % k);
+// One CTA per (b,h, cluster).  Member rows (in the stable sort's order) are staged through shared
+// memory with cp.async, kUpdRows rows per batch, double-buffered; thread i < d sums dimension i
+// over the batch sequentially in float64, which is the oracle's order, so the sums match it bit
+// for bit.  Then c = float32(sum / count), the bf16 hi/lo split and ||c||^2.
+constexpr int kUpdBufBytes = 16384;  // per buffer: 64 bf16 rows of d = 128
+constexpr int kUpdThreads = 256;
+
+template <int D, bool F32>
+__global__ void __launch_bounds__(kUpdThreads) update_kernel(const void* __restrict__ X, int BH, int N, int k,
+                                                              int kpad, const int32_t* __restrict__ perm,
+                                                              const int32_t* __restrict__ offsets,
+                                                              float* __restrict__ C, uint16_t* __restrict__ hi,
+                                                              uint16_t* __restrict__ lo, float* __restrict__ norm) {
+  constexpr int ESZ = F32 ? 4 : 2;
+  constexpr int ROWB = D * ESZ;                 // bytes per row
+  constexpr int CH = ROWB / 16;                 // 16-byte chunks per row
+  constexpr int kUpdRows = kUpdBufBytes / ROWB; // rows per batch
+  __shared__ __align__(16) uint8_t buf[2][kUpdBufBytes];
+  __shared__ float red[kUpdThreads / 32];
+  const int bh = blockIdx.x / k, j = blockIdx.x % k;
   const int o0 = offsets[static_cast<size_t>(bh) * (k + 1) + j];
   const int o1 = offsets[static_cast<size_t>(bh) * (k + 1) + j + 1];
   const int cnt = o1 - o0;
+  const int tid = threadIdx.x;
   float* cj = C + (static_cast<size_t>(bh) * k + j) * D;
-  float c[E];
-  if (cnt > 0) {
-    double acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.0;
-    const int32_t* pr = perm + static_cast<size_t>(bh) * N;
-    const size_t xb = static_cast<size_t>(bh) * N * D + lane * E;
-    int r = o0;
-    constexpr int U = 8;
-    for (; r + U <= o1; r += U) {
-      float xv[U][E];
-#pragma unroll
-      for (int uu = 0; uu < U; ++uu) {
-        const size_t ro = xb + static_cast<size_t>(__ldg(pr + r + uu)) * D;
-#pragma unroll
-        for (int e = 0; e < E; ++e) xv[uu][e] = ld_elem(X, ro + e, f32);
+  const int32_t* pr = perm + static_cast<size_t>(bh) * N;
+  const char* xb = static_cast<const char*>(X) + static_cast<size_t>(bh) * N * ROWB;
+  auto issue = [&](int batch, int b) {
+    const int r0 = o0 + batch * kUpdRows;
+    const int nr = min(kUpdRows, o1 - r0);
+    for (int q = tid; q < nr * CH; q += kUpdThreads) {
+      const int r = q / CH, c = q - r * CH;
+      int t = __ldg(pr + r0 + r);
+      t = t < 0 ? 0 : (t >= N ? N - 1 : t);
+      cp_async16(smem_u32(&buf[b][r * ROWB + c * 16]), xb + static_cast<size_t>(t) * ROWB + c * 16);
+    }
+    cp_async_commit();
+  };
+  double acc = 0.0;
+  const int nb = (cnt + kUpdRows - 1) / kUpdRows;
+  if (nb > 0) issue(0, 0);
+  for (int b = 0; b < nb; ++b) {
+    if (b + 1 < nb) {
+      issue(b + 1, (b + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (tid < D) {
+      const int nr = min(kUpdRows, cnt - b * kUpdRows);
+      const uint8_t* src = buf[b & 1];
+      for (int r = 0; r < nr; ++r) {
+        float x;
+        if constexpr (F32) x = reinterpret_cast<const float*>(src + r * ROWB)[tid];
+        else x = bf16lo_to_f32(reinterpret_cast<const uint16_t*>(src + r * ROWB)[tid]);
+        acc = __dadd_rn(acc, static_cast<double>(x));
       }
-#pragma unroll
-      for (int uu = 0; uu < U; ++uu)
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = __dadd_rn(acc[e], static_cast<double>(xv[uu][e]));
     }
-    for (; r < o1; ++r) {
-      const size_t ro = xb + static_cast<size_t>(__ldg(pr + r)) * D;
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = __dadd_rn(acc[e], static_cast<double>(ld_elem(X, ro + e, f32)));
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      c[e] = static_cast<float>(__ddiv_rn(acc[e], static_cast<double>(cnt)));
-      cj[lane * E + e] = c[e];
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < E; ++e) c[e] = cj[lane * E + e];
+    __syncthreads();
   }
-  float nrm = 0.f;
-  const size_t ro = (static_cast<size_t>(bh) * kpad + j) * D + lane * E;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(c[e]);
-    const __nv_bfloat16 l = __float2bfloat16_rn(c[e] - __bfloat162float(h));
-    hi[ro + e] = __bfloat16_as_ushort(h);
-    lo[ro + e] = __bfloat16_as_ushort(l);
-    nrm = fmaf(c[e], c[e], nrm);
+  float c = 0.f;
+  if (tid < D) {
+    if (cnt > 0) {
+      c = static_cast<float>(__ddiv_rn(acc, static_cast<double>(cnt)));
+      cj[tid] = c;
+    } else {
+      c = cj[tid];
+    }
+    const size_t ro = (static_cast<size_t>(bh) * kpad + j) * D + tid;
+    const __nv_bfloat16 h = __float2bfloat16_rn(c);
+    const __nv_bfloat16 l = __float2bfloat16_rn(c - __bfloat162float(h));
+    hi[ro] = __bfloat16_as_ushort(h);
+    lo[ro] = __bfloat16_as_ushort(l);
   }
+  float nrm = c * c;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
-  if (lane == 0) norm[static_cast<size_t>(bh) * kpad + j] = nrm;
+  if ((tid & 31) == 0) red[tid >> 5] = nrm;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < D / 32; ++w) t += red[w];
+    norm[static_cast<size_t>(bh) * kpad + j] = t;
+  }
 }
 
 int num_sms() {
@@ -601,8 +943,26 @@ int num_sms() {
 
 }  // namespace
 
+template <int E, bool F32>
+cudaError_t launch_pp_cluster(const void* X, int BH, int N, int k, const double* u, float* C, cudaStream_t s) {
+  const int per_cta = (N + kPpCtas - 1) / kPpCtas;
+  const size_t smem = pp_smem_bytes(per_cta);
+  cudaError_t e = cudaFuncSetAttribute(kmeanspp_cluster_kernel<E, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kmeanspp_cluster_kernel<E, F32><<<BH * kPpCtas, kPpThreads, smem, s>>>(X, N, k, u, C);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
                             float* centroids, double* dist, int32_t* near, cudaStream_t s) {
+  const int per_cta = (N + kPpCtas - 1) / kPpCtas;
+  if (per_cta <= kPpMaxTokensPerCta) {
+    if (d == 128) return x_f32 ? launch_pp_cluster<4, true>(X, BH, N, k, u, centroids, s)
+                               : launch_pp_cluster<4, false>(X, BH, N, k, u, centroids, s);
+    return x_f32 ? launch_pp_cluster<2, true>(X, BH, N, k, u, centroids, s)
+                 : launch_pp_cluster<2, false>(X, BH, N, k, u, centroids, s);
+  }
   kmeanspp_kernel<<<BH, 1024, 0, s>>>(X, x_f32, N, d, k, u, centroids, dist, near);
   return cudaGetLastError();
 }
@@ -641,13 +1001,19 @@ cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k
 cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
                           const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
                           float* c_norm, cudaStream_t s) {
-  const long long warps = static_cast<long long>(BH) * k;
-  const int blocks = static_cast<int>((warps * 32 + 255) / 256);
+  const int blocks = BH * k;
   const int kp = kpad_of(k);
-  if (d == 128)
-    update_kernel<128><<<blocks, 256, 0, s>>>(X, x_f32, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
-  else
-    update_kernel<64><<<blocks, 256, 0, s>>>(X, x_f32, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+  if (d == 128) {
+    if (x_f32)
+      update_kernel<128, true><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+    else
+      update_kernel<128, false><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+  } else {
+    if (x_f32)
+      update_kernel<64, true><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+    else
+      update_kernel<64, false><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+  }
   return cudaGetLastError();
 }
 
