@@ -121,6 +121,21 @@ def config_dict(cfg, top_p):
             "parallelism": "replicas"}
 
 
+def max_over_ranks(value: float, world: int, dist, device) -> float:
+    """The slowest rank's time (a multi-GPU number is the max over ranks, never one rank's clock)."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_ms_per_layer(ms_per_step: float, world: int) -> float:
+    """Weak scaling with one layer per rank per step: the job finishes `world` layers per step."""
+    return ms_per_step / world
+
+
 # ------------------------------------------------------------------------------------------ clocks
 class ClockSampler:
     def __init__(self, index):
@@ -269,11 +284,7 @@ def main():
     if world > 1:
         dist.barrier()
     svg2.raise_on_device_error(ws)
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dist, dev)
     ms_per_step = total_ms / args.steps
     stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
     attn_ms = stage_ms["sparse_attn"]
@@ -300,7 +311,7 @@ def main():
                           f"of {cfg.N} rows; extrapolated to the layer"), "parts_s": parts}
     launches = kernel_launches(cfg)
     line = {
-        "metric": METRIC, "value": ms_per_step / world, "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": whole_job_ms_per_layer(ms_per_step, world), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.top_p),
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel", "achieved": achieved_tflops,
@@ -359,13 +370,9 @@ def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
     b.record()
     torch.cuda.synchronize(dev)
     svg2.raise_on_device_error(ws)
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dist, dev)
     h2d = 3 * hq.numel() * 2 + (huq.numel() + huk.numel()) * 8
-    return {"value": ms / world, "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
+    return {"value": whole_job_ms_per_layer(ms, world), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
             "steps": steps, "api": "svg2_layer"}
 
 
