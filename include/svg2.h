@@ -185,6 +185,27 @@ SVG2_API int svg2_layer(const void* Q, const void* K, const void* V, int dtype, 
                const svg2_layer_outputs* outs, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * svg2_sparse_attn without a workspace, for callers that cannot allocate device memory at call
+ * time (no cudaMalloc and no caching allocator available to them, e.g. code that must not grow
+ * its memory footprint once running).  The paper has no counterpart; this is an interface
+ * convenience.  Same inputs, outputs and semantics as svg2_sparse_attn, but its scratch — the
+ * attention work plan and a status word — is a fixed 1 MiB array inside the library, which every
+ * GPU that loads the library keeps until the process exits.  Sizes whose plan needs more than that
+ * (about B*H*(ceil(N/256) + nQ) * 16 bytes plus a few KB) return SVG2_ERR_UNSUPPORTED.
+ * The call allocates nothing.  Its first call on a device looks up the array's device address
+ * (once per device, with that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents, so calls whose kernels
+ * may overlap on the GPU (different streams, or other threads) race: serialise them.
+ *   device_status  optional 16-byte, 16-byte-aligned caller-owned device word that must start at
+ *                  zero; device-side errors (SVG2_ERR_DEVICE_*) are latched there.  If NULL, the
+ *                  library's own word is used (cleared at every call) and such errors are not
+ *                  reported to the caller. */
+SVG2_API int svg2_sparse_attn_noalloc(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
+                                      const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx,
+                                      int B, int H, int N, int d, int nQ, int nK, float scale,
+                                      const int32_t* perm_q, void* O, uint32_t* device_status, void* stream);
+
+/*
  * Self-test of the tensor-core building blocks (not part of the method): C = A * B^T for
  * bf16 A [128, 128] and B [n, 128] (n in {64, 128, 256}), loaded by TMA with 128-byte swizzle,
  * multiplied by tcgen05.mma into TMEM (float32); then P = bf16(C[:, :128]) is written back to

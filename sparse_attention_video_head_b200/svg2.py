@@ -22,7 +22,7 @@ MAX_CLUSTERS = 1024
 
 _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeans", "svg2_select",
             "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
-            "svg2_unpermute", "svg2_layer", "svg2_selftest_mma")
+            "svg2_unpermute", "svg2_layer", "svg2_selftest_mma", "svg2_sparse_attn_noalloc")
 
 _lib = None
 
@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.svg2_layer.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(SvgParams), P, P, P, P, P,
                                  ctypes.POINTER(SvgLayerOutputs), P, S, P]
         L.svg2_selftest_mma.argtypes = [P, P, I, P, P, P, P, S, P]
+        L.svg2_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
         for name in _EXPORTS:
             if name != "svg2_status_string":
                 getattr(L, name).restype = I
@@ -188,6 +189,19 @@ def svg2_sparse_attn(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off
     _check(lib().svg2_sparse_attn(_p(Qp), _p(Kp), _p(Vp), _p(q_off), _p(k_off), _p(sel_count), _p(sel_idx), B, H, N,
                                   d, nQ, nK, float(scale), _p(perm_q), _p(O), _p(ws), ws.numel(), _stream(stream)),
            "svg2_sparse_attn")
+
+
+def svg2_sparse_attn_noalloc(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off: torch.Tensor,
+                             k_off: torch.Tensor, sel_count: torch.Tensor, sel_idx: torch.Tensor, scale: float,
+                             O: torch.Tensor, perm_q: Optional[torch.Tensor] = None,
+                             device_status: Optional[torch.Tensor] = None, stream=None):
+    """svg2_sparse_attn for callers that cannot allocate: scratch is the library's fixed array."""
+    B, H, N, d = Qp.shape
+    nQ = q_off.shape[-1] - 1
+    nK = k_off.shape[-1] - 1
+    _check(lib().svg2_sparse_attn_noalloc(_p(Qp), _p(Kp), _p(Vp), _p(q_off), _p(k_off), _p(sel_count), _p(sel_idx),
+                                          B, H, N, d, nQ, nK, float(scale), _p(perm_q), _p(O), _p(device_status),
+                                          _stream(stream)), "svg2_sparse_attn_noalloc")
 
 
 def svg2_unpermute(Op: torch.Tensor, perm: torch.Tensor, O: torch.Tensor, stream=None):
