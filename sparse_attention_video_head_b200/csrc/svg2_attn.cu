@@ -11,6 +11,7 @@
 //               the 128-byte-swizzled layout the tensor core reads (two stages)
 //   warp 12     Q tiles by TMA, then the single-thread MMA issuer
 //   warp 13     TMEM allocator (512 columns: S_A, S_B, O_A, O_B; P overwrites S as bf16)
+// Registers are re-split after set-up: the softmax warpgroups take 192 per thread, the others 64.
 // MMA order per key tile j: PV_A(j-1) -> S_A(j) -> PV_B(j-1) -> S_B(j).  Because tcgen05 ops of
 // one thread complete in order, "S_X(j) done" also means "O_X holds every PV up to j-1", so the
 // softmax warps rescale O_X in TMEM (only when the row max grows by more than 2^8) before
@@ -35,6 +36,9 @@ template <int D>
 constexpr uint32_t attn_smem() { return 6 * tile_bytes<D>() + 1024 /*align*/ + 4096 /*ranges*/ + 4096 + 64 /*cum*/ + 256; }
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 32 scores of a row, this many (the last ones) get 2^x from a polynomial on the FMA pipe
+// instead of the MUFU, which would otherwise bound the softmax.
+constexpr int kEmuPerChunk = 12;
 
 struct AttnBars {
   uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], o_full, mma_done;
@@ -193,9 +197,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nranges = bars->nranges;
   const int nt = (L + 127) / 128;
 
-  if (warp == 12) {
+  // Warpgroups 0-1 (softmax) take registers from warpgroups 2-3 (producer; MMA, allocator):
+  // 256 x 192 + 256 x 64 = 512 x 128, the launch's allocation.
+  if (warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
     // ---------------- Q by TMA, then MMA issue ----------------
-    if (elect_one()) {
+    if (warp == 12 && elect_one()) {
       prefetch_tensormap(&tm_q);
       const uint32_t qbar = smem_u32(&bars->q_full);
       const uint32_t qa = smem_u32(q_s), qb = smem_u32(q_s + kTile);
@@ -275,17 +282,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(smem_u32(&bars->mma_done), 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
       if (!ok) mbar_wait(qbar, 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
     }
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
     // ---------------- key/value gather producer ----------------
-    const int r = threadIdx.x - 256;
+    // Warp w fills rows 32w..32w+31 of each key tile.  Each lane first finds the source row of one
+    // stream position; then every cp.async instruction moves whole rows (16 lanes x 16 bytes per
+    // row at d = 128), so one instruction touches 2 rows instead of 32.
+    constexpr int CPR = D / 8;       // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;    // rows per warp instruction
+    const int wr0 = (warp - 8) * 32;
     const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
     const size_t head_row0 = static_cast<size_t>(bh) * N;
+    const int my_chunk = lane % CPR, my_sub = lane / CPR;
+    const int hf = my_chunk >> 3, cc = my_chunk & 7;
     for (int j = 0; j < nt; ++j) {
       const int stage = j & 1;
       if (j >= 2) {
         if (!mbar_wait(smem_u32(&bars->kv_empty[stage]), ((j >> 1) - 1) & 1, st, kWhereAttnProducer)) break;
       }
-      int p = j * 128 + r;
+      int p = j * 128 + wr0 + lane;
       if (p >= L) p = L - 1;
       // largest e with r_cum[e] <= p
       int lo = 0, hi = nranges - 1;
@@ -295,18 +310,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       int krow = r_start[lo] + (p - r_cum[lo]);
       krow = krow < 0 ? 0 : (krow >= N ? N - 1 : krow);
-      const __nv_bfloat16* ksrc = Kp + (head_row0 + krow) * D;
-      const __nv_bfloat16* vsrc = Vp + (head_row0 + krow) * D;
       const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cp_async16(kdst + h * 16384 + sw128_offset(r, c), ksrc + h * 64 + c * 8);
+      for (int it = 0; it < 32 / RPI; ++it) {
+        const int rr = it * RPI + my_sub;  // row within the warp's 32
+        const int src = __shfl_sync(0xffffffffu, krow, rr);
+        cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * D + my_chunk * 8);
+      }
       cp_async_commit();
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cp_async16(vdst + h * 16384 + sw128_offset(r, c), vsrc + h * 64 + c * 8);
+      for (int it = 0; it < 32 / RPI; ++it) {
+        const int rr = it * RPI + my_sub;
+        const int src = __shfl_sync(0xffffffffu, krow, rr);
+        cp_async16(vdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Vp + (head_row0 + src) * D + my_chunk * 8);
+      }
       cp_async_commit();
       cp_async_wait<1>();
       fence_proxy_async_smem();
@@ -316,7 +333,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(smem_u32(&bars->v_full[stage]));
     }
     cp_async_wait<0>();
-  } else if (warp < 8) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
     // ---------------- softmax / correction / epilogue for tile X ----------------
     const int x = warp >> 2;
     const int q = warp & 3;
@@ -338,15 +356,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int valid = min(128, L - j * 128);
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_s + c * 32, v);
-          tmem_wait_ld();
+        uint32_t sv[128];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+        for (int c = 0; c < 4; ++c) tmem_ld32p(t_s + c * 32, sv + c * 32);
+        tmem_wait_ld();
+        float mx = -INFINITY;
+        if (valid == 128) {
+#pragma unroll
+          for (int e = 0; e < 128; e += 2) mx = fmaxf(mx, fmaxf(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e < valid) mx = fmaxf(mx, __uint_as_float(sv[e]));
         }
         const float m_new = fmaxf(m_used, mx * sl2);
         const bool grow = m_new > m_used + kRescaleThreshold;
@@ -369,22 +390,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(t_o + c * 32, v);
           }
         }
-#pragma unroll 1
+        // p = 2^(s * scale * log2(e) - m): the argument for two keys at once, the exponentials on
+        // the MUFU, the row sum over float32 p (pairs), bf16 pairs written over S as the P operand
+        const float2 scl = make_float2(sl2, sl2), negm = make_float2(-m_used, -m_used);
+        float2 lsum = make_float2(0.f, 0.f);
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_s + c * 32, v);
-          tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int col = c * 32 + 2 * e;
-            const float p0 = col < valid ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), sl2, -m_used)) : 0.f;
-            const float p1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), sl2, -m_used)) : 0.f;
-            pk[e] = pack_bf16x2(p0, p1);
-            l += bf16lo_to_f32(pk[e]) + bf16hi_to_f32(pk[e]);
+            const float2 t = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), scl, negm);
+            float2 pe;
+            if (2 * e >= 32 - kEmuPerChunk) pe = exp2_poly2(t);
+            else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            if (valid < 128) {
+              if (col >= valid) pe.x = 0.f;
+              if (col + 1 >= valid) pe.y = 0.f;
+            }
+            pk[e] = pack_bf16x2(pe.x, pe.y);
+            lsum = add2(lsum, pe);
           }
           tmem_st16(t_s + c * 16, pk);
         }
+        l += lsum.x + lsum.y;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
