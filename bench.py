@@ -44,6 +44,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="run only this many heads of the layer (profiling cases)")
+    ap.add_argument("--no-warm", action="store_true", help="skip the warm-start denoising-sequence measurement")
+    ap.add_argument("--warm-steps", type=int, default=10)
+    ap.add_argument("--seed-tokens", type=int, default=16384,
+                    help="k-means++ candidates per (b,h): every ceil(N/seed_tokens)-th token (0 = all tokens)")
     return ap.parse_args()
 
 
@@ -68,16 +72,16 @@ def gen_inputs(cfg, step=0):
 
 
 # ------------------------------------------------------------------------------------------ oracle
-def oracle_sample(cfg, top_p, rows=96, head=0):
+def oracle_sample(cfg, top_p, rows=96, head=0, seed_tokens=0):
     """The CPU oracle on a bounded sample of the layer: one head's k-means (Q and K), selection and
     permutation in full, and attention for `rows` query rows; extrapolated to the whole layer."""
     from oracle import oracle as O
     hi = I.head_inputs(cfg, 0, head)
     scale = float(np.float32(cfg.scale))
     t0 = time.perf_counter()
-    cq, lq, count_q = O.kmeans(hi["q"], cfg.nQ, cfg.iters, hi["uq"])
+    cq, lq, count_q = O.kmeans(hi["q"], cfg.nQ, cfg.iters, hi["uq"], seed_tokens=seed_tokens)
     t1 = time.perf_counter()
-    ck, lk, count_k = O.kmeans(hi["k"], cfg.nK, cfg.iters, hi["uk"])
+    ck, lk, count_k = O.kmeans(hi["k"], cfg.nK, cfg.iters, hi["uk"], seed_tokens=seed_tokens)
     t2 = time.perf_counter()
     w = O.select_weights(cq.astype(np.float32), ck.astype(np.float32), count_k, scale)
     mask = O.topp(w, count_k, top_p)
@@ -96,10 +100,10 @@ def oracle_sample(cfg, top_p, rows=96, head=0):
 def run_reference(args, cfg):
     cores = len(os.sched_getaffinity(0))
     for _ in range(args.warmup):
-        oracle_sample(cfg, args.top_p, rows=16)
+        oracle_sample(cfg, args.top_p, rows=16, seed_tokens=args.seed_tokens)
     vals = []
     for _ in range(args.steps):
-        v, _ = oracle_sample(cfg, args.top_p)
+        v, _ = oracle_sample(cfg, args.top_p, seed_tokens=args.seed_tokens)
         vals.append(v)
     value = statistics.median(vals)
     sample = (f"one head of {cfg.H}: full k-means++ + {cfg.iters} Lloyd iterations on Q and K, selection, "
@@ -107,15 +111,16 @@ def run_reference(args, cfg):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "ms", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_dict(cfg, args.top_p),
+            "config": config_dict(cfg, args.top_p, args.seed_tokens),
             "cpu_baseline": {"value": value, "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_dict(cfg, top_p):
+def config_dict(cfg, top_p, seed_tokens):
     return {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "grid": list(cfg.grid), "d": cfg.d,
             "nQ": cfg.nQ, "nK": cfg.nK, "iters": cfg.iters, "init": "kmeans++", "top_p": top_p,
+            "kmeanspp_seed_tokens": seed_tokens,
             "components": cfg.components, "sigma": cfg.sigma,
             "l2": "inputs larger than L2 (each of Q, K, V is %.0f MB)" % (cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6),
             "parallelism": "replicas"}
@@ -241,9 +246,11 @@ def main():
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        svg2.svg2_kmeans(Q, cfg.nQ, cfg.iters, KPP, cq, lab_q, cnt_q, ws, u=uq, perm=perm_q, offsets=q_off)
+        svg2.svg2_kmeans(Q, cfg.nQ, cfg.iters, KPP, cq, lab_q, cnt_q, ws, u=uq, perm=perm_q, offsets=q_off,
+                         seed_tokens=args.seed_tokens)
         mark(1)
-        svg2.svg2_kmeans(K, cfg.nK, cfg.iters, KPP, ck, lab_k, cnt_k, ws, u=uk, perm=perm_k, offsets=k_off)
+        svg2.svg2_kmeans(K, cfg.nK, cfg.iters, KPP, ck, lab_k, cnt_k, ws, u=uk, perm=perm_k, offsets=k_off,
+                         seed_tokens=args.seed_tokens)
         mark(2)
         svg2.svg2_select(cq, ck, cnt_k, args.top_p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
         mark(3)
@@ -290,6 +297,18 @@ def main():
     attn_ms = stage_ms["sparse_attn"]
     achieved_tflops = actual_flops / (attn_ms * 1e-3) / 1e12
 
+    # k-means with k-means++ over all tokens (seed_tokens = 0), for comparison with the sampled seeding
+    full_seed = None
+    if args.seed_tokens != 0:
+        ea = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ea[0].record(stream)
+        svg2.svg2_kmeans(Q, cfg.nQ, cfg.iters, KPP, cq, lab_q, cnt_q, ws, u=uq, perm=perm_q, offsets=q_off, seed_tokens=0)
+        ea[1].record(stream)
+        svg2.svg2_kmeans(K, cfg.nK, cfg.iters, KPP, ck, lab_k, cnt_k, ws, u=uk, perm=perm_k, offsets=k_off, seed_tokens=0)
+        ea[2].record(stream)
+        torch.cuda.synchronize(dev)
+        full_seed = {"kmeans_q_ms": ea[0].elapsed_time(ea[1]), "kmeans_k_ms": ea[1].elapsed_time(ea[2])}
+
     # the same layer through the single public call with host buffers (copies inside the timed region)
     e2e = None
     if not args.no_e2e:
@@ -299,13 +318,17 @@ def main():
     if not args.no_dense and rank == 0:
         dense_ms = time_dense(torch, Q, K, V, scale)
 
+    warm = None
+    if not args.no_warm:
+        warm = measure_warm(svg2, torch, cfg, args, dev, Q, K, V, ws, scale)
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        v, parts = oracle_sample(cfg, args.top_p)
+        v, parts = oracle_sample(cfg, args.top_p, seed_tokens=args.seed_tokens)
         cpu = {"value": v, "unit": "ms", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
                "sample": (f"one head of {cfg.H}: full k-means (Q and K), selection, permutation, attention for 96 "
                           f"of {cfg.N} rows; extrapolated to the layer"), "parts_s": parts}
@@ -313,7 +336,7 @@ def main():
     line = {
         "metric": METRIC, "value": whole_job_ms_per_layer(ms_per_step, world), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.top_p),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.top_p, args.seed_tokens),
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel", "achieved": achieved_tflops,
                      "peak": P["bf16_sustained"], "unit": "TFLOP/s",
                      "frac": achieved_tflops / P["bf16_sustained"],
@@ -325,7 +348,7 @@ def main():
         "attn_tflops_effective": dense_flops / (attn_ms * 1e-3) / 1e12,
         "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
         "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
-        "dense_sdpa_ms": dense_ms,
+        "dense_sdpa_ms": dense_ms, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -346,7 +369,8 @@ def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
     uk = torch.empty(huk.shape, dtype=torch.float64, device=dev)
     cq = torch.zeros(B, H, cfg.nQ, d, device=dev)
     ck = torch.zeros(B, H, cfg.nK, d, device=dev)
-    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, args.top_p, float(np.float32(cfg.scale)), 1)
+    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, args.top_p, float(np.float32(cfg.scale)), 1,
+                           args.seed_tokens)
 
     def one():
         Q.copy_(hq, non_blocking=True)
@@ -374,6 +398,84 @@ def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
     h2d = 3 * hq.numel() * 2 + (huq.numel() + huk.numel()) * 8
     return {"value": whole_job_ms_per_layer(ms, world), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
             "steps": steps, "api": "svg2_layer"}
+
+
+def measure_warm(svg2, torch, cfg, args, dev, Q0, K0, V0, ws, scale):
+    """Denoising-step sequence on the same shapes (the pages' centroid cache, section 4.3 Fig. 7(a)):
+    step s uses Q_s = Q_0 + 0.05 s eps_s, K_s likewise, a fresh V_s; k-means starts from step s-1's
+    centroids and runs 2 iterations (warm), and is also run cold (k-means++ + cfg.iters) on the same
+    inputs.  Reports per-step warm layer ms, warm vs cold k-means ms, centroid drift, and the
+    relative L2 error of both outputs against dense attention (torch SDPA) of step s."""
+    B, H, N, d = Q0.shape
+    i32 = dict(dtype=torch.int32, device=dev)
+    bufs = {}
+
+    def kbufs(tag, k):
+        if tag not in bufs:
+            bufs[tag] = (torch.empty(B, H, N, **i32), torch.empty(B, H, k, **i32), torch.empty(B, H, N, **i32),
+                         torch.empty(B, H, k + 1, **i32))
+        return bufs[tag]
+
+    lab_q, cnt_q, perm_q, q_off = kbufs("q", cfg.nQ)
+    lab_k, cnt_k, perm_k, k_off = kbufs("k", cfg.nK)
+    mask = torch.empty(B, H, cfg.nQ, cfg.nK, dtype=torch.uint8, device=dev)
+    sel_count, sel_idx = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nQ, cfg.nK, **i32)
+    Qp, Kp, Vp = torch.empty_like(Q0), torch.empty_like(Q0), torch.empty_like(Q0)
+    O_w, O_c = torch.empty_like(Q0), torch.empty_like(Q0)
+    g = torch.Generator(device=dev)
+    gen_u = np.random.default_rng(12345)
+    uq = torch.from_numpy(gen_u.random((B, H, cfg.nQ))).to(dev)
+    uk = torch.from_numpy(gen_u.random((B, H, cfg.nK))).to(dev)
+    cq = torch.zeros(B, H, cfg.nQ, d, device=dev)
+    ck = torch.zeros(B, H, cfg.nK, d, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def layer(Q, K, V, cqx, ckx, init, iters, O):
+        e = [ev() for _ in range(4)]
+        e[0].record()
+        svg2.svg2_kmeans(Q, cfg.nQ, iters, init, cqx, lab_q, cnt_q, ws, u=uq, perm=perm_q, offsets=q_off,
+                         seed_tokens=args.seed_tokens)
+        svg2.svg2_kmeans(K, cfg.nK, iters, init, ckx, lab_k, cnt_k, ws, u=uk, perm=perm_k, offsets=k_off,
+                         seed_tokens=args.seed_tokens)
+        e[1].record()
+        svg2.svg2_select(cqx, ckx, cnt_k, args.top_p, scale, mask, sel_count, sel_idx, ws)
+        svg2.svg2_gather(Q, perm_q, Qp)
+        svg2.svg2_gather(K, perm_k, Kp)
+        svg2.svg2_gather(V, perm_k, Vp)
+        svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
+        e[2].record()
+        return e
+
+    # step 0: cold start, fills the cache
+    layer(Q0, K0, V0, cq, ck, svg2.SVG2_INIT_KMEANSPP, cfg.iters, O_c)
+    out = {"steps": args.warm_steps, "warm_iters": 2, "cold": "k-means++ + %d iterations" % cfg.iters,
+           "layer_ms_warm": [], "kmeans_ms_warm": [], "kmeans_ms_cold": [], "drift_q": [], "drift_k": [],
+           "rel_l2_vs_dense_warm": [], "rel_l2_vs_dense_cold": []}
+    for step in range(1, args.warm_steps + 1):
+        g.manual_seed(1000 + step)
+        Q = (Q0.float() + 0.05 * step * torch.randn(Q0.shape, device=dev, generator=g)).to(torch.bfloat16)
+        K = (K0.float() + 0.05 * step * torch.randn(K0.shape, device=dev, generator=g)).to(torch.bfloat16)
+        V = torch.randn(V0.shape, device=dev, generator=g).to(torch.bfloat16)
+        cq_prev, ck_prev = cq.clone(), ck.clone()
+        ew = layer(Q, K, V, cq, ck, svg2.SVG2_INIT_GIVEN, 2, O_w)
+        cq_c, ck_c = torch.zeros_like(cq), torch.zeros_like(ck)
+        ec = layer(Q, K, V, cq_c, ck_c, svg2.SVG2_INIT_KMEANSPP, cfg.iters, O_c)
+        dense = torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=scale).float()
+        torch.cuda.synchronize(dev)
+        dn = dense.norm()
+        out["layer_ms_warm"].append(ew[0].elapsed_time(ew[2]))
+        out["kmeans_ms_warm"].append(ew[0].elapsed_time(ew[1]))
+        out["kmeans_ms_cold"].append(ec[0].elapsed_time(ec[1]))
+        out["drift_q"].append(float((cq - cq_prev).norm() / cq_prev.norm()))
+        out["drift_k"].append(float((ck - ck_prev).norm() / ck_prev.norm()))
+        out["rel_l2_vs_dense_warm"].append(float((O_w.float() - dense).norm() / dn))
+        out["rel_l2_vs_dense_cold"].append(float((O_c.float() - dense).norm() / dn))
+    svg2.raise_on_device_error(ws)
+    med = lambda v: float(statistics.median(v))
+    out["summary"] = {"layer_ms_warm": med(out["layer_ms_warm"]), "kmeans_ms_warm": med(out["kmeans_ms_warm"]),
+                      "kmeans_ms_cold": med(out["kmeans_ms_cold"]),
+                      "kmeans_speedup": med(out["kmeans_ms_cold"]) / med(out["kmeans_ms_warm"])}
+    return out
 
 
 def time_dense(torch, Q, K, V, scale, reps=3):

@@ -57,6 +57,11 @@ typedef enum { SVG2_BF16 = 0, SVG2_F32 = 1 } svg2_dtype;
  * previous denoising step's centroids.  KMEANSPP: k-means++ seeding from the data (Method (1)). */
 typedef enum { SVG2_INIT_GIVEN = 0, SVG2_INIT_KMEANSPP = 1 } svg2_init;
 
+/* k-means++ seeding looks at every stride-th token, stride = ceil(N / seed_tokens), so that at most
+ * seed_tokens tokens are candidates (0 = all tokens).  The Lloyd iterations always use all tokens.
+ * This default keeps the seeding cheap on video-length layers. */
+#define SVG2_DEFAULT_SEED_TOKENS 16384
+
 /* Largest supported sizes of this build. */
 #define SVG2_MAX_CLUSTERS 1024
 #define SVG2_MAX_TOKENS (1 << 24)
@@ -82,6 +87,8 @@ SVG2_API int svg2_check_status(void* ws, void* stream, int* device_status, uint3
  *   init       SVG2_INIT_GIVEN (centroids holds the start, e.g. the previous step's cache) or
  *              SVG2_INIT_KMEANSPP (seeding from the data; `u` must then hold B*H*k uniforms in
  *              [0,1), float64, one per seed, and seeds are chosen by fixed-point D^2 sampling).
+ *   seed_tokens  k-means++ candidates: every ceil(N / seed_tokens)-th token (0 = all tokens; see
+ *              SVG2_DEFAULT_SEED_TOKENS); the candidate count must be >= k.
  *   centroids  float32 [B, H, k, d], in (GIVEN) and out (final centroids).
  *   labels     int32 [B, H, N], out: labels of the last assignment (the ones the final centroids
  *              were computed from).
@@ -91,7 +98,7 @@ SVG2_API int svg2_check_status(void* ws, void* stream, int* device_status, uint3
  *   offsets    int32 [B, H, k+1], out (optional): exclusive scan of counts.
  * 1 <= k <= min(N, SVG2_MAX_CLUSTERS). */
 SVG2_API int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int iters, int init,
-                const double* u, float* centroids, int32_t* labels, int32_t* counts, int32_t* perm,
+                const double* u, int seed_tokens, float* centroids, int32_t* labels, int32_t* counts, int32_t* perm,
                 int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
 /*
@@ -159,6 +166,7 @@ typedef struct {
   int init;            /* svg2_init: GIVEN = warm start from cq/ck, KMEANSPP = cold start */
   float top_p;         /* (0, 1]; >= 1 keeps every pair */
   float scale;         /* softmax scale, usually 1/sqrt(d) */
+  int seed_tokens;     /* k-means++ candidates, as in svg2_kmeans (0 = all tokens) */
   int fuse_unpermute;  /* 1: write O in token order from the attention epilogue (default path);
                           0: write permuted rows, then run svg2_unpermute */
 } svg2_params;

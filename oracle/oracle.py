@@ -171,22 +171,30 @@ def dense_attention_rows(Q, K, V, scale, rows=None):
     return out
 
 
+def seed_stride(N: int, seed_tokens: int) -> int:
+    """k-means++ candidates are every stride-th token so that at most seed_tokens are used (0 = all)."""
+    if seed_tokens <= 0 or seed_tokens >= N:
+        return 1
+    return -(-N // seed_tokens)
+
+
 def kmeans(X: np.ndarray, k: int, iters: int, u: Optional[np.ndarray] = None,
-           C0: Optional[np.ndarray] = None):
-    """k-means++ seeding (or the given C0), then `iters` Lloyd iterations."""
+           C0: Optional[np.ndarray] = None, seed_tokens: int = 0):
+    """k-means++ seeding on the candidate tokens X[::stride] (or the given C0), then `iters` Lloyd
+    iterations over all tokens."""
     if C0 is None:
-        _, C0 = kmeanspp(X, k, u)
+        _, C0 = kmeanspp(np.ascontiguousarray(X[::seed_stride(X.shape[0], seed_tokens)]), k, u)
     return lloyd(X, C0, iters)
 
 
 def layer_head(q, k, v, nQ, nK, iters, top_p, scale, uq=None, uk=None, cq0=None, ck0=None,
-               rows=None) -> Dict[str, np.ndarray]:
+               rows=None, seed_tokens: int = 0) -> Dict[str, np.ndarray]:
     """The whole layer for one (batch, head), as the Method section orders it.
 
     `rows` (original token indices) restricts the attention to those output rows.
     """
-    cq, lq, count_q = kmeans(q, nQ, iters, uq, cq0)
-    ck, lk, count_k = kmeans(k, nK, iters, uk, ck0)
+    cq, lq, count_q = kmeans(q, nQ, iters, uq, cq0, seed_tokens)
+    ck, lk, count_k = kmeans(k, nK, iters, uk, ck0, seed_tokens)
     w = select_weights(cq.astype(np.float32), ck.astype(np.float32), count_k, scale)
     mask = topp(w, count_k, top_p)
     perm_q, q_off = permute(lq, nQ)

@@ -96,10 +96,11 @@ void carve_layer(Carve& c, int BH, int N, int d, int nQ, int nK, const svg2_laye
 }
 
 cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int iters, int init, const double* u,
-                       float* C, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets,
+                       int seed_tokens, float* C, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets,
                        const KmeansScratch& s, DeviceStatus* st, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
-  if (init == SVG2_INIT_KMEANSPP) e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, stream);
+  if (init == SVG2_INIT_KMEANSPP)
+    e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, seed_tokens, stream);
   if (e == cudaSuccess) e = launch_centroid_prep(C, BH, k, d, s.c_hi, s.c_lo, s.c_norm, stream);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
     e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, st, stream);
@@ -176,7 +177,7 @@ int svg2_check_status(void* ws, void* stream, int* device_status, uint32_t* wher
 }
 
 int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int iters, int init, const double* u,
-                float* centroids, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets, void* ws,
+                int seed_tokens, float* centroids, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets, void* ws,
                 size_t ws_bytes, void* stream) {
   try {
     int r = check_sizes(B, H, N, d);
@@ -196,7 +197,10 @@ int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int
     if (r != SVG2_OK) return r;
     if (perm == nullptr) perm = s.perm;
     if (offsets == nullptr) offsets = s.offsets;
-    return to_status(run_kmeans(X, dtype == SVG2_F32, BH, N, d, k, iters, init, u, centroids, labels, counts, perm,
+    if (seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
+    if (init == SVG2_INIT_KMEANSPP && (N + kmeanspp_stride(N, seed_tokens) - 1) / kmeanspp_stride(N, seed_tokens) < k)
+      return SVG2_ERR_INVALID_ARG;  // fewer candidates than seeds
+    return to_status(run_kmeans(X, dtype == SVG2_F32, BH, N, d, k, iters, init, u, seed_tokens, centroids, labels, counts, perm,
                                 offsets, s, st, static_cast<cudaStream_t>(stream)));
   } catch (...) {
     return SVG2_ERR_CUDA;
@@ -336,6 +340,11 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
     if (r != SVG2_OK) return r;
     if (!valid_dtype(dtype) || p->iters < 1 || (p->init != SVG2_INIT_GIVEN && p->init != SVG2_INIT_KMEANSPP))
       return SVG2_ERR_INVALID_ARG;
+    if (p->seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
+    if (p->init == SVG2_INIT_KMEANSPP) {
+      const int stride = kmeanspp_stride(N, p->seed_tokens);
+      if ((N + stride - 1) / stride < (p->nQ > p->nK ? p->nQ : p->nK)) return SVG2_ERR_INVALID_ARG;
+    }
     if (!(p->top_p > 0.f) || p->scale != p->scale) return SVG2_ERR_INVALID_ARG;
     if (Q == nullptr || K == nullptr || V == nullptr || cq == nullptr || ck == nullptr || O == nullptr)
       return SVG2_ERR_INVALID_ARG;
@@ -351,10 +360,10 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
     if (r != SVG2_OK) return r;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f32 = dtype == SVG2_F32;
-    cudaError_t e = run_kmeans(Q, f32, BH, N, d, p->nQ, p->iters, p->init, uq, cq, L.labels_q, L.count_q, L.perm_q,
+    cudaError_t e = run_kmeans(Q, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q, L.perm_q,
                                L.q_off, L.kq, L.st, s);
     if (e == cudaSuccess)
-      e = run_kmeans(K, f32, BH, N, d, p->nK, p->iters, p->init, uk, ck, L.labels_k, L.count_k, L.perm_k, L.k_off,
+      e = run_kmeans(K, f32, BH, N, d, p->nK, p->iters, p->init, uk, p->seed_tokens, ck, L.labels_k, L.count_k, L.perm_k, L.k_off,
                      L.kk, L.st, s);
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, L.weights, L.mask,

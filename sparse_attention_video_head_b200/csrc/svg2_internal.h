@@ -112,7 +112,9 @@ cudaError_t launch_unpermute(const void* Op, const int32_t* perm, int BH, int N,
                              cudaStream_t s);
 
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
-                            float* centroids, double* dist, int32_t* near, cudaStream_t s);
+                            float* centroids, double* dist, int32_t* near, int seed_tokens, cudaStream_t s);
+// Spacing of the k-means++ candidates: every stride-th token, so that at most seed_tokens are used.
+int kmeanspp_stride(int N, int seed_tokens);
 cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, uint16_t* c_hi, uint16_t* c_lo,
                                  float* c_norm, cudaStream_t s);
 cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,

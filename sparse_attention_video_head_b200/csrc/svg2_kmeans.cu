@@ -83,20 +83,23 @@ __device__ unsigned long long block_exscan_u64(unsigned long long v, unsigned lo
   return warp_buf[32];
 }
 
-__global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restrict__ X, bool f32, int N, int d,
-                                                            int k, const double* __restrict__ u,
+// Fallback for candidate sets too large for shared memory: one CTA per (b,h), state in global memory.
+__global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restrict__ X, bool f32, int Ntok, int stride,
+                                                            int d, int k, const double* __restrict__ u,
                                                             float* __restrict__ C, double* __restrict__ Dg,
                                                             int32_t* __restrict__ Ag) {
+  const int N = (Ntok + stride - 1) / stride;  // candidates: every stride-th token
   __shared__ float cs[128];
   __shared__ float ss[1024];
   __shared__ unsigned long long warp_buf[33];
   __shared__ double red[32];
   __shared__ int pick_sh;
   const int bh = blockIdx.x, tid = threadIdx.x;
-  const size_t xbase = static_cast<size_t>(bh) * N * d;
+  const size_t xbase = static_cast<size_t>(bh) * Ntok * d;
+  const size_t rstride = static_cast<size_t>(stride) * d;  // elements between candidate rows
   float* Ch = C + static_cast<size_t>(bh) * k * d;
-  double* D = Dg + static_cast<size_t>(bh) * N;
-  int32_t* A = Ag + static_cast<size_t>(bh) * N;
+  double* D = Dg + static_cast<size_t>(bh) * Ntok;
+  int32_t* A = Ag + static_cast<size_t>(bh) * Ntok;
   const double* uh = u + static_cast<size_t>(bh) * k;
   const int per = (N + blockDim.x - 1) / blockDim.x;
   const int t0 = min(N, tid * per), t1 = min(N, t0 + per);
@@ -105,14 +108,14 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
   if (pick >= N) pick = N - 1;
   if (pick < 0) pick = 0;
   for (int i = tid; i < d; i += blockDim.x) {
-    const float v = ld_elem(X, xbase + static_cast<size_t>(pick) * d + i, f32);
+    const float v = ld_elem(X, xbase + static_cast<size_t>(pick) * rstride + i, f32);
     cs[i] = v;
     Ch[i] = v;
   }
   __syncthreads();
   double lmax = 0.0;
   for (int t = t0; t < t1; ++t) {
-    const double v = sqdist_exact(X, xbase + static_cast<size_t>(t) * d, f32, cs, d);
+    const double v = sqdist_exact(X, xbase + static_cast<size_t>(t) * rstride, f32, cs, d);
     D[t] = v;
     A[t] = 0;
     lmax = fmax(lmax, v);
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
     __syncthreads();
     const int p = pick_sh < 0 ? N - 1 : pick_sh;
     for (int i = tid; i < d; i += blockDim.x) {
-      const float v = ld_elem(X, xbase + static_cast<size_t>(p) * d + i, f32);
+      const float v = ld_elem(X, xbase + static_cast<size_t>(p) * rstride + i, f32);
       cs[i] = v;
       Ch[static_cast<size_t>(s) * d + i] = v;
     }
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
     for (int t = t0; t < t1; ++t) {
       const double Dt = D[t];
       if (static_cast<double>(ss[A[t]]) >= 4.0001 * Dt) continue;  // new seed provably farther
-      const size_t ro = xbase + static_cast<size_t>(t) * d;
+      const size_t ro = xbase + static_cast<size_t>(t) * rstride;
       const float f = sqdist_f32(X, ro, f32, cs, d);
       if (static_cast<double>(f) > Dt * (1.0 + 1e-3)) continue;
       const double nd = sqdist_exact(X, ro, f32, cs, d);
@@ -187,19 +190,12 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
 }
 
 // ------------------------------------------------------------------------------------------------
-// k-means++ on a cluster of kPpCtas CTAs per (b,h): each CTA keeps D^2 (float64) and the nearest
-// seed (uint16) of its token range in shared memory; warps read token rows cooperatively (each lane
-// d/32 consecutive values, so one warp load covers a row); per seed, the CTAs exchange their
-// fixed-point weight totals through distributed shared memory and the CTA holding the sampling
-// target finds the token.  The float64 D^2 of a token is summed per lane over its values and then
-// across lanes in a fixed butterfly order; it can differ from a sequential sum in the last bit,
-// which moves the fixed-point weight floor(D^2 / M0 * 2^32) only when D^2 / M0 * 2^32 lies within
-// ~1e-6 of an integer, and changes a pick only if the sampling target sits exactly on that step.
+// k-means++ seeding kernels with shared-memory state (see kmeanspp_kernel2 below)
 // ------------------------------------------------------------------------------------------------
-constexpr int kPpCtas = 8;
-constexpr int kPpThreads = 1024;
+constexpr int kPpThreads = 512;
 constexpr int kPpWarps = kPpThreads / 32;
-constexpr int kPpMaxTokensPerCta = 15360;   // 10 bytes of state per token: 150 KB of shared memory
+constexpr int kPpMaxPerCta = 15360;   // 10 bytes of state per candidate: 150 KB of shared memory
+constexpr int kPpClusterCtas = 8;
 
 __host__ __device__ constexpr size_t pp_smem_bytes(int per_cta) {
   return static_cast<size_t>(per_cta) * 10 + 16;
@@ -228,6 +224,78 @@ __device__ __forceinline__ void pp_load_row(const void* X, size_t row_elem, int 
   }
 }
 
+// Raw row values of lane `lane` (E per lane) as 32-bit words: bf16 pairs, or float32 values.
+template <int E, bool F32>
+constexpr int pp_words() { return F32 ? E : E / 2; }
+
+template <int E, bool F32>
+__device__ __forceinline__ void pp_load_raw(const void* X, size_t row_elem, int lane,
+                                            uint32_t (&w)[pp_words<E, F32>()]) {
+  if constexpr (F32) {
+    static_assert(E == 2, "float32 rows use d = 64 on this path");
+    const float2 a = __ldg(reinterpret_cast<const float2*>(static_cast<const float*>(X) + row_elem + lane * E));
+    w[0] = __float_as_uint(a.x);
+    w[1] = __float_as_uint(a.y);
+  } else {
+    const unsigned short* p = static_cast<const unsigned short*>(X) + row_elem + lane * E;
+    if constexpr (E == 4) {
+      const uint2 a = __ldg(reinterpret_cast<const uint2*>(p));
+      w[0] = a.x;
+      w[1] = a.y;
+    } else {
+      w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+    }
+  }
+}
+
+template <int E, bool F32>
+__device__ __forceinline__ void pp_unpack(const uint32_t (&w)[pp_words<E, F32>()], float (&v)[E]) {
+  if constexpr (F32) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) v[i] = __uint_as_float(w[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      v[2 * i] = bf16lo_to_f32(w[i]);
+      v[2 * i + 1] = bf16hi_to_f32(w[i]);
+    }
+  }
+}
+
+// Exact float64 D^2 of one token row against cs, sequential over i (the oracle's order, no FMA).
+template <int D, bool F32>
+__device__ __forceinline__ double pp_exact_seq(const void* X, size_t row_elem, const float* cs) {
+  double acc = 0.0;
+  if constexpr (F32) {
+    const float4* r = reinterpret_cast<const float4*>(static_cast<const float*>(X) + row_elem);
+#pragma unroll 4
+    for (int q = 0; q < D / 4; ++q) {
+      const float4 a = __ldg(r + q);
+      const float x[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const double df = __dsub_rn(static_cast<double>(x[e]), static_cast<double>(cs[4 * q + e]));
+        acc = __dadd_rn(acc, __dmul_rn(df, df));
+      }
+    }
+  } else {
+    const uint4* r = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(X) + row_elem);
+#pragma unroll 4
+    for (int q = 0; q < D / 8; ++q) {
+      const uint4 a = __ldg(r + q);
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const double d0 = __dsub_rn(static_cast<double>(bf16lo_to_f32(w[e])), static_cast<double>(cs[8 * q + 2 * e]));
+        acc = __dadd_rn(acc, __dmul_rn(d0, d0));
+        const double d1 = __dsub_rn(static_cast<double>(bf16hi_to_f32(w[e])), static_cast<double>(cs[8 * q + 2 * e + 1]));
+        acc = __dadd_rn(acc, __dmul_rn(d1, d1));
+      }
+    }
+  }
+  return acc;
+}
+
 template <int E>
 __device__ __forceinline__ double pp_exact(const float (&v)[E], const float* cs, int lane) {
   double acc = 0.0;
@@ -241,119 +309,226 @@ __device__ __forceinline__ double pp_exact(const float (&v)[E], const float* cs,
   return __shfl_sync(0xffffffffu, acc, 0);  // lane 0's summation order decides
 }
 
-template <int E, bool F32>
-__global__ void __cluster_dims__(kPpCtas, 1, 1) __launch_bounds__(kPpThreads, 1)
-    kmeanspp_cluster_kernel(const void* __restrict__ X, int N, int k, const double* __restrict__ u,
-                            float* __restrict__ C) {
+template <int CL>
+__device__ __forceinline__ void pp_sync() {
+  if constexpr (CL > 1) cluster_sync();
+  else __syncthreads();
+}
+
+template <int CL>
+__device__ __forceinline__ void pp_bcast_u64(unsigned long long* var, unsigned long long v) {
+  if constexpr (CL > 1) {
+    for (uint32_t r = 0; r < CL; ++r) st_cluster_u64(var, r, v);
+  } else {
+    *var = v;
+  }
+}
+
+// k-means++ seeding over a candidate set: every `stride`-th token (stride 1 = all tokens), S in all.
+// One (b,h) runs on CL CTAs: CL = 1 keeps the whole candidate set's state (D^2 in float64 and the
+// nearest seed) in one CTA's shared memory; CL = kPpClusterCtas spreads it over a thread-block
+// cluster and exchanges the per-seed totals through distributed shared memory.  Lane l of warp w
+// owns a contiguous piece of the warp's candidates, so a lane's running fixed-point weight total is
+// its piece's total and the sampling search needs no division until the final piece scan.
+// Per seed: ||c_new - c_near||^2 >= 4.0001 D^2 proves a candidate cannot get closer; the rest get
+// a float32 distance (warp-cooperative, or a transpose-reduce over 32 candidates when many are
+// left); those within 1e-3 of their D^2 get the float64 D^2 (per-lane sums over d/32 values, then a
+// fixed butterfly across lanes, lane 0's order).  That can differ from a sequential sum in the last
+// bit, which moves the fixed-point weight floor(D^2 / M0 * 2^32) only when D^2 / M0 * 2^32 lies
+// within ~1e-6 of an integer, and changes a seed only if the sampling target sits exactly on it.
+template <int E, bool F32, int CL>
+__global__ void __launch_bounds__(kPpThreads, 1)
+    kmeanspp_kernel2(const void* __restrict__ X, int N, int stride, int S, int k, const double* __restrict__ u,
+                     float* __restrict__ C) {
   constexpr int D = E * 32;
-  constexpr int kBatch = 8;  // token rows in flight per warp
   extern __shared__ uint8_t pp_smem[];
   __shared__ float cs[D];
   __shared__ float ss[1024];
   __shared__ unsigned long long wsum[kPpWarps];
-  __shared__ unsigned long long cta_tot[kPpCtas];
-  __shared__ double cta_max[kPpCtas];
+  __shared__ unsigned long long cta_tot[CL];
+  __shared__ unsigned long long cta_max[CL];
   __shared__ unsigned long long pick_bcast;
   __shared__ unsigned long long hit_base;
   __shared__ int hit_warp;
-  const uint32_t rank = cluster_rank();
-  const int bh = blockIdx.x / kPpCtas;
+  const uint32_t rank = CL > 1 ? cluster_rank() : 0u;
+  const int bh = blockIdx.x / CL;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per_cta = (N + kPpCtas - 1) / kPpCtas;
-  const int lo = min(N, static_cast<int>(rank) * per_cta), hi = min(N, lo + per_cta);
+  const int per_cta = (S + CL - 1) / CL;
+  const int lo = min(S, static_cast<int>(rank) * per_cta), hi = min(S, lo + per_cta);
   const int per_warp = (hi - lo + kPpWarps - 1) / kPpWarps;
   const int wlo = min(hi, lo + warp * per_warp), whi = min(hi, wlo + per_warp);
+  const int P = (whi - wlo + 31) / 32;  // candidates per lane piece
+  const int plo = min(whi, wlo + lane * P), phi = min(whi, plo + P);
   double* Ds = reinterpret_cast<double*>(pp_smem);
   uint16_t* As = reinterpret_cast<uint16_t*>(pp_smem + static_cast<size_t>(per_cta) * 8);
   const size_t xbase = static_cast<size_t>(bh) * N * D;
   float* Ch = C + static_cast<size_t>(bh) * k * D;
   const double* uh = u + static_cast<size_t>(bh) * k;
+  auto row_of = [&](int cand) { return xbase + static_cast<size_t>(cand) * stride * D; };
 
-  auto load_seed = [&](int p, int s) {
+  auto load_seed = [&](int cand, int s) {
     for (int i = threadIdx.x; i < D; i += blockDim.x) {
       float v;
-      if constexpr (F32) v = static_cast<const float*>(X)[xbase + static_cast<size_t>(p) * D + i];
-      else v = bf16lo_to_f32(static_cast<const unsigned short*>(X)[xbase + static_cast<size_t>(p) * D + i]);
+      if constexpr (F32) v = static_cast<const float*>(X)[row_of(cand) + i];
+      else v = bf16lo_to_f32(static_cast<const unsigned short*>(X)[row_of(cand) + i]);
       cs[i] = v;
       if (rank == 0) Ch[static_cast<size_t>(s) * D + i] = v;
     }
   };
 
-  unsigned long long qsum = 0ull;  // this warp's total fixed-point weight (held by lane 0)
+  unsigned long long qsum = 0ull;  // fixed-point weight of this lane's piece
   double M0 = 0.0;
 
-  // Lower D^2 of this warp's tokens with seed s (already in cs; ss holds seed-to-seed distances).
+  // float64 D^2 of up to 4 candidates at once (warp-cooperative; every lane gets lane 0's sums)
+  auto exact4 = [&](const int (&cb)[4], double (&nd)[4]) {
+    double acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[i] = 0.0;
+      if (cb[i] >= 0) {
+        float v[E];
+        pp_load_row<E, F32>(X, row_of(cb[i]), lane, v);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const double df = __dsub_rn(static_cast<double>(v[e]), static_cast<double>(cs[lane * E + e]));
+          acc[i] = __dadd_rn(acc[i], __dmul_rn(df, df));
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = __dadd_rn(acc[i], __shfl_xor_sync(0xffffffffu, acc[i], o));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) nd[i] = __shfl_sync(0xffffffffu, acc[i], 0);
+  };
+
   auto update_pass = [&](int s, bool first) {
-    for (int tb = wlo; tb < whi; tb += 32) {
-      const int t = tb + lane;
+    for (int i = 0; i < P; ++i) {
+      const int c = plo + i;  // this lane's candidate in slice i
       double Dt = INFINITY;
       bool cand = false;
-      if (t < whi) {
+      if (c < phi) {
         if (first) {
           cand = true;
         } else {
-          Dt = Ds[t - lo];
-          cand = static_cast<double>(ss[As[t - lo]]) < 4.0001 * Dt;  // else provably not closer
+          Dt = Ds[c - lo];
+          cand = static_cast<double>(ss[As[c - lo]]) < 4.0001 * Dt;  // else provably not closer
         }
       }
-      unsigned m = __ballot_sync(0xffffffffu, cand);
-      while (m) {
-        int tl[kBatch];
+      const unsigned m = __ballot_sync(0xffffffffu, cand);
+      if (m == 0u) continue;
+      bool need = cand;
+      if (!first) {
+        float f = 0.f;
+        if (__popc(m) <= 8) {
+          // few candidates: one warp-cooperative float32 distance each, 4 at a time
+          unsigned mm = m;
+          while (mm) {
+            int bl[4];
+            float part[4];
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          tl[i] = m ? __ffs(m) - 1 : -1;
-          if (m) m &= m - 1;
-        }
-        float part[kBatch];
+            for (int q = 0; q < 4; ++q) {
+              bl[q] = mm ? __ffs(mm) - 1 : -1;
+              if (mm) mm &= mm - 1;
+            }
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          part[i] = 0.f;
-          if (tl[i] >= 0) {
-            float v[E];
-            pp_load_row<E, F32>(X, xbase + static_cast<size_t>(tb + tl[i]) * D, lane, v);
+            for (int q = 0; q < 4; ++q) {
+              part[q] = 0.f;
+              const int cq = __shfl_sync(0xffffffffu, c, bl[q] < 0 ? 0 : bl[q]);
+              if (bl[q] >= 0) {
+                float v[E];
+                pp_load_row<E, F32>(X, row_of(cq), lane, v);
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-              const float df = v[e] - cs[lane * E + e];
-              part[i] = fmaf(df, df, part[i]);
+                for (int e = 0; e < E; ++e) {
+                  const float df = v[e] - cs[lane * E + e];
+                  part[q] = fmaf(df, df, part[q]);
+                }
+              }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) part[q] += __shfl_xor_sync(0xffffffffu, part[q], o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float fq = __shfl_sync(0xffffffffu, part[q], 0);
+              if (lane == bl[q]) f = fq;
             }
           }
-        }
+        } else {
+          // many candidates: all rows in flight, then a transpose-reduce leaves lane l its own sum
+          uint32_t raw[32][pp_words<E, F32>()];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
+          for (int r = 0; r < 32; ++r) {
+            const int cr = __shfl_sync(0xffffffffu, c, r);
+            if ((m >> r) & 1u) pp_load_raw<E, F32>(X, row_of(cr), lane, raw[r]);
+          }
+          float pr[32];
 #pragma unroll
-          for (int i = 0; i < kBatch; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+          for (int r = 0; r < 32; ++r) {
+            pr[r] = 0.f;
+            if ((m >> r) & 1u) {
+              float v[E];
+              pp_unpack<E, F32>(raw[r], v);
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          if (tl[i] < 0) continue;                                        // warp-uniform
-          const float f = __shfl_sync(0xffffffffu, part[i], 0);            // one value for the warp
-          const double Di = __shfl_sync(0xffffffffu, Dt, tl[i]);
-          if (!first && static_cast<double>(f) > Di * (1.0 + 1e-3)) continue;  // float32 error << 1e-3
-          float v[E];
-          pp_load_row<E, F32>(X, xbase + static_cast<size_t>(tb + tl[i]) * D, lane, v);
-          const double nd = pp_exact<E>(v, cs, lane);
-          if (nd < Di && lane == 0) {
-            if (!first) {
-              qsum -= fixed_weight(Di, M0);
-              qsum += fixed_weight(nd, M0);
+              for (int e = 0; e < E; ++e) {
+                const float df = v[e] - cs[lane * E + e];
+                pr[r] = fmaf(df, df, pr[r]);
+              }
             }
-            Ds[tb + tl[i] - lo] = nd;
-            As[tb + tl[i] - lo] = static_cast<uint16_t>(s);
+          }
+#pragma unroll
+          for (int o = 16, n = 16; o > 0; o >>= 1, n >>= 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int q = 0; q < n; ++q) {
+              const float keep = upper ? pr[q + n] : pr[q];
+              const float send = upper ? pr[q] : pr[q + n];
+              pr[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+          }
+          f = pr[0];
+        }
+        need = cand && static_cast<double>(f) <= Dt * (1.0 + 1e-3);  // float32 error << 1e-3
+      }
+      unsigned nm = __ballot_sync(0xffffffffu, need);
+      while (nm) {
+        int bl[4], cb[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          bl[q] = nm ? __ffs(nm) - 1 : -1;
+          if (nm) nm &= nm - 1;
+          const int cq = __shfl_sync(0xffffffffu, c, bl[q] < 0 ? 0 : bl[q]);
+          cb[q] = bl[q] >= 0 ? cq : -1;
+        }
+        double nd[4];
+        exact4(cb, nd);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (lane == bl[q] && nd[q] < Dt) {
+            if (!first) {
+              qsum -= fixed_weight(Dt, M0);
+              qsum += fixed_weight(nd[q], M0);
+            }
+            Ds[c - lo] = nd[q];
+            As[c - lo] = static_cast<uint16_t>(s);
           }
         }
       }
     }
   };
 
-  // ---- seed 0, the initial D^2 and the fixed-point scale M0 (cluster-wide maximum)
-  long long p0 = static_cast<long long>(floor(uh[0] * static_cast<double>(N)));
-  if (p0 >= N) p0 = N - 1;
+  // ---- seed 0, the initial D^2 and the fixed-point scale M0 (maximum over all candidates)
+  long long p0 = static_cast<long long>(floor(uh[0] * static_cast<double>(S)));
+  if (p0 >= S) p0 = S - 1;
   if (p0 < 0) p0 = 0;
   load_seed(static_cast<int>(p0), 0);
   __syncthreads();
   update_pass(0, true);
   __syncwarp();
   double lmax = 0.0;
-  for (int t = wlo + lane; t < whi; t += 32) lmax = fmax(lmax, Ds[t - lo]);
+  for (int c = plo; c < phi; ++c) lmax = fmax(lmax, Ds[c - lo]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
   if (lane == 0) wsum[warp] = static_cast<unsigned long long>(__double_as_longlong(lmax));
@@ -361,33 +536,34 @@ __global__ void __cluster_dims__(kPpCtas, 1, 1) __launch_bounds__(kPpThreads, 1)
   if (threadIdx.x == 0) {
     double mx = 0.0;
     for (int w = 0; w < kPpWarps; ++w) mx = fmax(mx, __longlong_as_double(static_cast<long long>(wsum[w])));
-    for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_f64(&cta_max[rank], r, mx);
+    pp_bcast_u64<CL>(&cta_max[rank], static_cast<unsigned long long>(__double_as_longlong(mx)));
   }
-  cluster_sync();
-  for (int r = 0; r < kPpCtas; ++r) M0 = fmax(M0, cta_max[r]);
-  if (lane == 0)
-    for (int t = wlo; t < whi; ++t) qsum += fixed_weight(Ds[t - lo], M0);
+  pp_sync<CL>();
+  for (int r = 0; r < CL; ++r) M0 = fmax(M0, __longlong_as_double(static_cast<long long>(cta_max[r])));
+  for (int c = plo; c < phi; ++c) qsum += fixed_weight(Ds[c - lo], M0);
 
   for (int s = 1; s < k; ++s) {
-    // ---- totals: warps -> CTA -> every CTA of the cluster
-    if (lane == 0) wsum[warp] = qsum;
+    // ---- totals: lanes -> warps -> CTA -> every CTA of the cluster
+    unsigned long long wq = qsum;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wq += __shfl_xor_sync(0xffffffffu, wq, o);
+    if (lane == 0) wsum[warp] = wq;
     __syncthreads();
     if (threadIdx.x == 0) {
       unsigned long long t = 0;
       for (int w = 0; w < kPpWarps; ++w) t += wsum[w];
-      for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_u64(&cta_tot[rank], r, t);
+      pp_bcast_u64<CL>(&cta_tot[rank], t);
     }
-    cluster_sync();
+    pp_sync<CL>();
     unsigned long long U = 0, base = 0;
-    for (int r = 0; r < kPpCtas; ++r) {
+    for (int r = 0; r < CL; ++r) {
       if (r < static_cast<int>(rank)) base += cta_tot[r];
       U += cta_tot[r];
     }
     if (U == 0ull) {
       if (threadIdx.x == 0 && rank == 0) {
-        const long long p = static_cast<long long>(floor(uh[s] * static_cast<double>(N)));
-        const unsigned long long pk = static_cast<unsigned long long>(p >= N ? N - 1 : p);
-        for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_u64(&pick_bcast, r, pk);
+        const long long p = static_cast<long long>(floor(uh[s] * static_cast<double>(S)));
+        pp_bcast_u64<CL>(&pick_bcast, static_cast<unsigned long long>(p >= S ? S - 1 : p));
       }
     } else {
       unsigned long long target = static_cast<unsigned long long>(floor(uh[s] * static_cast<double>(U)));
@@ -406,33 +582,28 @@ __global__ void __cluster_dims__(kPpCtas, 1, 1) __launch_bounds__(kPpThreads, 1)
         }
         __syncthreads();
         if (warp == hit_warp) {
-          // lanes split the warp's tokens into contiguous pieces; scan the piece sums
-          const int piece = (whi - wlo + 31) / 32;
-          const int plo = min(whi, wlo + lane * piece), phi = min(whi, plo + piece);
-          unsigned long long ps = 0;
-          for (int t = plo; t < phi; ++t) ps += fixed_weight(Ds[t - lo], M0);
-          unsigned long long incl = ps;
+          unsigned long long incl = qsum;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
           }
-          unsigned long long run = hit_base + incl - ps;
-          if (ps > 0ull && run <= target && target < run + ps) {
+          unsigned long long run = hit_base + incl - qsum;
+          if (qsum > 0ull && run <= target && target < run + qsum) {
             int pk = phi - 1;
-            for (int t = plo; t < phi; ++t) {
-              run += fixed_weight(Ds[t - lo], M0);
+            for (int c = plo; c < phi; ++c) {
+              run += fixed_weight(Ds[c - lo], M0);
               if (run > target) {
-                pk = t;
+                pk = c;
                 break;
               }
             }
-            for (uint32_t r = 0; r < kPpCtas; ++r) st_cluster_u64(&pick_bcast, r, static_cast<unsigned long long>(pk));
+            pp_bcast_u64<CL>(&pick_bcast, static_cast<unsigned long long>(pk));
           }
         }
       }
     }
-    cluster_sync();
+    pp_sync<CL>();
     const int p = static_cast<int>(pick_bcast);
     load_seed(p, s);
     __syncthreads();
@@ -455,7 +626,7 @@ __global__ void __cluster_dims__(kPpCtas, 1, 1) __launch_bounds__(kPpThreads, 1)
     update_pass(s, false);
     __syncthreads();
   }
-  cluster_sync();  // no CTA leaves while another may still write into its shared memory
+  if constexpr (CL > 1) cluster_sync();  // no CTA leaves while another may still write into its shared memory
 }
 
 // Split float32 centroids into bf16 hi + lo parts, zero the padding rows, compute ||c||^2.
@@ -943,27 +1114,56 @@ int num_sms() {
 
 }  // namespace
 
-template <int E, bool F32>
-cudaError_t launch_pp_cluster(const void* X, int BH, int N, int k, const double* u, float* C, cudaStream_t s) {
-  const int per_cta = (N + kPpCtas - 1) / kPpCtas;
+template <int E, bool F32, int CL>
+cudaError_t launch_pp(const void* X, int BH, int N, int stride, int S, int k, const double* u, float* C,
+                      cudaStream_t s) {
+  const int per_cta = (S + CL - 1) / CL;
   const size_t smem = pp_smem_bytes(per_cta);
-  cudaError_t e = cudaFuncSetAttribute(kmeanspp_cluster_kernel<E, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kmeanspp_kernel2<E, F32, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kmeanspp_cluster_kernel<E, F32><<<BH * kPpCtas, kPpThreads, smem, s>>>(X, N, k, u, C);
-  return cudaGetLastError();
+  if constexpr (CL == 1) {
+    kmeanspp_kernel2<E, F32, 1><<<BH, kPpThreads, smem, s>>>(X, N, stride, S, k, u, C);
+    return cudaGetLastError();
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(BH * CL);
+    cfg.blockDim = dim3(kPpThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kmeanspp_kernel2<E, F32, CL>, X, N, stride, S, k, u, C);
+  }
+}
+
+template <int E, bool F32>
+cudaError_t launch_pp_any(const void* X, int BH, int N, int stride, int S, int k, const double* u, float* C,
+                          cudaStream_t s) {
+  if (S <= kPpMaxPerCta) return launch_pp<E, F32, 1>(X, BH, N, stride, S, k, u, C, s);
+  return launch_pp<E, F32, kPpClusterCtas>(X, BH, N, stride, S, k, u, C, s);
+}
+
+int kmeanspp_stride(int N, int seed_tokens) {
+  if (seed_tokens <= 0 || seed_tokens >= N) return 1;
+  return (N + seed_tokens - 1) / seed_tokens;
 }
 
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
-                            float* centroids, double* dist, int32_t* near, cudaStream_t s) {
-  const int per_cta = (N + kPpCtas - 1) / kPpCtas;
-  if (per_cta <= kPpMaxTokensPerCta) {
-    if (d == 128) return x_f32 ? launch_pp_cluster<4, true>(X, BH, N, k, u, centroids, s)
-                               : launch_pp_cluster<4, false>(X, BH, N, k, u, centroids, s);
-    return x_f32 ? launch_pp_cluster<2, true>(X, BH, N, k, u, centroids, s)
-                 : launch_pp_cluster<2, false>(X, BH, N, k, u, centroids, s);
+                            float* centroids, double* dist, int32_t* near, int seed_tokens, cudaStream_t s) {
+  const int stride = kmeanspp_stride(N, seed_tokens);
+  const int S = (N + stride - 1) / stride;
+  if ((S + kPpClusterCtas - 1) / kPpClusterCtas <= kPpMaxPerCta && !(x_f32 && d == 128)) {
+    if (d == 128) return launch_pp_any<4, false>(X, BH, N, stride, S, k, u, centroids, s);
+    return x_f32 ? launch_pp_any<2, true>(X, BH, N, stride, S, k, u, centroids, s)
+                 : launch_pp_any<2, false>(X, BH, N, stride, S, k, u, centroids, s);
   }
-  kmeanspp_kernel<<<BH, 1024, 0, s>>>(X, x_f32, N, d, k, u, centroids, dist, near);
+  kmeanspp_kernel<<<BH, 1024, 0, s>>>(X, x_f32, N, stride, d, k, u, centroids, dist, near);
   return cudaGetLastError();
 }
 

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libsvg2.so")
 SVG2_BF16, SVG2_F32 = 0, 1
 SVG2_INIT_GIVEN, SVG2_INIT_KMEANSPP = 0, 1
 MAX_CLUSTERS = 1024
+DEFAULT_SEED_TOKENS = 16384  # SVG2_DEFAULT_SEED_TOKENS
 
 _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeans", "svg2_select",
             "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
@@ -35,7 +36,8 @@ class Svg2Error(RuntimeError):
 
 class SvgParams(ctypes.Structure):
     _fields_ = [("nQ", ctypes.c_int), ("nK", ctypes.c_int), ("iters", ctypes.c_int), ("init", ctypes.c_int),
-                ("top_p", ctypes.c_float), ("scale", ctypes.c_float), ("fuse_unpermute", ctypes.c_int)]
+                ("top_p", ctypes.c_float), ("scale", ctypes.c_float), ("seed_tokens", ctypes.c_int),
+                ("fuse_unpermute", ctypes.c_int)]
 
 
 class SvgLayerOutputs(ctypes.Structure):
@@ -57,7 +59,7 @@ def lib() -> ctypes.CDLL:
         L.svg2_workspace_size.argtypes = [I, I, I, I, I, I, ctypes.POINTER(S)]
         L.svg2_check_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_uint32),
                                         ctypes.POINTER(ctypes.c_uint32)]
-        L.svg2_kmeans.argtypes = [P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, S, P]
+        L.svg2_kmeans.argtypes = [P, I, I, I, I, I, I, I, I, P, I, P, P, P, P, P, P, S, P]
         L.svg2_select.argtypes = [P, P, P, I, I, I, I, I, F, F, P, P, P, P, P, P, S, P]
         L.svg2_select_from_weights.argtypes = [P, P, I, I, I, I, F, P, P, P, P, P, S, P]
         L.svg2_sort.argtypes = [P, I, I, I, I, P, P, P, P, S, P]
@@ -136,9 +138,11 @@ def raise_on_device_error(ws: torch.Tensor, stream=None):
 
 def svg2_kmeans(X: torch.Tensor, k: int, iters: int, init: int, centroids: torch.Tensor, labels: torch.Tensor,
                 counts: torch.Tensor, ws: torch.Tensor, u: Optional[torch.Tensor] = None,
-                perm: Optional[torch.Tensor] = None, offsets: Optional[torch.Tensor] = None, stream=None):
+                perm: Optional[torch.Tensor] = None, offsets: Optional[torch.Tensor] = None,
+                seed_tokens: int = DEFAULT_SEED_TOKENS, stream=None):
     B, H, N, d = X.shape
-    _check(lib().svg2_kmeans(_p(X), _dtype(X), B, H, N, d, k, iters, init, _p(u), _p(centroids), _p(labels),
+    _check(lib().svg2_kmeans(_p(X), _dtype(X), B, H, N, d, k, iters, init, _p(u), int(seed_tokens), _p(centroids),
+                             _p(labels),
                              _p(counts), _p(perm), _p(offsets), _p(ws), ws.numel(), _stream(stream)), "svg2_kmeans")
 
 
@@ -218,9 +222,11 @@ class LayerParams:
     top_p: float = 0.9
     scale: float = 1.0 / 128 ** 0.5
     fuse_unpermute: int = 1
+    seed_tokens: int = DEFAULT_SEED_TOKENS
 
     def c(self) -> SvgParams:
-        return SvgParams(self.nQ, self.nK, self.iters, self.init, self.top_p, self.scale, self.fuse_unpermute)
+        return SvgParams(self.nQ, self.nK, self.iters, self.init, self.top_p, self.scale, self.seed_tokens,
+                         self.fuse_unpermute)
 
 
 def layer_output_buffers(B: int, H: int, N: int, nQ: int, nK: int, device="cuda") -> Dict[str, torch.Tensor]:

@@ -74,12 +74,12 @@ FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails va
 
 def test_kmeans_rejects_bad_arguments(L):
     P = None
-    args = lambda **kw: dict(dict(X=FAKE, dt=0, B=1, H=1, N=100, d=128, k=4, it=1, init=0, u=P, C=FAKE, lab=FAKE,
-                                  cnt=FAKE, perm=P, off=P, ws=FAKE, wsb=1 << 30), **kw)
+    args = lambda **kw: dict(dict(X=FAKE, dt=0, B=1, H=1, N=100, d=128, k=4, it=1, init=0, u=P, st=0, C=FAKE,
+                                  lab=FAKE, cnt=FAKE, perm=P, off=P, ws=FAKE, wsb=1 << 30), **kw)
     def call(**kw):
         a = args(**kw)
         return L.svg2_kmeans(a["X"], a["dt"], a["B"], a["H"], a["N"], a["d"], a["k"], a["it"], a["init"], a["u"],
-                             a["C"], a["lab"], a["cnt"], a["perm"], a["off"], a["ws"], a["wsb"], None)
+                             a["st"], a["C"], a["lab"], a["cnt"], a["perm"], a["off"], a["ws"], a["wsb"], None)
     assert call(X=None) == INVALID
     assert call(dt=7) == INVALID
     assert call(k=0) == INVALID
@@ -88,6 +88,8 @@ def test_kmeans_rejects_bad_arguments(L):
     assert call(it=0) == INVALID
     assert call(init=5) == INVALID
     assert call(init=1, u=None) == INVALID           # k-means++ needs its uniforms
+    assert call(st=-1) == INVALID
+    assert call(init=1, u=FAKE, N=100, k=40, st=30) == INVALID   # 34 candidates for 40 seeds
     assert call(ws=None) == WORKSPACE
     assert call(wsb=16) == WORKSPACE
     assert call(ws=ctypes.c_void_p(0x10010)) == WORKSPACE   # not 256-byte aligned
@@ -129,13 +131,13 @@ def test_attention_and_layer_reject_bad_arguments(L):
                               FAKE, 1 << 30, None) == INVALID
     assert L.svg2_sparse_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1000, 128, 4, 4, F(0.1), None, FAKE,
                               FAKE, 64, None) == WORKSPACE
-    p = SvgParams(4, 8, 2, 1, 0.9, 0.1, 1)
+    p = SvgParams(4, 8, 2, 1, 0.9, 0.1, 0, 1)
     args = [FAKE, FAKE, FAKE, 0, 1, 1, 1000, 128, ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 34,
             None]
-    bad = SvgParams(4, 8, 2, 1, 0.9, 0.1, 1)
+    bad = SvgParams(4, 8, 2, 1, 0.9, 0.1, 0, 1)
     bad.top_p = -1.0
     assert L.svg2_layer(*args[:8], ctypes.byref(bad), *args[9:]) == INVALID
-    bad = SvgParams(4, 8, 0, 1, 0.9, 0.1, 1)
+    bad = SvgParams(4, 8, 0, 1, 0.9, 0.1, 0, 1)
     assert L.svg2_layer(*args[:8], ctypes.byref(bad), *args[9:]) == INVALID
     assert L.svg2_layer(*args[:9], None, *args[10:]) == INVALID          # k-means++ without uniforms
     assert L.svg2_layer(*args[:16], 1024, None) == WORKSPACE

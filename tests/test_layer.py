@@ -17,7 +17,7 @@ from tests.gpu_helpers import bf16_dev, host, pool_layer_inputs, require_gpu, to
 MAX_ABS, MEAN_ABS = 2e-2, 2e-3
 
 
-def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1):
+def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1, seed_tokens=None):
     B, H, N, d = data["q"].shape
     conv = to_dev if cfg.dtype == "f32" else bf16_dev
     Q, K, V = conv(data["q"]), conv(data["k"]), conv(data["v"])
@@ -27,7 +27,8 @@ def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1):
     outs = svg2.layer_output_buffers(B, H, N, cfg.nQ, cfg.nK)
     ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK)
     prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP if init is None else init, top_p,
-                           float(np.float32(cfg.scale)), fuse)
+                           float(np.float32(cfg.scale)), fuse,
+                           svg2.DEFAULT_SEED_TOKENS if seed_tokens is None else seed_tokens)
     svg2.svg2_layer(Q, K, V, prm, cq, ck, O, ws, to_dev(data["uq"]), to_dev(data["uk"]), outs)
     torch.cuda.synchronize()
     svg2.raise_on_device_error(ws)
@@ -81,7 +82,8 @@ def test_layer_small_configs_every_head(oracle, cfg_name):
     for h in range(cfg.H):
         st = check_head(oracle, cfg, data, res, h, top_p)
         e2e = oracle.layer_head(data["q"][0, h], data["k"][0, h], data["v"][0, h], cfg.nQ, cfg.nK, cfg.iters, top_p,
-                                float(np.float32(cfg.scale)), data["uq"][0, h], data["uk"][0, h])
+                                float(np.float32(cfg.scale)), data["uq"][0, h], data["uk"][0, h],
+                                seed_tokens=svg2.DEFAULT_SEED_TOKENS)
         agree_q = float((res["labels_q"][0, h] == e2e["labels_q"]).mean())
         agree_k = float((res["labels_k"][0, h] == e2e["labels_k"]).mean())
         o_rel = float(np.linalg.norm(res["o"][0, h] - e2e["o"]) / np.linalg.norm(e2e["o"]))

@@ -17,14 +17,14 @@ def _xdev(cfg, x):
     return to_dev(x) if cfg.dtype == "f32" else bf16_dev(x)
 
 
-def _run(svg2, cfg, X, k, iters, init, C0=None, u=None):
+def _run(svg2, cfg, X, k, iters, init, C0=None, u=None, seed_tokens=0):
     B, H, N, d = X.shape
     Xd = _xdev(cfg, X)
     C = to_dev(C0.astype(np.float32)) if C0 is not None else torch.zeros(B, H, k, d, device="cuda")
     lab = torch.empty(B, H, N, dtype=torch.int32, device="cuda")
     cnt = torch.empty(B, H, k, dtype=torch.int32, device="cuda")
     ws = svg2.workspace(B, H, N, d, k, k)
-    svg2.svg2_kmeans(Xd, k, iters, init, C, lab, cnt, ws, u=None if u is None else to_dev(u))
+    svg2.svg2_kmeans(Xd, k, iters, init, C, lab, cnt, ws, u=None if u is None else to_dev(u), seed_tokens=seed_tokens)
     torch.cuda.synchronize()
     svg2.raise_on_device_error(ws)
     return host(C), host(lab), host(cnt)
@@ -46,10 +46,11 @@ def _check_assign(labels, ref_labels, d1, d2, what):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("cfg_name,heads,role", [("tiny", [0], "q"), ("tiny", [0], "k"), ("small", [0, 5], "q"),
-                                                 ("small", [0, 5], "k"), ("wan720p", [7], "k"),
-                                                 ("hunyuan720p", [3], "k")])
-def test_kmeanspp_then_lockstep_lloyd(oracle, cfg_name, heads, role):
+@pytest.mark.parametrize("cfg_name,heads,role,seed_tokens", [
+    ("tiny", [0], "q", 0), ("tiny", [0], "k", 0), ("small", [0, 5], "q", 0), ("small", [0, 5], "k", 0),
+    ("wan720p", [7], "k", 0), ("wan720p", [7], "q", 16384), ("wan720p", [2], "k", 16384),
+    ("hunyuan720p", [3], "k", 0), ("hunyuan720p", [5], "k", 16384)])
+def test_kmeanspp_then_lockstep_lloyd(oracle, cfg_name, heads, role, seed_tokens):
     svg2 = require_gpu()
     cfg = I.CONFIGS[cfg_name]
     data = pool_layer_inputs(cfg, heads)
@@ -58,17 +59,20 @@ def test_kmeanspp_then_lockstep_lloyd(oracle, cfg_name, heads, role):
     k = cfg.nQ if role == "q" else cfg.nK
     iters = cfg.iters
     # iteration 1 from k-means++ seeds (the seeds themselves are checked through it)
-    C1, lab1, cnt1 = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_KMEANSPP, u=u)
+    C1, lab1, cnt1 = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_KMEANSPP, u=u, seed_tokens=seed_tokens)
+    stride = oracle.seed_stride(X.shape[2], seed_tokens)
+    seeds0 = lambda h: oracle.kmeanspp(np.ascontiguousarray(X[0, h][::stride]), k, u[0, h])[1]
     stats = []
     for h in range(len(heads)):
-        _, C0 = oracle.kmeanspp(X[0, h], k, u[0, h])
+        C0 = seeds0(h)
         ref_lab, d1, d2 = oracle.assign(X[0, h], C0)
         stats.append(_check_assign(lab1[0, h], ref_lab, d1, d2, f"{cfg_name} head {heads[h]} iter 1"))
         Cref, cref = oracle.update(X[0, h], lab1[0, h], C0)          # same labels: exact up to fp32 rounding
         np.testing.assert_allclose(C1[0, h], Cref.astype(np.float32), rtol=0, atol=0)
         assert np.array_equal(cnt1[0, h], cref)
     # lockstep: every further iteration starts from the oracle's own centroids
-    Cor = np.stack([oracle.lloyd(X[0, h], oracle.kmeanspp(X[0, h], k, u[0, h])[1], 1)[0] for h in range(len(heads))])
+    Cor = np.stack([oracle.lloyd(X[0, h], seeds0(h), 1)[0] for h in range(len(heads))])
+    flipped_clusters = 0
     for it in range(2, iters + 1):
         Cin = Cor.astype(np.float32).astype(np.float64)
         C, lab, cnt = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_GIVEN, C0=Cin[None])
@@ -76,11 +80,23 @@ def test_kmeanspp_then_lockstep_lloyd(oracle, cfg_name, heads, role):
         for h in range(len(heads)):
             ref_lab, d1, d2 = oracle.assign(X[0, h], Cin[h])
             stats.append(_check_assign(lab[0, h], ref_lab, d1, d2, f"{cfg_name} head {heads[h]} iter {it}"))
+            # the update given the GPU's own labels is exact (float64 sums in the oracle's order)
+            Cg, cg = oracle.update(X[0, h], lab[0, h], Cin[h])
+            np.testing.assert_array_equal(C[0, h], Cg.astype(np.float32))
+            assert np.array_equal(cnt[0, h], cg)
+            # against the oracle's labels: every cluster no near-tie flip touched is within 1e-3
             Cref, cref = oracle.update(X[0, h], ref_lab, Cin[h])
-            assert _rel_centroid_err(C[0, h], Cref, cref) <= 1e-3
+            moved = lab[0, h] != ref_lab
+            touched = np.zeros(k, bool)
+            touched[lab[0, h][moved]] = True
+            touched[ref_lab[moved]] = True
+            flipped_clusters += int(touched.sum())
+            keep = ~touched
+            assert _rel_centroid_err(C[0, h][keep], Cref[keep], cref[keep]) <= 1e-3
             nxt.append(oracle.update(X[0, h], oracle.assign(X[0, h], Cor[h])[0], Cor[h])[0])
         Cor = np.stack(nxt)
-    print(f"{cfg_name}/{role}: (near-tie mismatches, near-ties) per head and iteration: {stats}")
+    print(f"{cfg_name}/{role}: clusters touched by near-tie flips over the lockstep run: {flipped_clusters}")
+    print(f"{cfg_name}/{role} seed_tokens={seed_tokens}: (near-tie mismatches, near-ties) per head/iteration: {stats}")
 
 
 @pytest.mark.gpu
