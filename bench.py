@@ -71,6 +71,23 @@ def gen_inputs(cfg, step=0):
     return {k: np.stack([p[k] for p in parts])[None] for k in parts[0]}
 
 
+# DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 243.4 MB + 70.2 MB), scaled by heads; valid
+# only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
+ATTN_TRAFFIC = {"sha256": "e853a74c2f1e353f865310ab0cc119bbb5313c7e949f2c6ed77f7952024473f6",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 243.374080e6 + 70.152704e6,
+                "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
+
+
+def attn_traffic(cfg):
+    import hashlib
+    src = os.path.join(ROOT, "sparse_attention_video_head_b200", "csrc", "svg2_attn.cu")
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != ATTN_TRAFFIC["sha256"] or cfg.name != ATTN_TRAFFIC["workload"]:
+            return None
+    return ATTN_TRAFFIC["bytes_captured"] * cfg.B * cfg.H / ATTN_TRAFFIC["heads_captured"]
+
+
 # ------------------------------------------------------------------------------------------ oracle
 def oracle_sample(cfg, top_p, rows=96, head=0, seed_tokens=0):
     """The CPU oracle on a bounded sample of the layer: one head's k-means (Q and K), selection and
@@ -341,7 +358,8 @@ def main():
                      "peak": P["bf16_sustained"], "unit": "TFLOP/s",
                      "frac": achieved_tflops / P["bf16_sustained"],
                      "peak_source": P["source"] + " bf16 cuBLAS, sustained (kernel timed inside a long step)",
-                     "traffic": None},
+                     "traffic": attn_traffic(cfg), "traffic_unit": "bytes per launch",
+                     "algorithmic_bytes": 4.0 * B * H * N * d * 2},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches * args.steps,
         "clocks": clk.summary(), "stages_ms": stage_ms, "density": density,
         "attn_tflop_actual": actual_flops / 1e12, "attn_tflop_dense_equiv": dense_flops / 1e12,
