@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
 constexpr int kPpThreads = 512;
 constexpr int kPpWarps = kPpThreads / 32;
 constexpr int kPpMaxPerCta = 15360;   // 10 bytes of state per candidate: 150 KB of shared memory
-constexpr int kPpClusterCtas = 8;
+constexpr int kPpMaxCluster = 16;     // non-portable cluster size limit
 
 __host__ __device__ constexpr size_t pp_smem_bytes(int per_cta) {
   return static_cast<size_t>(per_cta) * 10 + 16;
@@ -309,25 +309,24 @@ __device__ __forceinline__ double pp_exact(const float (&v)[E], const float* cs,
   return __shfl_sync(0xffffffffu, acc, 0);  // lane 0's summation order decides
 }
 
-template <int CL>
-__device__ __forceinline__ void pp_sync() {
-  if constexpr (CL > 1) cluster_sync();
+__device__ __forceinline__ void pp_sync(int ncl) {
+  if (ncl > 1) cluster_sync();
   else __syncthreads();
 }
 
-template <int CL>
-__device__ __forceinline__ void pp_bcast_u64(unsigned long long* var, unsigned long long v) {
-  if constexpr (CL > 1) {
-    for (uint32_t r = 0; r < CL; ++r) st_cluster_u64(var, r, v);
+// Store v into `var` of every CTA of the cluster (this CTA's own copy when there is no cluster).
+__device__ __forceinline__ void pp_bcast_u64(unsigned long long* var, unsigned long long v, int ncl) {
+  if (ncl > 1) {
+    for (int r = 0; r < ncl; ++r) st_cluster_u64(var, static_cast<uint32_t>(r), v);
   } else {
     *var = v;
   }
 }
 
 // k-means++ seeding over a candidate set: every `stride`-th token (stride 1 = all tokens), S in all.
-// One (b,h) runs on CL CTAs: CL = 1 keeps the whole candidate set's state (D^2 in float64 and the
-// nearest seed) in one CTA's shared memory; CL = kPpClusterCtas spreads it over a thread-block
-// cluster and exchanges the per-seed totals through distributed shared memory.  Lane l of warp w
+// One (b,h) runs on the CTAs of one thread-block cluster (1 to kPpMaxCluster of them, chosen at
+// launch): each keeps its share of the candidates' state (D^2 in float64 and the nearest seed) in
+// shared memory, and the per-seed totals and the pick travel through distributed shared memory.  Lane l of warp w
 // owns a contiguous piece of the warp's candidates, so a lane's running fixed-point weight total is
 // its piece's total and the sampling search needs no division until the final piece scan.
 // Per seed: ||c_new - c_near||^2 >= 4.0001 D^2 proves a candidate cannot get closer; the rest get
@@ -336,7 +335,7 @@ __device__ __forceinline__ void pp_bcast_u64(unsigned long long* var, unsigned l
 // fixed butterfly across lanes, lane 0's order).  That can differ from a sequential sum in the last
 // bit, which moves the fixed-point weight floor(D^2 / M0 * 2^32) only when D^2 / M0 * 2^32 lies
 // within ~1e-6 of an integer, and changes a seed only if the sampling target sits exactly on it.
-template <int E, bool F32, int CL>
+template <int E, bool F32>
 __global__ void __launch_bounds__(kPpThreads, 1)
     kmeanspp_kernel2(const void* __restrict__ X, int N, int stride, int S, int k, const double* __restrict__ u,
                      float* __restrict__ C) {
@@ -345,12 +344,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   __shared__ float cs[D];
   __shared__ float ss[1024];
   __shared__ unsigned long long wsum[kPpWarps];
-  __shared__ unsigned long long cta_tot[CL];
-  __shared__ unsigned long long cta_max[CL];
+  __shared__ unsigned long long cta_tot[kPpMaxCluster];
+  __shared__ unsigned long long cta_max[kPpMaxCluster];
   __shared__ unsigned long long pick_bcast;
   __shared__ unsigned long long hit_base;
   __shared__ int hit_warp;
-  const uint32_t rank = CL > 1 ? cluster_rank() : 0u;
+  const int CL = static_cast<int>(cluster_nctas());  // 1 for a launch without clusters
+  const uint32_t rank = cluster_rank();
   const int bh = blockIdx.x / CL;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_cta = (S + CL - 1) / CL;
@@ -536,9 +536,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   if (threadIdx.x == 0) {
     double mx = 0.0;
     for (int w = 0; w < kPpWarps; ++w) mx = fmax(mx, __longlong_as_double(static_cast<long long>(wsum[w])));
-    pp_bcast_u64<CL>(&cta_max[rank], static_cast<unsigned long long>(__double_as_longlong(mx)));
+    pp_bcast_u64(&cta_max[rank], static_cast<unsigned long long>(__double_as_longlong(mx)), CL);
   }
-  pp_sync<CL>();
+  pp_sync(CL);
   for (int r = 0; r < CL; ++r) M0 = fmax(M0, __longlong_as_double(static_cast<long long>(cta_max[r])));
   for (int c = plo; c < phi; ++c) qsum += fixed_weight(Ds[c - lo], M0);
 
@@ -552,9 +552,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (threadIdx.x == 0) {
       unsigned long long t = 0;
       for (int w = 0; w < kPpWarps; ++w) t += wsum[w];
-      pp_bcast_u64<CL>(&cta_tot[rank], t);
+      pp_bcast_u64(&cta_tot[rank], t, CL);
     }
-    pp_sync<CL>();
+    pp_sync(CL);
     unsigned long long U = 0, base = 0;
     for (int r = 0; r < CL; ++r) {
       if (r < static_cast<int>(rank)) base += cta_tot[r];
@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (U == 0ull) {
       if (threadIdx.x == 0 && rank == 0) {
         const long long p = static_cast<long long>(floor(uh[s] * static_cast<double>(S)));
-        pp_bcast_u64<CL>(&pick_bcast, static_cast<unsigned long long>(p >= S ? S - 1 : p));
+        pp_bcast_u64(&pick_bcast, static_cast<unsigned long long>(p >= S ? S - 1 : p), CL);
       }
     } else {
       unsigned long long target = static_cast<unsigned long long>(floor(uh[s] * static_cast<double>(U)));
@@ -598,35 +598,48 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 break;
               }
             }
-            pp_bcast_u64<CL>(&pick_bcast, static_cast<unsigned long long>(pk));
+            pp_bcast_u64(&pick_bcast, static_cast<unsigned long long>(pk), CL);
           }
         }
       }
     }
-    pp_sync<CL>();
+    pp_sync(CL);
     const int p = static_cast<int>(pick_bcast);
     load_seed(p, s);
     __syncthreads();
-    // ---- squared distances from the new seed to every earlier seed (float32, for pruning)
-    for (int a = threadIdx.x; a < s; a += blockDim.x) {
-      const float* ca = Ch + static_cast<size_t>(a) * D;
-      float acc = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < D; i += 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(ca + i);
-        const float d0 = cs[i] - c4.x, d1 = cs[i + 1] - c4.y, d2 = cs[i + 2] - c4.z, d3 = cs[i + 3] - c4.w;
-        acc = fmaf(d0, d0, acc);
-        acc = fmaf(d1, d1, acc);
-        acc = fmaf(d2, d2, acc);
-        acc = fmaf(d3, d3, acc);
+    // ---- squared distances from the new seed to every earlier seed (float32, for pruning): warp w
+    // takes seeds w*32 .. w*32+31 of each block of 32*kPpWarps, all 32 rows in flight at once
+    for (int a0 = warp * 32; a0 < s; a0 += 32 * kPpWarps) {
+      float pr[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        pr[r] = 0.f;
+        if (a0 + r < s) {
+          const float* ca = Ch + static_cast<size_t>(a0 + r) * D + lane * E;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float df = cs[lane * E + e] - ca[e];
+            pr[r] = fmaf(df, df, pr[r]);
+          }
+        }
       }
-      ss[a] = acc;
+#pragma unroll
+      for (int o = 16, n = 16; o > 0; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int q = 0; q < n; ++q) {
+          const float keep = upper ? pr[q + n] : pr[q];
+          const float send = upper ? pr[q] : pr[q + n];
+          pr[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      if (a0 + lane < s) ss[a0 + lane] = pr[0];
     }
     __syncthreads();
     update_pass(s, false);
     __syncthreads();
   }
-  if constexpr (CL > 1) cluster_sync();  // no CTA leaves while another may still write into its shared memory
+  if (CL > 1) cluster_sync();  // no CTA leaves while another may still write into its shared memory
 }
 
 // Split float32 centroids into bf16 hi + lo parts, zero the padding rows, compute ||c||^2.
@@ -1114,39 +1127,58 @@ int num_sms() {
 
 }  // namespace
 
-template <int E, bool F32, int CL>
-cudaError_t launch_pp(const void* X, int BH, int N, int stride, int S, int k, const double* u, float* C,
-                      cudaStream_t s) {
-  const int per_cta = (S + CL - 1) / CL;
-  const size_t smem = pp_smem_bytes(per_cta);
-  cudaError_t e = cudaFuncSetAttribute(kmeanspp_kernel2<E, F32, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  if constexpr (CL == 1) {
-    kmeanspp_kernel2<E, F32, 1><<<BH, kPpThreads, smem, s>>>(X, N, stride, S, k, u, C);
-    return cudaGetLastError();
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(BH * CL);
+// Launch configuration of the seeding kernel for `ncl` CTAs per (b,h).
+struct PpLaunch {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  PpLaunch(int BH, int ncl, size_t smem, cudaStream_t s) : cfg{}, attr{} {
+    cfg.gridDim = dim3(BH * ncl);
     cfg.blockDim = dim3(kPpThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.x = ncl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kmeanspp_kernel2<E, F32, CL>, X, N, stride, S, k, u, C);
   }
-}
+};
 
+// Cluster size for BH problems of S candidates: the largest size (fewer candidates per CTA, so a
+// shorter pass) whose clusters all fit on the GPU at once; past that, more clusters only queue.
 template <int E, bool F32>
-cudaError_t launch_pp_any(const void* X, int BH, int N, int stride, int S, int k, const double* u, float* C,
-                          cudaStream_t s) {
-  if (S <= kPpMaxPerCta) return launch_pp<E, F32, 1>(X, BH, N, stride, S, k, u, C, s);
-  return launch_pp<E, F32, kPpClusterCtas>(X, BH, N, stride, S, k, u, C, s);
+cudaError_t launch_pp(const void* X, int BH, int N, int stride, int S, int k, const double* u, float* C,
+                      cudaStream_t s) {
+  auto kern = kmeanspp_kernel2<E, F32>;
+  const size_t smem_max = pp_smem_bytes(kPpMaxPerCta);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+  const int cl_min = (S + kPpMaxPerCta - 1) / kPpMaxPerCta;
+  if (cl_min > kPpMaxCluster) return cudaErrorInvalidValue;
+  int best = cl_min;
+  double best_cost = 0.0;
+  for (int ncl = cl_min; ncl <= kPpMaxCluster; ++ncl) {
+    const int per_cta = (S + ncl - 1) / ncl;
+    if (per_cta < 32 * kPpWarps && ncl > cl_min) break;  // fewer than one candidate per lane
+    PpLaunch L(BH, ncl, pp_smem_bytes(per_cta), s);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &L.cfg) != cudaSuccess || active < 1) {
+      cudaGetLastError();  // a size this GPU cannot co-schedule: not a launch error
+      continue;
+    }
+    const int waves = (BH + active - 1) / active;
+    // a pass costs about its candidates plus a fixed part (the totals, the pick, the new seed)
+    const double cost = waves * (static_cast<double>(per_cta) + (ncl > 1 ? 600.0 : 200.0));
+    if (best_cost == 0.0 || cost < best_cost) {
+      best_cost = cost;
+      best = ncl;
+    }
+  }
+  PpLaunch L(BH, best, pp_smem_bytes((S + best - 1) / best), s);
+  return cudaLaunchKernelEx(&L.cfg, kern, X, N, stride, S, k, u, C);
 }
 
 int kmeanspp_stride(int N, int seed_tokens) {
@@ -1158,10 +1190,10 @@ cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int
                             float* centroids, double* dist, int32_t* near, int seed_tokens, cudaStream_t s) {
   const int stride = kmeanspp_stride(N, seed_tokens);
   const int S = (N + stride - 1) / stride;
-  if ((S + kPpClusterCtas - 1) / kPpClusterCtas <= kPpMaxPerCta && !(x_f32 && d == 128)) {
-    if (d == 128) return launch_pp_any<4, false>(X, BH, N, stride, S, k, u, centroids, s);
-    return x_f32 ? launch_pp_any<2, true>(X, BH, N, stride, S, k, u, centroids, s)
-                 : launch_pp_any<2, false>(X, BH, N, stride, S, k, u, centroids, s);
+  if ((S + kPpMaxCluster - 1) / kPpMaxCluster <= kPpMaxPerCta && !(x_f32 && d == 128)) {
+    if (d == 128) return launch_pp<4, false>(X, BH, N, stride, S, k, u, centroids, s);
+    return x_f32 ? launch_pp<2, true>(X, BH, N, stride, S, k, u, centroids, s)
+                 : launch_pp<2, false>(X, BH, N, stride, S, k, u, centroids, s);
   }
   kmeanspp_kernel<<<BH, 1024, 0, s>>>(X, x_f32, N, stride, d, k, u, centroids, dist, near);
   return cudaGetLastError();
