@@ -102,6 +102,18 @@ SVG2_API int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, i
                 int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * k-means++ seeding alone (Method (1): the cold start of svg2_kmeans with SVG2_INIT_KMEANSPP).
+ * Per (b, h): seed 0 is candidate floor(u_0 * S); seed s is the first candidate whose running sum
+ * of floor(D^2 / M0 * 2^32) exceeds floor(u_s * U), where D^2 is the float64 squared distance to
+ * the nearest earlier seed, M0 the largest D^2 after seed 0 and U the sum of all weights (a
+ * uniform pick when U = 0).  Candidates are every ceil(N / seed_tokens)-th token (0 = all).
+ *   u          float64 [B, H, k] uniforms in [0, 1).
+ *   centroids  float32 [B, H, k, d], out: the seed rows.
+ * Same sizes, dtype and workspace rules as svg2_kmeans; the candidate count must be >= k. */
+SVG2_API int svg2_kmeanspp(const void* X, int dtype, int B, int H, int N, int d, int k, const double* u,
+                  int seed_tokens, float* centroids, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Critical-cluster selection (section 4.2, Eq. 1-2; Method (3)).  Per (b, h, Q-cluster i):
  * l_ij = (cq_i . ck_j) * scale, w_ij = count_k[j] * exp(l_ij - max_j l_ij) over non-empty j
  * (w = 0 for empty j), then top-p: the shortest prefix of the K clusters ordered by (w desc, j asc)

@@ -100,7 +100,7 @@ cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int
                        const KmeansScratch& s, DeviceStatus* st, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
   if (init == SVG2_INIT_KMEANSPP)
-    e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, seed_tokens, stream);
+    e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, s.c_hi, seed_tokens, st, stream);
   if (e == cudaSuccess) e = launch_centroid_prep(C, BH, k, d, s.c_hi, s.c_lo, s.c_norm, stream);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
     e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, st, stream);
@@ -121,6 +121,22 @@ cudaError_t make_tmap_bf16_rows(void* map, const void* base, uint64_t rows, uint
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                        dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_bf16_3d(void* map, const void* base, uint32_t d, uint64_t rows, uint64_t planes,
+                              uint64_t row_pitch, uint64_t plane_pitch, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  if (!aligned(base, 16) || rows == 0 || planes == 0 || box_rows == 0 || box_rows > 256) return cudaErrorInvalidValue;
+  if (row_pitch % 16 != 0 || plane_pitch % 16 != 0) return cudaErrorInvalidValue;
+  const cuuint64_t dims[3] = {d, rows, planes};
+  const cuuint64_t strides[2] = {row_pitch, plane_pitch};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
                         dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -174,6 +190,30 @@ int svg2_check_status(void* ws, void* stream, int* device_status, uint32_t* wher
     info[1] = h.info1;
   }
   return SVG2_OK;
+}
+
+int svg2_kmeanspp(const void* X, int dtype, int B, int H, int N, int d, int k, const double* u, int seed_tokens,
+                  float* centroids, void* ws, size_t ws_bytes, void* stream) {
+  try {
+    int r = check_sizes(B, H, N, d);
+    if (r == SVG2_OK) r = check_k(k, N);
+    if (r != SVG2_OK) return r;
+    if (!valid_dtype(dtype) || X == nullptr || u == nullptr || centroids == nullptr || seed_tokens < 0)
+      return SVG2_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(centroids, 16)) return SVG2_ERR_INVALID_ARG;
+    if ((N + kmeanspp_stride(N, seed_tokens) - 1) / kmeanspp_stride(N, seed_tokens) < k) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+    KmeansScratch s;
+    carve_kmeans(c, BH, N, d, k, s, false);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    return to_status(launch_kmeanspp(X, dtype == SVG2_F32, BH, N, d, k, u, centroids, s.pp_dist, s.pp_near,
+                                     s.c_hi, seed_tokens, st, static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
 }
 
 int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int iters, int init, const double* u,

@@ -31,6 +31,10 @@ enum : uint32_t {
   kWhereSelftest = 6,
   kWhereAssignTail = 7,
   kWhereAttnDrain = 8,
+  kWhereSeedProducer = 9,
+  kWhereSeedMma = 10,
+  kWhereSeedEpilogue = 11,
+  kWhereSeedDrain = 12,
 };
 
 constexpr int kStatusBytes = 256;
@@ -112,7 +116,13 @@ cudaError_t launch_unpermute(const void* Op, const int32_t* perm, int BH, int N,
                              cudaStream_t s);
 
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
-                            float* centroids, double* dist, int32_t* near, int seed_tokens, cudaStream_t s);
+                            float* centroids, double* dist, int32_t* near, uint16_t* seeds_bf16, int seed_tokens,
+                            DeviceStatus* st, cudaStream_t s);
+// k-means++ seeding on the tensor cores (bf16, d = 128); returns cudaErrorNotSupported for shapes
+// it does not take, so that the caller can use the CUDA-core kernels.
+// seeds_bf16: scratch of BH * k * d bf16 (the seeds' rows, for the seed-to-seed distances).
+cudaError_t launch_kmeanspp_tc(const void* X, int BH, int N, int stride, int S, int k, const double* u,
+                               float* centroids, uint16_t* seeds_bf16, DeviceStatus* st, cudaStream_t s);
 // Spacing of the k-means++ candidates: every stride-th token, so that at most seed_tokens are used.
 int kmeanspp_stride(int N, int seed_tokens);
 cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, uint16_t* c_hi, uint16_t* c_lo,
@@ -140,5 +150,10 @@ cudaError_t launch_selftest_mma(const void* A, const void* Bm, int n, const void
 // Tensor map over a [rows, d] bf16 matrix with a box of 64 columns x box_rows rows, 128B swizzle.
 cudaError_t make_tmap_bf16_rows(void* map /* CUtensorMap* */, const void* base, uint64_t rows, uint32_t d,
                                 uint32_t box_rows);
+
+// Tensor map over `planes` matrices of `rows` rows x d bf16 columns with the given pitches in bytes
+// (a row pitch above d * 2 selects every n-th row), box of 64 columns x box_rows rows, 128B swizzle.
+cudaError_t make_tmap_bf16_3d(void* map /* CUtensorMap* */, const void* base, uint32_t d, uint64_t rows,
+                              uint64_t planes, uint64_t row_pitch, uint64_t plane_pitch, uint32_t box_rows);
 
 }  // namespace svg2

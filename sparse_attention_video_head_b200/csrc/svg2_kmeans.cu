@@ -1187,9 +1187,14 @@ int kmeanspp_stride(int N, int seed_tokens) {
 }
 
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
-                            float* centroids, double* dist, int32_t* near, int seed_tokens, cudaStream_t s) {
+                            float* centroids, double* dist, int32_t* near, uint16_t* seeds_bf16, int seed_tokens,
+                            DeviceStatus* st, cudaStream_t s) {
   const int stride = kmeanspp_stride(N, seed_tokens);
   const int S = (N + stride - 1) / stride;
+  if (!x_f32 && d == 128) {
+    const cudaError_t e = launch_kmeanspp_tc(X, BH, N, stride, S, k, u, centroids, seeds_bf16, st, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if ((S + kPpMaxCluster - 1) / kPpMaxCluster <= kPpMaxPerCta && !(x_f32 && d == 128)) {
     if (d == 128) return launch_pp<4, false>(X, BH, N, stride, S, k, u, centroids, s);
     return x_f32 ? launch_pp<2, true>(X, BH, N, stride, S, k, u, centroids, s)

@@ -21,7 +21,7 @@ SVG2_INIT_GIVEN, SVG2_INIT_KMEANSPP = 0, 1
 MAX_CLUSTERS = 1024
 DEFAULT_SEED_TOKENS = 16384  # SVG2_DEFAULT_SEED_TOKENS
 
-_EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeans", "svg2_select",
+_EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeanspp", "svg2_kmeans", "svg2_select",
             "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
             "svg2_unpermute", "svg2_layer", "svg2_selftest_mma", "svg2_sparse_attn_noalloc")
 
@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
         L.svg2_workspace_size.argtypes = [I, I, I, I, I, I, ctypes.POINTER(S)]
         L.svg2_check_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_uint32),
                                         ctypes.POINTER(ctypes.c_uint32)]
+        L.svg2_kmeanspp.argtypes = [P, I, I, I, I, I, I, P, I, P, P, S, P]
         L.svg2_kmeans.argtypes = [P, I, I, I, I, I, I, I, I, P, I, P, P, P, P, P, P, S, P]
         L.svg2_select.argtypes = [P, P, P, I, I, I, I, I, F, F, P, P, P, P, P, P, S, P]
         L.svg2_select_from_weights.argtypes = [P, P, I, I, I, I, F, P, P, P, P, P, S, P]
@@ -134,6 +135,13 @@ def raise_on_device_error(ws: torch.Tensor, stream=None):
     code, where, info = svg2_check_status(ws, stream)
     if code != 0:
         raise Svg2Error(code, f"device status (kernel tag {where}, info {info})")
+
+
+def svg2_kmeanspp(X: torch.Tensor, k: int, u: torch.Tensor, centroids: torch.Tensor, ws: torch.Tensor,
+                  seed_tokens: int = DEFAULT_SEED_TOKENS, stream=None):
+    B, H, N, d = X.shape
+    _check(lib().svg2_kmeanspp(_p(X), _dtype(X), B, H, N, d, k, _p(u), int(seed_tokens), _p(centroids), _p(ws),
+                               ws.numel(), _stream(stream)), "svg2_kmeanspp")
 
 
 def svg2_kmeans(X: torch.Tensor, k: int, iters: int, init: int, centroids: torch.Tensor, labels: torch.Tensor,

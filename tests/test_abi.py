@@ -95,6 +95,22 @@ def test_kmeans_rejects_bad_arguments(L):
     assert call(ws=ctypes.c_void_p(0x10010)) == WORKSPACE   # not 256-byte aligned
 
 
+def test_kmeanspp_rejects_bad_arguments(L):
+    def call(X=FAKE, dt=0, B=1, H=1, N=100, d=128, k=4, u=FAKE, st=0, C=FAKE, ws=FAKE, wsb=1 << 30):
+        return L.svg2_kmeanspp(X, dt, B, H, N, d, k, u, st, C, ws, wsb, None)
+    assert call(X=None) == INVALID
+    assert call(u=None) == INVALID
+    assert call(C=None) == INVALID
+    assert call(dt=7) == INVALID
+    assert call(k=0) == INVALID
+    assert call(k=101) == INVALID
+    assert call(d=96) == UNSUPPORTED
+    assert call(st=-1) == INVALID
+    assert call(N=100, k=40, st=30) == INVALID   # 34 candidates for 40 seeds
+    assert call(ws=None) == WORKSPACE
+    assert call(wsb=16) == WORKSPACE
+
+
 def test_select_and_topp_reject_bad_arguments(L):
     F = ctypes.c_float
     assert L.svg2_select(FAKE, FAKE, FAKE, 1, 1, 4, 8, 128, F(0.0), F(0.1), None, FAKE, FAKE, FAKE, None, FAKE,

@@ -45,6 +45,53 @@ def _check_assign(labels, ref_labels, d1, d2, what):
     return int(diff.sum()), int(tie.sum())
 
 
+def _seeds(svg2, X, k, u, seed_tokens, dev_x):
+    B, H, N, d = X.shape
+    C = torch.zeros(B, H, k, d, device="cuda")
+    ws = svg2.workspace(B, H, N, d, k, k)
+    svg2.svg2_kmeanspp(dev_x, k, to_dev(u), C, ws, seed_tokens=seed_tokens)
+    torch.cuda.synchronize()
+    svg2.raise_on_device_error(ws)
+    return host(C)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg_name,heads,role,seed_tokens", [
+    ("tiny", [0], "k", 0),                     # float32, d = 64 (CUDA-core seeding)
+    ("small", [0, 3], "k", 0),                 # 12480 candidates, k = 256, clusters of several CTAs
+    ("small", [1], "q", 5000),                 # stride 3: 4160 candidates, ragged last tile
+    ("small", [2], "k", 300),                  # stride 42: 298 candidates for 256 seeds, one CTA
+    ("wan720p", [4], "q", 16384), ("wan720p", [9], "k", 16384),
+    ("wan720p", [1], "k", 0),                  # all 75600 tokens: 13+ CTAs per head
+    ("hunyuan720p", [6], "k", 16384)])         # k = 1000
+def test_kmeanspp_seeds_bit_exact(oracle, cfg_name, heads, role, seed_tokens):
+    """The seeds are the oracle's: same fixed-point D^2 sampling, float64 D^2 in the same order."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS[cfg_name]
+    data = pool_layer_inputs(cfg, heads)
+    X, u = data[role], data["u" + role]
+    k = cfg.nQ if role == "q" else cfg.nK
+    C = _seeds(svg2, X, k, u, seed_tokens, _xdev(cfg, X))
+    stride = oracle.seed_stride(X.shape[2], seed_tokens)
+    for h in range(len(heads)):
+        _, Cref = oracle.kmeanspp(np.ascontiguousarray(X[0, h][::stride]), k, u[0, h])
+        bad = np.nonzero((C[0, h] != Cref.astype(np.float32)).any(axis=1))[0]
+        assert bad.size == 0, f"{cfg_name} head {heads[h]}: first differing seed {bad[:1]} of {k}"
+
+
+@pytest.mark.gpu
+def test_kmeanspp_seeds_with_duplicate_tokens(oracle):
+    """Three distinct rows repeated: after three seeds every D^2 is 0, so the rest are uniform picks."""
+    svg2 = require_gpu()
+    rng = np.random.default_rng(11)
+    base = I.round_to_bf16(rng.standard_normal((3, 128)).astype(np.float32))
+    X = base[rng.integers(0, 3, size=4096)][None, None].copy()
+    u = rng.random((1, 1, 8))
+    C = _seeds(svg2, X, 8, u, 0, bf16_dev(X))
+    _, Cref = oracle.kmeanspp(X[0, 0], 8, u[0, 0])
+    np.testing.assert_array_equal(C[0, 0], Cref.astype(np.float32))
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("cfg_name,heads,role,seed_tokens", [
     ("tiny", [0], "q", 0), ("tiny", [0], "k", 0), ("small", [0, 5], "q", 0), ("small", [0, 5], "k", 0),
