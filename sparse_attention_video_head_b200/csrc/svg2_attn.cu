@@ -38,10 +38,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 32 scores of a row, this many (the last ones) get 2^x from a polynomial on the FMA pipe
 // instead of the MUFU, which would otherwise bound the softmax.
-constexpr int kEmuPerChunk = 12;
+constexpr int kEmuPerChunk = 0;
 
 struct AttnBars {
-  uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], o_full, mma_done;
+  uint64_t q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], p_full[2], o_full, mma_done;
   uint32_t tmem_base;
   int32_t L;
   int32_t nranges;
@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->k_full[i]), 128);
       mbar_init(smem_u32(&bars->v_full[i]), 128);
-      mbar_init(smem_u32(&bars->kv_empty[i]), 1);
+      mbar_init(smem_u32(&bars->k_empty[i]), 1);
+      mbar_init(smem_u32(&bars->v_empty[i]), 1);
       mbar_init(smem_u32(&bars->s_full[i]), 1);
       mbar_init(smem_u32(&bars->p_full[i]), 4);
     }
@@ -198,9 +199,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nt = (L + 127) / 128;
 
   // Warpgroups 0-1 (softmax) take registers from warpgroups 2-3 (producer; MMA, allocator):
-  // 256 x 192 + 256 x 64 = 512 x 128, the launch's allocation.
+  // 256 x 192 + 128 x 40 + 128 x 88 = 512 x 128, the launch's allocation.
   if (warp >= 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
     // ---------------- Q by TMA, then MMA issue ----------------
     if (warp == 12 && elect_one()) {
       prefetch_tensormap(&tm_q);
@@ -217,30 +218,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t id_o = idesc_bf16_f32(128, D, 1);
       const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
+      // Descriptors of every operand tile, built once: stepping along K only moves the start
+      // address field (bits 0-13, in 16-byte units), which stays far below its 14-bit limit.
+      const uint64_t dq0 = sdesc_sw128(qa, 16, 1024), dq1 = sdesc_sw128(qb, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(kb, 16, 1024), dk1 = sdesc_sw128(kb + kTile, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(vb, 16384, 1024), dv1 = sdesc_sw128(vb + kTile, 16384, 1024);
       auto issue_s = [&](int x, int stage) {
-        const uint32_t qbase = x == 0 ? qa : qb;
-        const uint32_t kbase = kb + stage * kTile;
         const uint32_t d_tmem = tmem + x * 128;
+        const uint64_t aq = x == 0 ? dq0 : dq1, bk = stage == 0 ? dk0 : dk1;
 #pragma unroll
         for (int ks = 0; ks < kSteps; ++ks) {
-          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(d_tmem, sdesc_sw128(qbase + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024), id_s,
-                 ks > 0 ? 1u : 0u);
+          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+          mma_ss(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int x, int stage, int j) {
-        const uint32_t vbase = vb + stage * kTile;
         const uint32_t d_tmem = tmem + 256 + x * 128;
         const uint32_t p_tmem = tmem + x * 128;
+        const uint64_t bv = stage == 0 ? dv0 : dv1;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          mma_ts(d_tmem, p_tmem + ks * 8, sdesc_sw128(vbase + ks * 2048, 16384, 1024), id_o,
+          mma_ts(d_tmem, p_tmem + ks * 8, bv + static_cast<uint64_t>((ks * 2048) >> 4), id_o,
                  (j > 0 || ks > 0) ? 1u : 0u);
         }
       };
       if (ok && nt > 0) {
         ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma);
         if (ok) {
+          fence_proxy_async_smem();  // the key rows were written by cp.async (generic proxy)
           tc_fence_after();
           issue_s(0, 0);
           mma_commit(smem_u32(&bars->s_full[0]));
@@ -248,6 +253,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             issue_s(1, 0);
             mma_commit(smem_u32(&bars->s_full[1]));
           }
+          mma_commit(smem_u32(&bars->k_empty[0]));  // K(0) is not read again
         }
       }
       for (int j = 0; j < nt && ok; ++j) {
@@ -255,12 +261,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ok = mbar_wait(smem_u32(&bars->p_full[0]), j & 1, st, kWhereAttnMma);
         if (ok) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma);
         if (!ok) break;
+        fence_proxy_async_smem();
         tc_fence_after();
         issue_pv(0, stage, j);
         const bool more = j + 1 < nt;
         if (more) {
           ok = mbar_wait(smem_u32(&bars->k_full[stage ^ 1]), ((j + 1) >> 1) & 1, st, kWhereAttnMma);
           if (!ok) break;
+          fence_proxy_async_smem();
           tc_fence_after();
           issue_s(0, stage ^ 1);
           mma_commit(smem_u32(&bars->s_full[0]));
@@ -271,11 +279,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_after();
           issue_pv(1, stage, j);
         }
-        mma_commit(smem_u32(&bars->kv_empty[stage]));
+        mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
         if (has_b && more) {
           issue_s(1, stage ^ 1);
           mma_commit(smem_u32(&bars->s_full[1]));
         }
+        if (more) mma_commit(smem_u32(&bars->k_empty[stage ^ 1]));  // nor K(j+1) after its last S
       }
       if (ok) mma_commit(smem_u32(&bars->o_full));
       mma_commit(smem_u32(&bars->mma_done));
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) mbar_wait(qbar, 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
     }
   } else if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
     // ---------------- key/value gather producer ----------------
     // Warp w fills rows 32w..32w+31 of each key tile.  Each lane first finds the source row of one
     // stream position; then every cp.async instruction moves whole rows (16 lanes x 16 bytes per
@@ -297,9 +306,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int hf = my_chunk >> 3, cc = my_chunk & 7;
     for (int j = 0; j < nt; ++j) {
       const int stage = j & 1;
-      if (j >= 2) {
-        if (!mbar_wait(smem_u32(&bars->kv_empty[stage]), ((j >> 1) - 1) & 1, st, kWhereAttnProducer)) break;
-      }
       int p = j * 128 + wr0 + lane;
       if (p >= L) p = L - 1;
       // largest e with r_cum[e] <= p
@@ -311,26 +317,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int krow = r_start[lo] + (p - r_cum[lo]);
       krow = krow < 0 ? 0 : (krow >= N ? N - 1 : krow);
       const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
+      // K(j) may land as soon as the last S product of K(j-2) is done, V(j) once PV of V(j-2) is;
+      // each lands asynchronously and counts itself on its full barrier
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->k_empty[stage]), ((j >> 1) - 1) & 1, st,
+                                                       kWhereAttnProducer)))
+        break;
 #pragma unroll
       for (int it = 0; it < 32 / RPI; ++it) {
         const int rr = it * RPI + my_sub;  // row within the warp's 32
         const int src = __shfl_sync(0xffffffffu, krow, rr);
         cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * D + my_chunk * 8);
       }
-      cp_async_commit();
+      cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->v_empty[stage]), ((j >> 1) - 1) & 1, st,
+                                                       kWhereAttnProducer)))
+        break;
 #pragma unroll
       for (int it = 0; it < 32 / RPI; ++it) {
         const int rr = it * RPI + my_sub;
         const int src = __shfl_sync(0xffffffffu, krow, rr);
         cp_async16(vdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Vp + (head_row0 + src) * D + my_chunk * 8);
       }
-      cp_async_commit();
-      cp_async_wait<1>();
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&bars->k_full[stage]));
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&bars->v_full[stage]));
+      cp_async_mbar_arrive(smem_u32(&bars->v_full[stage]));
     }
     cp_async_wait<0>();
   } else {
@@ -362,8 +370,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_ld();
         float mx = -INFINITY;
         if (valid == 128) {
+          // four independent chains of three-input maxima
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int e = 0; e < 128; e += 2) mx = fmaxf(mx, fmaxf(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])));
+          for (int e = 0; e < 128; e += 8)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              m4[c] = fmax3(m4[c], __uint_as_float(sv[e + 2 * c]), __uint_as_float(sv[e + 2 * c + 1]));
+          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         } else {
 #pragma unroll
           for (int e = 0; e < 128; ++e)
@@ -393,9 +407,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // p = 2^(s * scale * log2(e) - m): the argument for two keys at once, the exponentials on
         // the MUFU, the row sum over float32 p (pairs), bf16 pairs written over S as the P operand
         const float2 scl = make_float2(sl2, sl2), negm = make_float2(-m_used, -m_used);
-        float2 lsum = make_float2(0.f, 0.f);
+        float2 lsum4[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          float2& lsum = lsum4[c];
+          lsum = make_float2(0.f, 0.f);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -413,7 +429,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_st16(t_s + c * 16, pk);
         }
-        l += lsum.x + lsum.y;
+        const float2 ls = add2(add2(lsum4[0], lsum4[1]), add2(lsum4[2], lsum4[3]));
+        l += ls.x + ls.y;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
