@@ -41,7 +41,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kEmuPerChunk = 0;
 
 struct AttnBars {
-  uint64_t q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], p_full[2], o_full, mma_done;
+  uint64_t q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], o_full, mma_done;
+  uint64_t s_full[2][2], p_full[2][2];  // [Q tile][S slot]
+  uint64_t pv_done[2];                  // one phase per PV product of each Q tile
   uint32_t tmem_base;
   int32_t L;
   int32_t nranges;
@@ -136,8 +138,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(smem_u32(&bars->v_full[i]), 128);
       mbar_init(smem_u32(&bars->k_empty[i]), 1);
       mbar_init(smem_u32(&bars->v_empty[i]), 1);
-      mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->p_full[i]), 4);
+      for (int t = 0; t < 2; ++t) {
+        mbar_init(smem_u32(&bars->s_full[i][t]), 1);
+        mbar_init(smem_u32(&bars->p_full[i][t]), 4);
+      }
+      mbar_init(smem_u32(&bars->pv_done[i]), 1);
     }
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->mma_done), 1);
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (has_b) tma_load_2d(qb + hf * 16384, &tm_q, hf * 64, y + 128, qbar);
       }
       bool ok = mbar_wait(qbar, 0, st, kWhereAttnMma);
-      const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
+      const uint32_t id_s = idesc_bf16_f32(128, 64, 0);
       const uint32_t id_o = idesc_bf16_f32(128, D, 1);
       const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
       // Descriptors of every operand tile, built once: stepping along K only moves the start
@@ -223,68 +228,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = sdesc_sw128(qa, 16, 1024), dq1 = sdesc_sw128(qb, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(kb, 16, 1024), dk1 = sdesc_sw128(kb + kTile, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(vb, 16384, 1024), dv1 = sdesc_sw128(vb + kTile, 16384, 1024);
-      auto issue_s = [&](int x, int stage) {
-        const uint32_t d_tmem = tmem + x * 128;
-        const uint64_t aq = x == 0 ? dq0 : dq1, bk = stage == 0 ? dk0 : dk1;
+      // S for sub-tile k of Q tile x: 64 keys (rows 64h.. of K tile k/2) into S slot k%2
+      auto issue_s = [&](int x, int k) {
+        const int h = k & 1, stage = (k >> 1) & 1;
+        const uint32_t d_tmem = tmem + x * 128 + h * 64;
+        const uint64_t aq = x == 0 ? dq0 : dq1;
+        const uint64_t bk = (stage == 0 ? dk0 : dk1) + static_cast<uint64_t>((h * 64 * 128) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kSteps; ++ks) {
           const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
           mma_ss(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
         }
+        mma_commit(smem_u32(&bars->s_full[x][h]));
       };
-      auto issue_pv = [&](int x, int stage, int j) {
+      // O_x += P(k) V(k): P is the bf16 pair-packed first 32 columns of S slot k%2
+      auto issue_pv = [&](int x, int k) {
+        const int h = k & 1, stage = (k >> 1) & 1;
         const uint32_t d_tmem = tmem + 256 + x * 128;
-        const uint32_t p_tmem = tmem + x * 128;
+        const uint32_t p_tmem = tmem + x * 128 + h * 64;
         const uint64_t bv = stage == 0 ? dv0 : dv1;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          mma_ts(d_tmem, p_tmem + ks * 8, bv + static_cast<uint64_t>((ks * 2048) >> 4), id_o,
-                 (j > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_ts(d_tmem, p_tmem + ks * 8, bv + static_cast<uint64_t>(((h * 4 + ks) * 2048) >> 4), id_o,
+                 (k > 0 || ks > 0) ? 1u : 0u);
         }
+        mma_commit(smem_u32(&bars->pv_done[x]));
       };
-      if (ok && nt > 0) {
+      const int T = (L + 63) / 64;  // 64-key sub-tiles; S slots alternate, so S(k+1) and S(k+2)
+                                    // are computed while the softmax of k runs
+      if (ok && T > 0) {
         ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma);
         if (ok) {
           fence_proxy_async_smem();  // the key rows were written by cp.async (generic proxy)
           tc_fence_after();
-          issue_s(0, 0);
-          mma_commit(smem_u32(&bars->s_full[0]));
-          if (has_b) {
-            issue_s(1, 0);
-            mma_commit(smem_u32(&bars->s_full[1]));
+          for (int k = 0; k < 2 && k < T; ++k) {
+            issue_s(0, k);
+            if (has_b) issue_s(1, k);
           }
           mma_commit(smem_u32(&bars->k_empty[0]));  // K(0) is not read again
         }
       }
-      for (int j = 0; j < nt && ok; ++j) {
-        const int stage = j & 1;
-        ok = mbar_wait(smem_u32(&bars->p_full[0]), j & 1, st, kWhereAttnMma);
-        if (ok) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma);
+      for (int k = 0; k < T && ok; ++k) {
+        const int h = k & 1, j = k >> 1, stage = j & 1;
+        ok = mbar_wait(smem_u32(&bars->p_full[0][h]), j & 1, st, kWhereAttnMma);
+        if (ok && h == 0) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma);
         if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_after();
-        issue_pv(0, stage, j);
-        const bool more = j + 1 < nt;
-        if (more) {
-          ok = mbar_wait(smem_u32(&bars->k_full[stage ^ 1]), ((j + 1) >> 1) & 1, st, kWhereAttnMma);
-          if (!ok) break;
-          fence_proxy_async_smem();
-          tc_fence_after();
-          issue_s(0, stage ^ 1);
-          mma_commit(smem_u32(&bars->s_full[0]));
+        issue_pv(0, k);
+        const int k2 = k + 2;
+        const int j2 = k2 >> 1, stage2 = j2 & 1;
+        if (k2 < T) {
+          if ((k2 & 1) == 0) {
+            ok = mbar_wait(smem_u32(&bars->k_full[stage2]), (j2 >> 1) & 1, st, kWhereAttnMma);
+            if (!ok) break;
+            fence_proxy_async_smem();
+            tc_fence_after();
+          }
+          issue_s(0, k2);
         }
         if (has_b) {
-          ok = mbar_wait(smem_u32(&bars->p_full[1]), j & 1, st, kWhereAttnMma);
+          ok = mbar_wait(smem_u32(&bars->p_full[1][h]), j & 1, st, kWhereAttnMma);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(1, stage, j);
+          issue_pv(1, k);
         }
-        mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
-        if (has_b && more) {
-          issue_s(1, stage ^ 1);
-          mma_commit(smem_u32(&bars->s_full[1]));
+        if (h == 1 || k == T - 1) mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
+        if (k2 < T) {
+          if (has_b) issue_s(1, k2);
+          if ((k2 & 1) == 1 || k2 == T - 1) mma_commit(smem_u32(&bars->k_empty[stage2]));  // nor K(j2)
         }
-        if (more) mma_commit(smem_u32(&bars->k_empty[stage ^ 1]));  // nor K(j+1) after its last S
       }
       if (ok) mma_commit(smem_u32(&bars->o_full));
       mma_commit(smem_u32(&bars->mma_done));
@@ -319,8 +332,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
       // K(j) may land as soon as the last S product of K(j-2) is done, V(j) once PV of V(j-2) is;
       // each lands asynchronously and counts itself on its full barrier
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->k_empty[stage]), ((j >> 1) - 1) & 1, st,
-                                                       kWhereAttnProducer)))
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->k_empty[stage]), ((j >> 1) - 1) & 1, st,
+                                                             kWhereAttnProducer)))
         break;
 #pragma unroll
       for (int it = 0; it < 32 / RPI; ++it) {
@@ -329,8 +342,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * D + my_chunk * 8);
       }
       cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->v_empty[stage]), ((j >> 1) - 1) & 1, st,
-                                                       kWhereAttnProducer)))
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->v_empty[stage]), ((j >> 1) - 1) & 1, st,
+                                                             kWhereAttnProducer)))
         break;
 #pragma unroll
       for (int it = 0; it < 32 / RPI; ++it) {
@@ -359,41 +372,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // runs under warp-uniform control flow; per-row decisions only select values.
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nt; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x]), j & 1, st, kWhereAttnSoftmax));
+      const int T = (L + 63) / 64;
+      for (int k = 0; k < T; ++k) {
+        const int h = k & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x][h]), (k >> 1) & 1, st, kWhereAttnSoftmax));
         if (!ok) break;
         tc_fence_after();
-        const int valid = min(128, L - j * 128);
-        uint32_t sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32p(t_s + c * 32, sv + c * 32);
+        const uint32_t t_sk = t_s + h * 64;
+        const int valid = min(64, L - k * 64);
+        uint32_t sv[64];
+        tmem_ld32p(t_sk, sv);
+        tmem_ld32p(t_sk + 32, sv + 32);
         tmem_wait_ld();
         float mx = -INFINITY;
-        if (valid == 128) {
+        if (valid == 64) {
           // four independent chains of three-input maxima
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int e = 0; e < 128; e += 8)
+          for (int e = 0; e < 64; e += 8)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               m4[c] = fmax3(m4[c], __uint_as_float(sv[e + 2 * c]), __uint_as_float(sv[e + 2 * c + 1]));
           mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         } else {
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
+          for (int e = 0; e < 64; ++e)
             if (e < valid) mx = fmaxf(mx, __uint_as_float(sv[e]));
         }
         const float m_new = fmaxf(m_used, mx * sl2);
         const bool grow = m_new > m_used + kRescaleThreshold;
         float f = 1.f;
         if (grow) {
-          if (j > 0) f = fast_exp2(m_used - m_new);
+          if (k > 0) f = fast_exp2(m_used - m_new);
           l *= f;
           m_used = m_new;
         }
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O holds every PV product up to tile j-1 (S_X(j) completing implies it); rows that keep
-          // their max multiply by 1.
+        if (k > 0 && __any_sync(0xffffffffu, grow)) {
+          // O must hold every PV product up to k-1 before it is rescaled; rows that keep their
+          // max multiply by 1.
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->pv_done[x]), (k - 1) & 1, st, kWhereAttnSoftmax));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -409,34 +428,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float2 scl = make_float2(sl2, sl2), negm = make_float2(-m_used, -m_used);
         float2 lsum4[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float2& lsum = lsum4[c];
-          lsum = make_float2(0.f, 0.f);
-          uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) lsum4[c] = make_float2(0.f, 0.f);
+        uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int col = c * 32 + 2 * e;
-            const float2 t = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), scl, negm);
-            float2 pe;
-            if (2 * e >= 32 - kEmuPerChunk) pe = exp2_poly2(t);
-            else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-            if (valid < 128) {
-              if (col >= valid) pe.x = 0.f;
-              if (col + 1 >= valid) pe.y = 0.f;
-            }
-            pk[e] = pack_bf16x2(pe.x, pe.y);
-            lsum = add2(lsum, pe);
+        for (int e = 0; e < 32; ++e) {
+          const int col = 2 * e;
+          const float2 t = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), scl, negm);
+          float2 pe;
+          if ((e & 15) >= 16 - kEmuPerChunk / 2) pe = exp2_poly2(t);
+          else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          if (valid < 64) {
+            if (col >= valid) pe.x = 0.f;
+            if (col + 1 >= valid) pe.y = 0.f;
           }
-          tmem_st16(t_s + c * 16, pk);
+          pk[e] = pack_bf16x2(pe.x, pe.y);
+          lsum4[e & 3] = add2(lsum4[e & 3], pe);
         }
+        tmem_st32(t_sk, pk);
         const float2 ls = add2(add2(lsum4[0], lsum4[1]), add2(lsum4[2], lsum4[3]));
         l += ls.x + ls.y;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x]));
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x][h]));
       }
-      if (ok && nt > 0)
+      if (ok && T > 0)
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0, st, kWhereAttnSoftmax));
       if (ok) {
         tc_fence_after();
@@ -447,11 +463,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (tk < 0 || tk >= N) tk = -1;  // an invalid permutation entry is skipped
         }
         uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<size_t>(bh) * N + (tk < 0 ? 0 : tk)) * D);
-        const float inv = (nt > 0 && l > 0.f) ? 1.f / l : 0.f;
+        const float inv = (T > 0 && l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          if (nt > 0) {
+          if (T > 0) {
             tmem_ld32(t_o + c * 32, v);
             tmem_wait_ld();
           } else {

@@ -92,6 +92,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceS
   }
 }
 
+// The same wait for threads that are not on the critical path: between polls the thread sleeps,
+// leaving the scheduler (and the shared-memory pipe the polls use) to the warps that are.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, DeviceStatus* st,
+                                                uint32_t where, uint32_t ns = 128,
+                                                long long budget = kWaitBudgetCycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  uint32_t spins = 0;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 15u) == 0) {
+      if (status_set(st)) return false;
+      if (clock64() - t0 > budget) {
+        raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
+        return false;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Fences
 // ------------------------------------------------------------------------------------------------
