@@ -705,17 +705,19 @@ __global__ void __launch_bounds__(128) assign_exact_kernel(const void* __restric
 // ------------------------------------------------------------------------------------------------
 // Tensor-core assignment (bf16 X, d = 128)
 // ------------------------------------------------------------------------------------------------
-// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM allocator, 3 = idle, 4..7 = epilogue
-// (warp w reads TMEM lanes 32*(w%4) .. +31, i.e. tokens 32*(w-4) .. +31 of the tile).
-constexpr int kAsgThreads = 256;
+// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM allocator, 3 = idle, 4..11 = epilogue in
+// two warpgroups that split every chunk's 128 columns (warpgroup h takes columns 64h .. 64h+63);
+// warp w reads TMEM lanes 32*(w%4) .. +31, i.e. tokens 32*(w%4) .. +31 of the tile.
+constexpr int kAsgThreads = 384;
 constexpr uint32_t kAsgXStage = 32768;   // 128 tokens x 128 d bf16 (two 16 KB halves)
 constexpr uint32_t kAsgCStage = 65536;   // 128 centroids x 128 d x {hi, lo}
 constexpr uint32_t kAsgSmem = 2 * kAsgXStage + 2 * kAsgCStage + 1024 /*align*/ + 256 /*barriers*/ +
-                               4 * 128 * 4 /*norms*/ + 128 * 33 * 4 /*scratch*/;
+                               128 * 9 * 4 /*half merge*/;
 constexpr uint32_t kAsgTmemCols = 512;   // 4 accumulators of 128 columns
 
 struct AsgBars {
   uint64_t x_full[2], x_empty[2], c_full[2], c_empty[2], acc_full[4], acc_empty[4], mma_done;
+  uint64_t merge_full[4], merge_empty[4];  // per warp quarter: warpgroup 1 -> warpgroup 0 handoff
   uint32_t tmem_base;
 };
 
@@ -765,7 +767,7 @@ __device__ __forceinline__ float tile_row_dist(const uint8_t* xt, int row, const
 }
 
 __device__ __forceinline__ float tile_row_norm(const uint8_t* xt, int row) {
-  float acc = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four chains: the sum is only used for the tolerance
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -775,11 +777,32 @@ __device__ __forceinline__ float tile_row_norm(const uint8_t* xt, int row) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float a = bf16lo_to_f32(w[e]), b = bf16hi_to_f32(w[e]);
-        acc = fmaf(a, a, acc);
-        acc = fmaf(b, b, acc);
+        acc[e] = fmaf(a, a, acc[e]);
+        acc[e] = fmaf(b, b, acc[e]);
       }
     }
-  return acc;
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Keep the 4 smallest (score, index) pairs: replace the worst entry if this one is better
+// (strictly: among equal scores the one seen first, i.e. the lower index, stays).
+__device__ __forceinline__ void cand_insert(float val, int j, float (&cv)[4], int (&ci)[4]) {
+  int wi = 0;
+  float wv = cv[0];
+#pragma unroll
+  for (int r = 1; r < 4; ++r)
+    if (cv[r] > wv) {
+      wv = cv[r];
+      wi = r;
+    }
+  if (val < wv) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      if (r == wi) {
+        cv[r] = val;
+        ci[r] = j;
+      }
+  }
 }
 
 __global__ void __launch_bounds__(kAsgThreads, 1)
@@ -807,7 +830,9 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(smem_u32(&bars->acc_full[i]), 1);
-      mbar_init(smem_u32(&bars->acc_empty[i]), 4);
+      mbar_init(smem_u32(&bars->acc_empty[i]), 8);
+      mbar_init(smem_u32(&bars->merge_full[i]), 1);
+      mbar_init(smem_u32(&bars->merge_empty[i]), 1);
     }
     mbar_init(smem_u32(&bars->mma_done), 1);
     fence_mbar_init();
@@ -902,24 +927,24 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: argmin over centroids ----------------
-    // Per 32-column group: scores s = ||c||^2 - 2 x.c (no branches), the group minimum, then a bit
-    // mask of the columns within tau of the running minimum; columns in the mask (rare: the
-    // minimum itself and near-ties) go through shared scratch into a 4-entry candidate list.
-    // tau = 2^-11 (||x||^2 + max(d_min, 0)) is >= 3x the bound on the split-bf16 score error
-    // 2^-15 (5 ||x||^2 + 2 d_min), so the true argmin is always among the candidates; when more
-    // than one candidate survives, exact float32 ||x - c||^2 decides (ties to the lower index).
+    // Per 32-column group: scores s = ||c||^2 - 2 x.c (packed pairs), the group minimum
+    // (three-input min, four chains), and only if that minimum is within tau of the running
+    // minimum, the columns within tau go into a 4-entry candidate list (the minimum itself and
+    // near-ties).  tau = 2^-11 (||x||^2 + max(d_min, 0)) is >= 3x the bound on the split-bf16 score
+    // error 2^-15 (5 ||x||^2 + 2 d_min), so the true argmin is always among the candidates.  The
+    // two warpgroups' lists are merged per token; when more than one candidate survives, exact
+    // float32 ||x - c||^2 decides (ties to the lower index).
     const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
     const int row = q * 32 + lane;
-    const int et = threadIdx.x - 128;  // 0..127
-    float* cn_s = reinterpret_cast<float*>(bars + 1);          // [4][128] staged norms
-    float* scr = cn_s + 4 * 128 + et * 33;                     // per-thread scratch, 32 scores
+    float* mrg = reinterpret_cast<float*>(bars + 1);  // [128][9]: warpgroup 1's minimum and list
     long long g = 0;
     int it = 0;
     bool ok = true;
     for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
       const int bh = static_cast<int>(w / ntiles), tile = static_cast<int>(w % ntiles);
       const int xsI = it & 1;
-      const float* cn = c_norm + static_cast<size_t>(bh) * kpad;
+      const float* cn = c_norm + static_cast<size_t>(bh) * kpad;  // 4 KB at most: stays in L1
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssignTail));
       if (!ok) break;
       const uint8_t* xt = xs + xsI * kAsgXStage;
@@ -929,53 +954,50 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
       int ci[4] = {-1, -1, -1, -1};
       for (int c = 0; c < nchunks; ++c, ++g) {
         const int a = static_cast<int>(g & 3);
-        cn_s[a * 128 + et] = __ldg(cn + c * kAssignChunkN + et);
-        asm volatile("bar.sync 2, 128;" ::: "memory");
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full[a]), (g >> 2) & 1, st, kWhereAssign));
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int qq = 0; qq < 4; ++qq) {
-          const int jb = c * kAssignChunkN + qq * 32;
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const int col0 = half * 64 + qq * 32;
+          const int jb = c * kAssignChunkN + col0;
           if (jb >= k) break;  // uniform
           uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kAssignChunkN + qq * 32, v);
+          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kAssignChunkN + col0, v);
           tmem_wait_ld();
-          const float* cnq = cn_s + a * 128 + qq * 32;
           float sc[32];
-          float mloc = INFINITY;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            sc[e] = fmaf(-2.f, __uint_as_float(v[e]), cnq[e]);
-            if (jb + 32 > k && jb + e >= k) sc[e] = INFINITY;
-            mloc = fminf(mloc, sc[e]);
+          for (int e = 0; e < 16; ++e) {
+            const float2 cn2 = __ldg(reinterpret_cast<const float2*>(cn + jb + 2 * e));
+            const float2 r2 = fma2(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
+                                   make_float2(-2.f, -2.f), cn2);
+            sc[2 * e] = r2.x;
+            sc[2 * e + 1] = r2.y;
           }
+          if (jb + 32 > k) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (jb + e >= k) sc[e] = INFINITY;
+          }
+          float m4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+#pragma unroll
+          for (int e = 0; e < 32; e += 8)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) m4[r] = fmin3(m4[r], sc[e + 2 * r], sc[e + 2 * r + 1]);
+          const float mloc = fmin3(m4[0], m4[1], fminf(m4[2], m4[3]));
           gmin = fminf(gmin, mloc);
           const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
-          unsigned hits = 0;
+          if (mloc <= thr) {  // rare after the first groups: the minimum lies elsewhere
+            unsigned hits = 0;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) hits |= (sc[e] <= thr ? 1u : 0u) << e;
-          if (hits) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) scr[e] = sc[e];
+            for (int e = 0; e < 32; ++e) hits |= (sc[e] <= thr ? 1u : 0u) << e;
             while (hits) {
               const int e = __ffs(hits) - 1;
               hits &= hits - 1;
-              const float val = scr[e];
-              // replace the worst candidate if this one is better (strictly: ties keep the earlier,
-              // i.e. lower, index)
-              int wi = 0;
+              float val = sc[0];
 #pragma unroll
-              for (int r = 1; r < 4; ++r)
-                if (cv[r] > cv[wi]) wi = r;
-              if (val < cv[wi]) {
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                  if (r == wi) {
-                    cv[r] = val;
-                    ci[r] = jb + e;
-                  }
-              }
+              for (int r = 1; r < 32; ++r) val = r == e ? sc[r] : val;
+              cand_insert(val, jb + e, cv, ci);
             }
           }
         }
@@ -984,39 +1006,68 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[a]));
       }
       if (!ok) break;
-      const int n = tile * kAssignTileM + row;
-      if (n < N) {
-        const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
-        int best = -1, nc = 0;
-        float bv = INFINITY;
+      // merge: warpgroup 1 hands its minimum and list to warpgroup 0 (per token)
+      float* mr = mrg + row * 9;
+      if (half == 1) {
+        if (it > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->merge_empty[q]), (it - 1) & 1, st, kWhereAssign));
+        if (!ok) break;
+        mr[0] = gmin;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          if (ci[r] >= 0 && cv[r] <= thr) {
-            ++nc;
-            if (cv[r] < bv || (cv[r] == bv && ci[r] < best)) {
-              bv = cv[r];
-              best = ci[r];
-            }
-          }
+          mr[1 + r] = cv[r];
+          mr[5 + r] = __int_as_float(ci[r]);
         }
-        if (nc > 1) {
-          const float* Cb = C + static_cast<size_t>(bh) * k * 128;
-          float bd = INFINITY;
-          best = -1;
-#pragma unroll 1
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->merge_full[q]));
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->merge_full[q]), it & 1, st, kWhereAssign));
+        if (!ok) break;
+        gmin = fminf(gmin, mr[0]);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int j = __float_as_int(mr[5 + r]);
+          if (j >= 0) cand_insert(mr[1 + r], j, cv, ci);  // higher indices than every own entry: ties keep own
+        }
+        const int n = tile * kAssignTileM + row;
+        if (n < N) {
+          const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
+          int best = -1, nc = 0;
+          float bv = INFINITY;
+#pragma unroll
           for (int r = 0; r < 4; ++r) {
-            if (ci[r] < 0 || cv[r] > thr) continue;
-            const float dd = tile_row_dist(xt, row, Cb + static_cast<size_t>(ci[r]) * 128);
-            if (dd < bd || (dd == bd && ci[r] < best)) {
-              bd = dd;
-              best = ci[r];
+            if (ci[r] >= 0 && cv[r] <= thr) {
+              ++nc;
+              if (cv[r] < bv || (cv[r] == bv && ci[r] < best)) {
+                bv = cv[r];
+                best = ci[r];
+              }
             }
           }
+          if (nc > 1) {
+            const float* Cb = C + static_cast<size_t>(bh) * k * 128;
+            float bd = INFINITY;
+            best = -1;
+#pragma unroll 1
+            for (int r = 0; r < 4; ++r) {
+              const float cvr = r == 0 ? cv[0] : r == 1 ? cv[1] : r == 2 ? cv[2] : cv[3];
+              const int cir = r == 0 ? ci[0] : r == 1 ? ci[1] : r == 2 ? ci[2] : ci[3];
+              if (cir < 0 || cvr > thr) continue;
+              const float dd = tile_row_dist(xt, row, Cb + static_cast<size_t>(cir) * 128);
+              if (dd < bd || (dd == bd && cir < best)) {
+                bd = dd;
+                best = cir;
+              }
+            }
+          }
+          labels[static_cast<size_t>(bh) * N + n] = best < 0 ? 0 : best;
         }
-        labels[static_cast<size_t>(bh) * N + n] = best < 0 ? 0 : best;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&bars->merge_empty[q]));  // mr may be overwritten
+          mbar_arrive(smem_u32(&bars->x_empty[xsI]));
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->x_empty[xsI]));
     }
   }
 
