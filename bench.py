@@ -72,10 +72,10 @@ def gen_inputs(cfg, step=0):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 243.4 MB + 70.2 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 239.3 MB + 68.6 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "e853a74c2f1e353f865310ab0cc119bbb5313c7e949f2c6ed77f7952024473f6",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 243.374080e6 + 70.152704e6,
+ATTN_TRAFFIC = {"sha256": "4380f672ad9ee1d203d7240f7d68218f247ab61a982c9c6a1c83a21a80f28e0b",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 239.277568e6 + 68.607232e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 
