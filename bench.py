@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the top-p sweep (selection + attention per p)")
     ap.add_argument("--heads", type=int, default=0, help="run only this many heads of the layer (profiling cases)")
     ap.add_argument("--no-warm", action="store_true", help="skip the warm-start denoising-sequence measurement")
     ap.add_argument("--warm-steps", type=int, default=10)
@@ -314,6 +315,31 @@ def main():
     attn_ms = stage_ms["sparse_attn"]
     achieved_tflops = actual_flops / (attn_ms * 1e-3) / 1e12
 
+    # the configuration's top-p sweep on the same clusters: selection + attention per p
+    sweep = None
+    if not args.no_sweep:
+        sweep = {}
+        kmeans_ms = stage_ms["kmeans_q"] + stage_ms["kmeans_k"]
+        for p in sorted(set(cfg.top_p) | {args.top_p}):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            svg2.svg2_select(cq, ck, cnt_k, p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
+            svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
+            torch.cuda.synchronize(dev)
+            ev[0].record(stream)
+            svg2.svg2_select(cq, ck, cnt_k, p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
+            ev[1].record(stream)
+            svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
+            ev[2].record(stream)
+            torch.cuda.synchronize(dev)
+            sl = stream_len.cpu().numpy().astype(np.float64)
+            flops = 4.0 * d * float((cq_h * sl).sum())
+            a_ms = ev[1].elapsed_time(ev[2])
+            sweep[str(p)] = {"density": flops / dense_flops, "select_ms": ev[0].elapsed_time(ev[1]),
+                             "attn_ms": a_ms, "attn_tflops_actual": flops / (a_ms * 1e-3) / 1e12,
+                             "attn_tflops_effective": dense_flops / (a_ms * 1e-3) / 1e12,
+                             "layer_ms": kmeans_ms + ev[0].elapsed_time(ev[1]) + stage_ms["permute"] + a_ms}
+        svg2.raise_on_device_error(ws)
+
     # k-means with k-means++ over all tokens (seed_tokens = 0), for comparison with the sampled seeding
     full_seed = None
     if args.seed_tokens != 0:
@@ -334,6 +360,7 @@ def main():
     dense_ms = None
     if not args.no_dense and rank == 0:
         dense_ms = time_dense(torch, Q, K, V, scale)
+
 
     warm = None
     if not args.no_warm:
@@ -367,6 +394,7 @@ def main():
         "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
         "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
         "dense_sdpa_ms": dense_ms, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
+        "top_p_sweep": sweep,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
