@@ -1,7 +1,9 @@
 // Critical-cluster identification ("Sparse VideoGen2" wiki summary, Key claims section 4.2,
 // Eq. 1-2; Method (3)): centroid-based scores weighted by K-cluster size, then top-p selection.
 //
-// One CTA of 1024 threads per (Q cluster, b,h); thread j owns K cluster j (nK <= 1024).
+// One CTA of 1024 threads per (group of kSelQ Q clusters, b,h); thread j owns K cluster j
+// (nK <= 1024) and computes its logits against the whole group, so each K centroid row is read
+// once per group (float4 loads streaming through L1) instead of once per Q cluster.
 //  * l_ij = (sum_m cq_im * ck_jm) * scale in float64, summed sequentially over m with no FMA
 //    (the oracle's order), w_ij = float32(count_j * exp(l_ij - max_j l_ij)) for non-empty j.
 //  * top-p in fixed point: u_j = floor(w_j / max w * 2^32) (correctly rounded float64 division),
@@ -16,6 +18,8 @@
 namespace svg2 {
 
 namespace {
+
+constexpr int kSelQ = 8;  // Q clusters per CTA
 
 __device__ double block_max_f64(double v, double* buf) {
 #pragma unroll
@@ -64,84 +68,110 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
                                                        uint8_t* __restrict__ mask, int32_t* __restrict__ sel_count,
                                                        int32_t* __restrict__ sel_idx,
                                                        int32_t* __restrict__ stream_len) {
-  __shared__ double cqs[128];
+  __shared__ double cqs[kSelQ][128];
   __shared__ double dbuf[32];
   __shared__ unsigned long long keys[1024];
   __shared__ unsigned long long ubuf[33];
-  const int i = blockIdx.x, bh = blockIdx.y, j = threadIdx.x;
-  const size_t row = static_cast<size_t>(bh) * nQ + i;
+  const int i0 = blockIdx.x * kSelQ, bh = blockIdx.y, j = threadIdx.x;
+  const int nq = min(kSelQ, nQ - i0);
   const bool valid = j < nK;
   const int cnt = valid ? count_k[static_cast<size_t>(bh) * nK + j] : 0;
 
-  float w = 0.f;
-  if (w_in != nullptr) {
-    if (valid) w = w_in[row * nK + j];
-  } else {
-    for (int m = j; m < d; m += blockDim.x) cqs[m] = static_cast<double>(cq[row * d + m]);
+  // logits of K cluster j against every Q cluster of the group: float64, summed over m in order
+  // with no FMA (the oracle's order)
+  double lg[kSelQ];
+#pragma unroll
+  for (int qq = 0; qq < kSelQ; ++qq) lg[qq] = -INFINITY;
+  if (w_in == nullptr) {
+    for (int e = j; e < nq * d; e += blockDim.x)
+      cqs[e / d][e % d] = static_cast<double>(cq[(static_cast<size_t>(bh) * nQ + i0) * d + e]);
     __syncthreads();
-    double l = -INFINITY;
     if (valid) {
-      const float* ckj = ck + (static_cast<size_t>(bh) * nK + j) * d;
-      double acc = 0.0;
-      for (int m = 0; m < d; ++m) acc = __dadd_rn(acc, __dmul_rn(cqs[m], static_cast<double>(__ldg(ckj + m))));
-      l = __dmul_rn(acc, static_cast<double>(scale));
+      const float4* ckj = reinterpret_cast<const float4*>(ck + (static_cast<size_t>(bh) * nK + j) * d);
+      double acc[kSelQ];
+#pragma unroll
+      for (int qq = 0; qq < kSelQ; ++qq) acc[qq] = 0.0;
+      for (int m4 = 0; m4 < d / 4; ++m4) {
+        const float4 c4 = __ldg(ckj + m4);
+        const double cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int qq = 0; qq < kSelQ; ++qq) acc[qq] = __dadd_rn(acc[qq], __dmul_rn(cqs[qq][4 * m4 + e], cv[e]));
+      }
+#pragma unroll
+      for (int qq = 0; qq < kSelQ; ++qq) lg[qq] = __dmul_rn(acc[qq], static_cast<double>(scale));
     }
-    const double mx = block_max_f64(cnt > 0 ? l : -INFINITY, dbuf);
-    if (cnt > 0) w = static_cast<float>(__dmul_rn(static_cast<double>(cnt), exp(__dsub_rn(l, mx))));
-    if (w_out != nullptr && valid) w_out[row * nK + j] = w;
   }
 
-  const double wmax = block_max_f64(cnt > 0 ? static_cast<double>(w) : 0.0, dbuf);
-  bool keep;
-  if (static_cast<double>(top_p) >= 1.0 || !(wmax > 0.0)) {
-    keep = cnt > 0;
-  } else {
-    unsigned long long u = 0ull;
-    if (cnt > 0 && w > 0.f) u = static_cast<unsigned long long>(floor(__ddiv_rn(static_cast<double>(w), wmax) * 4294967296.0));
-    const unsigned long long kMaxU = (1ull << 33) - 1ull;
-    keys[j] = valid ? (((kMaxU - u) << 11) | static_cast<unsigned long long>(j)) : ~0ull;
-    __syncthreads();
-    // bitonic sort, ascending, 1024 keys
-    for (int size = 2; size <= 1024; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        const int partner = j ^ stride;
-        if (partner > j) {
-          const unsigned long long a = keys[j], b = keys[partner];
-          const bool up = (j & size) == 0;
-          if ((a > b) == up) {
-            keys[j] = b;
-            keys[partner] = a;
-          }
-        }
-        __syncthreads();
-      }
+  for (int qq = 0; qq < nq; ++qq) {  // uniform
+    const size_t row = static_cast<size_t>(bh) * nQ + i0 + qq;
+    double l = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kSelQ; ++r)
+      if (r == qq) l = lg[r];
+    float w = 0.f;
+    if (w_in != nullptr) {
+      if (valid) w = w_in[row * nK + j];
+    } else {
+      const double mx = block_max_f64(cnt > 0 ? l : -INFINITY, dbuf);
+      if (cnt > 0) w = static_cast<float>(__dmul_rn(static_cast<double>(cnt), exp(__dsub_rn(l, mx))));
+      if (w_out != nullptr && valid) w_out[row * nK + j] = w;
     }
-    const unsigned long long kj = keys[j];
-    const bool kvalid = kj != ~0ull;
-    const unsigned long long uj = kvalid ? (kMaxU - (kj >> 11)) : 0ull;
-    unsigned long long U = 0ull;
-    const unsigned long long incl = block_inscan_u64(uj, ubuf, &U);
-    const unsigned long long T = static_cast<unsigned long long>(ceil(static_cast<double>(top_p) * static_cast<double>(U)));
-    const bool keep_sorted = kvalid && (incl - uj) < T;
-    __syncthreads();
-    // scatter the decision back to cluster order (reuse keys[] as a flag array)
-    keys[j] = 0ull;
-    __syncthreads();
-    if (keep_sorted) keys[static_cast<int>(kj & 2047ull)] = 1ull;
-    __syncthreads();
-    keep = valid && keys[j] != 0ull;
-    if (keep && cnt == 0) keep = false;
-  }
-  // compaction of kept indices in ascending j, count, and key-stream length
-  unsigned long long tot = 0ull;
-  const unsigned long long pos = block_inscan_u64(keep ? 1ull : 0ull, ubuf, &tot);
-  if (valid) mask[row * nK + j] = keep ? 1 : 0;
-  if (keep) sel_idx[row * nK + (pos - 1)] = j;
-  unsigned long long len_tot = 0ull;
-  block_inscan_u64(keep ? static_cast<unsigned long long>(cnt) : 0ull, ubuf, &len_tot);
-  if (j == 0) {
-    sel_count[row] = static_cast<int32_t>(tot);
-    if (stream_len != nullptr) stream_len[row] = static_cast<int32_t>(len_tot);
+
+    const double wmax = block_max_f64(cnt > 0 ? static_cast<double>(w) : 0.0, dbuf);
+    bool keep;
+    if (static_cast<double>(top_p) >= 1.0 || !(wmax > 0.0)) {
+      keep = cnt > 0;
+    } else {
+      unsigned long long u = 0ull;
+      if (cnt > 0 && w > 0.f) u = static_cast<unsigned long long>(floor(__ddiv_rn(static_cast<double>(w), wmax) * 4294967296.0));
+      const unsigned long long kMaxU = (1ull << 33) - 1ull;
+      __syncthreads();  // keys[] of the previous Q cluster is no longer read
+      keys[j] = valid ? (((kMaxU - u) << 11) | static_cast<unsigned long long>(j)) : ~0ull;
+      __syncthreads();
+      // bitonic sort, ascending, 1024 keys
+      for (int size = 2; size <= 1024; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const int partner = j ^ stride;
+          if (partner > j) {
+            const unsigned long long a = keys[j], b = keys[partner];
+            const bool up = (j & size) == 0;
+            if ((a > b) == up) {
+              keys[j] = b;
+              keys[partner] = a;
+            }
+          }
+          __syncthreads();
+        }
+      }
+      const unsigned long long kj = keys[j];
+      const bool kvalid = kj != ~0ull;
+      const unsigned long long uj = kvalid ? (kMaxU - (kj >> 11)) : 0ull;
+      unsigned long long U = 0ull;
+      const unsigned long long incl = block_inscan_u64(uj, ubuf, &U);
+      const unsigned long long T = static_cast<unsigned long long>(ceil(static_cast<double>(top_p) * static_cast<double>(U)));
+      const bool keep_sorted = kvalid && (incl - uj) < T;
+      __syncthreads();
+      // scatter the decision back to cluster order (reuse keys[] as a flag array)
+      keys[j] = 0ull;
+      __syncthreads();
+      if (keep_sorted) keys[static_cast<int>(kj & 2047ull)] = 1ull;
+      __syncthreads();
+      keep = valid && keys[j] != 0ull;
+      if (keep && cnt == 0) keep = false;
+    }
+    // compaction of kept indices in ascending j, count, and key-stream length
+    unsigned long long tot = 0ull;
+    const unsigned long long pos = block_inscan_u64(keep ? 1ull : 0ull, ubuf, &tot);
+    if (valid) mask[row * nK + j] = keep ? 1 : 0;
+    if (keep) sel_idx[row * nK + (pos - 1)] = j;
+    unsigned long long len_tot = 0ull;
+    block_inscan_u64(keep ? static_cast<unsigned long long>(cnt) : 0ull, ubuf, &len_tot);
+    if (j == 0) {
+      sel_count[row] = static_cast<int32_t>(tot);
+      if (stream_len != nullptr) stream_len[row] = static_cast<int32_t>(len_tot);
+    }
   }
 }
 
@@ -151,7 +181,7 @@ cudaError_t launch_select(const float* cq, const float* ck, const float* weights
                           int BH, int nQ, int nK, int d, float top_p, float scale, float* weights_out,
                           uint8_t* mask, int32_t* sel_count, int32_t* sel_idx, int32_t* stream_len,
                           cudaStream_t s) {
-  const dim3 grid(nQ, BH);
+  const dim3 grid((nQ + kSelQ - 1) / kSelQ, BH);
   select_kernel<<<grid, 1024, 0, s>>>(cq, ck, weights_in, count_k, nQ, nK, d, top_p, scale, weights_out, mask,
                                       sel_count, sel_idx, stream_len);
   return cudaGetLastError();
