@@ -384,21 +384,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32p(t_sk, sv);
         tmem_ld32p(t_sk + 32, sv + 32);
         tmem_wait_ld();
-        float mx = -INFINITY;
-        if (valid == 64) {
-          // four independent chains of three-input maxima
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int e = 0; e < 64; e += 8)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              m4[c] = fmax3(m4[c], __uint_as_float(sv[e + 2 * c]), __uint_as_float(sv[e + 2 * c + 1]));
-          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-        } else {
+        if (valid < 64) {  // the key stream's last sub-tile: columns past its end become -inf (p = 0)
 #pragma unroll
           for (int e = 0; e < 64; ++e)
-            if (e < valid) mx = fmaxf(mx, __uint_as_float(sv[e]));
+            if (e >= valid) sv[e] = __float_as_uint(-INFINITY);
         }
+        // four independent chains of three-input maxima
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < 64; e += 8)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            m4[c] = fmax3(m4[c], __uint_as_float(sv[e + 2 * c]), __uint_as_float(sv[e + 2 * c + 1]));
+        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         const float m_new = fmaxf(m_used, mx * sl2);
         const bool grow = m_new > m_used + kRescaleThreshold;
         float f = 1.f;
@@ -437,10 +435,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           float2 pe;
           if ((e & 15) >= 16 - kEmuPerChunk / 2) pe = exp2_poly2(t);
           else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-          if (valid < 64) {
-            if (col >= valid) pe.x = 0.f;
-            if (col + 1 >= valid) pe.y = 0.f;
-          }
           pk[e] = pack_bf16x2(pe.x, pe.y);
           lsum4[e & 3] = add2(lsum4[e & 3], pe);
         }
