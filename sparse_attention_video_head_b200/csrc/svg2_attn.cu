@@ -10,13 +10,15 @@
 //   warps 8-11  key/value producer: thread r gathers row r of each key tile with cp.async into
 //               the 128-byte-swizzled layout the tensor core reads (two stages)
 //   warp 12     Q tiles by TMA, then the single-thread MMA issuer
-//   warp 13     TMEM allocator (512 columns: S_A, S_B, O_A, O_B; P overwrites S as bf16)
-// Registers are re-split after set-up: the softmax warpgroups take 192 per thread, the others 64.
-// MMA order per key tile j: PV_A(j-1) -> S_A(j) -> PV_B(j-1) -> S_B(j).  Because tcgen05 ops of
-// one thread complete in order, "S_X(j) done" also means "O_X holds every PV up to j-1", so the
-// softmax warps rescale O_X in TMEM (only when the row max grows by more than 2^8) before
-// releasing P_X(j).  Softmax is exact: p = 2^(s*scale*log2e - m), O / l at the end, with l summed
-// over the bf16-rounded p that the PV product uses.
+//   warp 13     TMEM allocator (512 columns: S_A, S_B, O_A, O_B)
+// Registers are re-split after set-up: the softmax warpgroups take 192 per thread, the producer 40,
+// the MMA group 88.  S is computed in 64-key sub-tiles into a two-slot ring inside each Q tile's
+// 128 S columns, and P (bf16) overwrites the first 32 columns of its slot as the A operand of the
+// PV product, so per Q tile the chain is: softmax(k) -> PV(k) -> S(k+2) into the freed slot,
+// while the softmax of k+1 runs on the other slot.  MMA order per sub-tile k: PV_A(k), S_A(k+2),
+// PV_B(k), S_B(k+2).  The softmax rescales O in TMEM (only when the row max grows by more than
+// 2^8) after PV(k-1) has landed.  Softmax is exact: p = 2^(s*scale*log2e - m), O / l at the end,
+// with l summed over the float32 p whose bf16 rounding the PV product uses.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
