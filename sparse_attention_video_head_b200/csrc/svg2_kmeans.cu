@@ -966,13 +966,19 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
           tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kAssignChunkN + col0, v);
           tmem_wait_ld();
           float sc[32];
+          float4 cn4[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 cn2 = __ldg(reinterpret_cast<const float2*>(cn + jb + 2 * e));
-            const float2 r2 = fma2(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
-                                   make_float2(-2.f, -2.f), cn2);
-            sc[2 * e] = r2.x;
-            sc[2 * e + 1] = r2.y;
+          for (int e = 0; e < 8; ++e) cn4[e] = __ldg(reinterpret_cast<const float4*>(cn + jb) + e);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 r0 = fma2(make_float2(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1])),
+                                   make_float2(-2.f, -2.f), make_float2(cn4[e].x, cn4[e].y));
+            const float2 r1 = fma2(make_float2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])),
+                                   make_float2(-2.f, -2.f), make_float2(cn4[e].z, cn4[e].w));
+            sc[4 * e] = r0.x;
+            sc[4 * e + 1] = r0.y;
+            sc[4 * e + 2] = r1.x;
+            sc[4 * e + 3] = r1.y;
           }
           if (jb + 32 > k) {
 #pragma unroll
@@ -986,7 +992,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
             for (int r = 0; r < 4; ++r) m4[r] = fmin3(m4[r], sc[e + 2 * r], sc[e + 2 * r + 1]);
           const float mloc = fmin3(m4[0], m4[1], fminf(m4[2], m4[3]));
           gmin = fminf(gmin, mloc);
-          const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
+          const float thr = gmin + (xn + fmaxf(gmin + xn, 0.f)) * 0x1p-11f;
           if (mloc <= thr) {  // rare after the first groups: the minimum lies elsewhere
             unsigned hits = 0;
 #pragma unroll
@@ -1031,7 +1037,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         }
         const int n = tile * kAssignTileM + row;
         if (n < N) {
-          const float thr = gmin + ldexpf(xn + fmaxf(gmin + xn, 0.f), -11);
+          const float thr = gmin + (xn + fmaxf(gmin + xn, 0.f)) * 0x1p-11f;
           int best = -1, nc = 0;
           float bv = INFINITY;
 #pragma unroll
