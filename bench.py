@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--config", default="wan720p", choices=sorted(I.CONFIGS))
     ap.add_argument("--top-p", type=float, default=0.9)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-heads-per-group", type=int, default=8,
+                    help="heads per transfer group in the end-to-end call (copies overlap the other groups' compute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the top-p sweep (selection + attention per p)")
@@ -417,15 +419,13 @@ def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
     ck = torch.zeros(B, H, cfg.nK, d, device=dev)
     prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, args.top_p, float(np.float32(cfg.scale)), 1,
                            args.seed_tokens)
-
+    copy_stream = torch.cuda.Stream(device=dev)
+    # the uniforms are tiny; they go up on the compute stream before the layer call
     def one():
-        Q.copy_(hq, non_blocking=True)
-        K.copy_(hk, non_blocking=True)
-        V.copy_(hv, non_blocking=True)
         uq.copy_(huq, non_blocking=True)
         uk.copy_(huk, non_blocking=True)
-        svg2.svg2_layer(Q, K, V, prm, cq, ck, O, ws, uq, uk)
-        ho.copy_(O, non_blocking=True)
+        svg2.svg2_layer_host(hq, hk, hv, ho, Q, K, V, O, prm, cq, ck, ws, uq, uk,
+                             heads_per_group=args.e2e_heads_per_group, copy_stream=copy_stream)
 
     for _ in range(max(1, args.warmup)):
         one()
@@ -443,7 +443,7 @@ def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
     ms = max_over_ranks(a.elapsed_time(b) / steps, world, dist, dev)
     h2d = 3 * hq.numel() * 2 + (huq.numel() + huk.numel()) * 8
     return {"value": whole_job_ms_per_layer(ms, world), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
-            "steps": steps, "api": "svg2_layer"}
+            "steps": steps, "api": "svg2_layer_host", "heads_per_group": args.e2e_heads_per_group}
 
 
 def measure_warm(svg2, torch, cfg, args, dev, Q0, K0, V0, ws, scale):

@@ -205,6 +205,24 @@ SVG2_API int svg2_layer(const void* Q, const void* K, const void* V, int dtype, 
                const svg2_layer_outputs* outs, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * svg2_layer for inputs and output in host memory, with the transfers overlapped with the work:
+ * on `copy_stream` Q, then K, then V are copied to the caller's device staging buffers while, on
+ * `stream`, the k-means of Q starts as soon as Q has landed and that of K as soon as K has; the
+ * attention then runs in groups of `heads_per_group` (b,h) planes (0 = all at once) and each
+ * group's output is copied back while the next group is computed.  Host buffers must be
+ * page-locked (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.  The copies
+ * start only after the work already enqueued on `stream`; on return everything is enqueued and
+ * `stream` waits for the last copy, so synchronising `stream` covers the whole call.
+ * `copy_stream` may be NULL or equal to `stream` (no overlap).  Results equal svg2_layer's.
+ *   Qh, Kh, Vh   host [B,H,N,d] (dtype); Oh host bf16 [B,H,N,d], out.
+ *   Qd, Kd, Vd   device staging buffers [B,H,N,d] (dtype); Od device bf16 [B,H,N,d] (caller-owned).
+ *   uq, uk, cq, ck, params, ws as in svg2_layer (device memory). */
+SVG2_API int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, void* Qd, void* Kd,
+                             void* Vd, void* Od, int dtype, int B, int H, int N, int d, const svg2_params* params,
+                             const double* uq, const double* uk, float* cq, float* ck, int heads_per_group,
+                             void* ws, size_t ws_bytes, void* stream, void* copy_stream);
+
+/*
  * svg2_sparse_attn without a workspace, for callers that cannot allocate device memory at call
  * time (no cudaMalloc and no caching allocator available to them, e.g. code that must not grow
  * its memory footprint once running).  The paper has no counterpart; this is an interface

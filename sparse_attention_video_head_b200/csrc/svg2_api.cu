@@ -1,6 +1,7 @@
 // C-ABI entry points of libsvg2 (declared in include/svg2.h): argument validation, workspace
 // carving, tensor-map encoding and the launch sequence of each stage and of the whole layer.
 // Host code only; every step of the method runs in the kernels of the other .cu files.
+#include <vector>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -369,26 +370,34 @@ int svg2_unpermute(const void* Op, const int32_t* perm, int B, int H, int N, int
   }
 }
 
+// Checks shared by svg2_layer and svg2_layer_host (everything but the tensor pointers).
+static int check_layer_params(const svg2_params* p, int dtype, int B, int H, int N, int d, const double* uq,
+                              const double* uk, const float* cq, const float* ck) {
+  if (p == nullptr) return SVG2_ERR_INVALID_ARG;
+  int r = check_sizes(B, H, N, d);
+  if (r == SVG2_OK) r = check_k(p->nQ, N);
+  if (r == SVG2_OK) r = check_k(p->nK, N);
+  if (r != SVG2_OK) return r;
+  if (!valid_dtype(dtype) || p->iters < 1 || (p->init != SVG2_INIT_GIVEN && p->init != SVG2_INIT_KMEANSPP))
+    return SVG2_ERR_INVALID_ARG;
+  if (p->seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
+  if (p->init == SVG2_INIT_KMEANSPP) {
+    const int stride = kmeanspp_stride(N, p->seed_tokens);
+    if ((N + stride - 1) / stride < (p->nQ > p->nK ? p->nQ : p->nK)) return SVG2_ERR_INVALID_ARG;
+  }
+  if (!(p->top_p > 0.f) || p->scale != p->scale) return SVG2_ERR_INVALID_ARG;
+  if (cq == nullptr || ck == nullptr) return SVG2_ERR_INVALID_ARG;
+  if (p->init == SVG2_INIT_KMEANSPP && (uq == nullptr || uk == nullptr)) return SVG2_ERR_INVALID_ARG;
+  return SVG2_OK;
+}
+
 int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, int H, int N, int d,
                const svg2_params* p, const double* uq, const double* uk, float* cq, float* ck, void* O,
                const svg2_layer_outputs* outs, void* ws, size_t ws_bytes, void* stream) {
   try {
-    if (p == nullptr) return SVG2_ERR_INVALID_ARG;
-    int r = check_sizes(B, H, N, d);
-    if (r == SVG2_OK) r = check_k(p->nQ, N);
-    if (r == SVG2_OK) r = check_k(p->nK, N);
+    int r = check_layer_params(p, dtype, B, H, N, d, uq, uk, cq, ck);
     if (r != SVG2_OK) return r;
-    if (!valid_dtype(dtype) || p->iters < 1 || (p->init != SVG2_INIT_GIVEN && p->init != SVG2_INIT_KMEANSPP))
-      return SVG2_ERR_INVALID_ARG;
-    if (p->seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
-    if (p->init == SVG2_INIT_KMEANSPP) {
-      const int stride = kmeanspp_stride(N, p->seed_tokens);
-      if ((N + stride - 1) / stride < (p->nQ > p->nK ? p->nQ : p->nK)) return SVG2_ERR_INVALID_ARG;
-    }
-    if (!(p->top_p > 0.f) || p->scale != p->scale) return SVG2_ERR_INVALID_ARG;
-    if (Q == nullptr || K == nullptr || V == nullptr || cq == nullptr || ck == nullptr || O == nullptr)
-      return SVG2_ERR_INVALID_ARG;
-    if (p->init == SVG2_INIT_KMEANSPP && (uq == nullptr || uk == nullptr)) return SVG2_ERR_INVALID_ARG;
+    if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr) return SVG2_ERR_INVALID_ARG;
     if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(cq, 16) ||
         !aligned(ck, 16))
       return SVG2_ERR_INVALID_ARG;
@@ -420,6 +429,101 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
         if (e == cudaSuccess) e = launch_unpermute(L.Op, L.perm_q, BH, N, d, O, s);
       }
     }
+    return to_status(e);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, void* Qd, void* Kd, void* Vd, void* Od,
+                    int dtype, int B, int H, int N, int d, const svg2_params* p, const double* uq, const double* uk,
+                    float* cq, float* ck, int heads_per_group, void* ws, size_t ws_bytes, void* stream,
+                    void* copy_stream) {
+  try {
+    int r = check_layer_params(p, dtype, B, H, N, d, uq, uk, cq, ck);
+    if (r != SVG2_OK) return r;
+    if (Qh == nullptr || Kh == nullptr || Vh == nullptr || Oh == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (Qd == nullptr || Kd == nullptr || Vd == nullptr || Od == nullptr || heads_per_group < 0)
+      return SVG2_ERR_INVALID_ARG;
+    if (!aligned(Qd, 16) || !aligned(Kd, 16) || !aligned(Vd, 16) || !aligned(Od, 16) || !aligned(cq, 16) ||
+        !aligned(ck, 16))
+      return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    LayerCarve L;
+    carve_layer(c, BH, N, d, p->nQ, p->nK, nullptr, L);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    const int G = heads_per_group == 0 ? BH : (heads_per_group < BH ? heads_per_group : BH);
+    const int ngroups = (BH + G - 1) / G;
+    const bool f32 = dtype == SVG2_F32;
+    const size_t esz = f32 ? 4 : 2;
+    const size_t bytes_in = static_cast<size_t>(BH) * N * d * esz;
+    const size_t plane_out = static_cast<size_t>(N) * d * 2;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaStream_t cs = copy_stream != nullptr ? static_cast<cudaStream_t>(copy_stream) : s;
+
+    // events: entry (copies wait for prior work on `stream`), Q/K/V landed, each group's output
+    // ready, all copies done
+    std::vector<cudaEvent_t> ev(5 + ngroups, nullptr);
+    cudaError_t e = cudaSuccess;
+    for (auto& x : ev)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+    auto release = [&]() {
+      for (auto x : ev)
+        if (x) cudaEventDestroy(x);  // deferred by the runtime until the recorded work completes
+    };
+    if (e != cudaSuccess) {
+      release();
+      return SVG2_ERR_CUDA;
+    }
+    cudaEvent_t entry = ev[0], q_in = ev[1], k_in = ev[2], v_in = ev[3], all_out = ev[4];
+    auto ok = [&](cudaError_t x) {
+      if (e == cudaSuccess) e = x;
+      return e == cudaSuccess;
+    };
+    ok(cudaEventRecord(entry, s));
+    ok(cudaStreamWaitEvent(cs, entry, 0));
+    // inputs in the order the computation needs them: Q, then K while Q is clustered, then V
+    ok(cudaMemcpyAsync(Qd, Qh, bytes_in, cudaMemcpyHostToDevice, cs));
+    ok(cudaEventRecord(q_in, cs));
+    ok(cudaMemcpyAsync(Kd, Kh, bytes_in, cudaMemcpyHostToDevice, cs));
+    ok(cudaEventRecord(k_in, cs));
+    ok(cudaMemcpyAsync(Vd, Vh, bytes_in, cudaMemcpyHostToDevice, cs));
+    ok(cudaEventRecord(v_in, cs));
+    ok(cudaStreamWaitEvent(s, q_in, 0));
+    if (e == cudaSuccess)
+      e = run_kmeans(Qd, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q,
+                     L.perm_q, L.q_off, L.kq, L.st, s);
+    ok(cudaStreamWaitEvent(s, k_in, 0));
+    if (e == cudaSuccess)
+      e = run_kmeans(Kd, f32, BH, N, d, p->nK, p->iters, p->init, uk, p->seed_tokens, ck, L.labels_k, L.count_k,
+                     L.perm_k, L.k_off, L.kk, L.st, s);
+    if (e == cudaSuccess)
+      e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, nullptr, L.mask,
+                        L.sel_count, L.sel_idx, L.stream_len, s);
+    if (e == cudaSuccess) e = launch_gather(Qd, f32, L.perm_q, BH, N, d, L.Qp, s);
+    ok(cudaStreamWaitEvent(s, v_in, 0));
+    if (e == cudaSuccess) e = launch_gather2(Kd, Vd, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s);
+    // attention by head groups; each group's output goes back while the next group runs
+    const size_t plane_p = static_cast<size_t>(N) * d;  // elements of one permuted plane
+    for (int g = 0; g < ngroups && e == cudaSuccess; ++g) {
+      const size_t h0 = static_cast<size_t>(g) * G;
+      const int hn = (h0 + G <= static_cast<size_t>(BH)) ? G : BH - static_cast<int>(h0);
+      e = launch_sparse_attn(static_cast<const uint16_t*>(L.Qp) + h0 * plane_p,
+                             static_cast<const uint16_t*>(L.Kp) + h0 * plane_p,
+                             static_cast<const uint16_t*>(L.Vp) + h0 * plane_p, L.q_off + h0 * (p->nQ + 1),
+                             L.k_off + h0 * (p->nK + 1), L.sel_count + h0 * p->nQ,
+                             L.sel_idx + h0 * static_cast<size_t>(p->nQ) * p->nK, hn, N, d, p->nQ, p->nK, p->scale,
+                             L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st, s);
+      ok(cudaEventRecord(ev[5 + g], s));
+      ok(cudaStreamWaitEvent(cs, ev[5 + g], 0));
+      ok(cudaMemcpyAsync(static_cast<char*>(Oh) + h0 * plane_out, static_cast<const char*>(Od) + h0 * plane_out,
+                         hn * plane_out, cudaMemcpyDeviceToHost, cs));
+    }
+    ok(cudaEventRecord(all_out, cs));
+    ok(cudaStreamWaitEvent(s, all_out, 0));
+    release();
     return to_status(e);
   } catch (...) {
     return SVG2_ERR_CUDA;

@@ -23,7 +23,7 @@ DEFAULT_SEED_TOKENS = 16384  # SVG2_DEFAULT_SEED_TOKENS
 
 _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeanspp", "svg2_kmeans", "svg2_select",
             "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
-            "svg2_unpermute", "svg2_layer", "svg2_selftest_mma", "svg2_sparse_attn_noalloc")
+            "svg2_unpermute", "svg2_layer", "svg2_layer_host", "svg2_selftest_mma", "svg2_sparse_attn_noalloc")
 
 _lib = None
 
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.svg2_unpermute.argtypes = [P, P, I, I, I, I, P, P]
         L.svg2_layer.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(SvgParams), P, P, P, P, P,
                                  ctypes.POINTER(SvgLayerOutputs), P, S, P]
+        L.svg2_layer_host.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(SvgParams), P, P, P, P,
+                                      I, P, S, P, P]
         L.svg2_selftest_mma.argtypes = [P, P, I, P, P, P, P, S, P]
         L.svg2_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
         for name in _EXPORTS:
@@ -95,6 +97,13 @@ def _p(t: Optional[torch.Tensor]):
         raise ValueError("libsvg2 takes device tensors")
     if not t.is_contiguous():
         raise ValueError("libsvg2 takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _hp(t: torch.Tensor):
+    """Host pointer of a contiguous CPU tensor (argument marshalling only)."""
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous host tensor")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -264,6 +273,20 @@ def svg2_layer(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, params: LayerP
     _check(lib().svg2_layer(_p(Q), _p(K), _p(V), _dtype(Q), B, H, N, d, ctypes.byref(prm), _p(uq), _p(uk), _p(cq),
                             _p(ck), _p(O), ctypes.byref(c_outs) if c_outs is not None else None, _p(ws), ws.numel(),
                             _stream(stream)), "svg2_layer")
+
+
+def svg2_layer_host(Qh: torch.Tensor, Kh: torch.Tensor, Vh: torch.Tensor, Oh: torch.Tensor, Q: torch.Tensor,
+                    K: torch.Tensor, V: torch.Tensor, O: torch.Tensor, params: LayerParams, cq: torch.Tensor,
+                    ck: torch.Tensor, ws: torch.Tensor, uq: Optional[torch.Tensor] = None,
+                    uk: Optional[torch.Tensor] = None, heads_per_group: int = 0, stream=None, copy_stream=None):
+    """The layer with Q, K, V and O in (page-locked) host memory; Q, K, V, O here are the device
+    staging buffers.  Copies run on copy_stream, overlapped with the compute of other head groups."""
+    B, H, N, d = Qh.shape
+    prm = params.c()
+    cs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
+    _check(lib().svg2_layer_host(_hp(Qh), _hp(Kh), _hp(Vh), _hp(Oh), _p(Q), _p(K), _p(V), _p(O), _dtype(Qh), B, H, N, d,
+                                 ctypes.byref(prm), _p(uq), _p(uk), _p(cq), _p(ck), int(heads_per_group), _p(ws),
+                                 ws.numel(), _stream(stream), cs), "svg2_layer_host")
 
 
 def svg2_selftest_mma(A: torch.Tensor, Bm: torch.Tensor, V: torch.Tensor, ws: torch.Tensor, stream=None):

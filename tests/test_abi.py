@@ -111,6 +111,24 @@ def test_kmeanspp_rejects_bad_arguments(L):
     assert call(wsb=16) == WORKSPACE
 
 
+def test_layer_host_rejects_bad_arguments(L):
+    from sparse_attention_video_head_b200 import svg2
+    prm = svg2.SvgParams(4, 8, 2, 1, 0.9, 0.1, 0, 1)
+    def call(Qh=FAKE, Oh=FAKE, Qd=FAKE, B=1, H=2, N=100, d=128, hpg=1, p=ctypes.byref(prm), cq=FAKE, u=FAKE, ws=FAKE,
+             wsb=1 << 30):
+        return L.svg2_layer_host(Qh, FAKE, FAKE, Oh, Qd, FAKE, FAKE, FAKE, 0, B, H, N, d, p, u, u, cq, FAKE, hpg, ws,
+                                 wsb, None, None)
+    assert call(Qh=None) == INVALID
+    assert call(Oh=None) == INVALID
+    assert call(Qd=None) == INVALID
+    assert call(hpg=-1) == INVALID
+    assert call(p=None) == INVALID
+    assert call(cq=None) == INVALID
+    assert call(u=None) == INVALID          # k-means++ needs its uniforms
+    assert call(d=96) == UNSUPPORTED
+    assert call(wsb=16) == WORKSPACE        # checked for every head group before any copy
+
+
 def test_select_and_topp_reject_bad_arguments(L):
     F = ctypes.c_float
     assert L.svg2_select(FAKE, FAKE, FAKE, 1, 1, 4, 8, 128, F(0.0), F(0.1), None, FAKE, FAKE, FAKE, None, FAKE,

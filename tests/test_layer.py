@@ -156,3 +156,33 @@ def test_warm_start_sequence_tracks_cold_start(oracle):
         print(f"step {step}: rel-L2 vs dense warm {e_w:.4f} cold {e_c:.4f}")
         assert e_w <= 1.5 * e_c + 0.02
         cq, ck = torch.from_numpy(warm["cq"]).cuda(), torch.from_numpy(warm["ck"]).cuda()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("heads_per_group,separate_copy_stream", [(3, True), (0, True), (8, False)])
+def test_host_buffer_layer_matches_device_layer(heads_per_group, separate_copy_stream):
+    """svg2_layer_host (pinned host in/out, head groups, copies on their own stream) gives the same
+    bits as svg2_layer on device buffers: the heads are independent and every kernel is the same."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS["small"]
+    data = pool_layer_inputs(cfg, range(cfg.H))
+    ref = run_layer(svg2, cfg, data, 0.9)
+    B, H, N, d = data["q"].shape
+    pin = lambda x: torch.from_numpy(x).to(torch.bfloat16).pin_memory()
+    hq, hk, hv = pin(data["q"]), pin(data["k"]), pin(data["v"])
+    ho = torch.empty(B, H, N, d, dtype=torch.bfloat16).pin_memory()
+    Q, K, V = (torch.empty(B, H, N, d, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    O = torch.empty_like(Q)
+    cq = torch.zeros(B, H, cfg.nQ, d, device="cuda")
+    ck = torch.zeros(B, H, cfg.nK, d, device="cuda")
+    ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK)
+    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, 0.9, float(np.float32(cfg.scale)), 1,
+                           svg2.DEFAULT_SEED_TOKENS)
+    cs = torch.cuda.Stream() if separate_copy_stream else None
+    svg2.svg2_layer_host(hq, hk, hv, ho, Q, K, V, O, prm, cq, ck, ws, to_dev(data["uq"]), to_dev(data["uk"]),
+                         heads_per_group=heads_per_group, copy_stream=cs)
+    torch.cuda.current_stream().synchronize()
+    svg2.raise_on_device_error(ws)
+    assert torch.equal(ho.view(torch.int16), torch.from_numpy(ref["o"]).to(torch.bfloat16).view(torch.int16))
+    np.testing.assert_array_equal(host(cq), ref["cq"])
+    np.testing.assert_array_equal(host(ck), ref["ck"])
