@@ -75,10 +75,10 @@ def gen_inputs(cfg, step=0):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 239.3 MB + 68.6 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 240.4 MB + 69.6 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "4380f672ad9ee1d203d7240f7d68218f247ab61a982c9c6a1c83a21a80f28e0b",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 239.277568e6 + 68.607232e6,
+ATTN_TRAFFIC = {"sha256": "5417b3a76e68752364c031ffe180745c47cc2cd53d012c74c18184396a1c516b",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 240.430080e6 + 69.561600e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 
@@ -92,29 +92,42 @@ def attn_traffic(cfg):
 
 
 # ------------------------------------------------------------------------------------------ oracle
-def oracle_sample(cfg, top_p, rows=96, head=0, seed_tokens=0):
-    """The CPU oracle on a bounded sample of the layer: one head's k-means (Q and K), selection and
-    permutation in full, and attention for `rows` query rows; extrapolated to the whole layer."""
+def oracle_sample(cfg, top_p, rows=96, heads=(0,), seed_tokens=0):
+    """The CPU oracle on a bounded sample of the layer: for each head in `heads`, k-means (Q and K),
+    selection and permutation in full, and attention for `rows` query rows; extrapolated to the
+    whole layer (attention x N/rows, the mean head x H)."""
     from oracle import oracle as O
-    hi = I.head_inputs(cfg, 0, head)
     scale = float(np.float32(cfg.scale))
-    t0 = time.perf_counter()
-    cq, lq, count_q = O.kmeans(hi["q"], cfg.nQ, cfg.iters, hi["uq"], seed_tokens=seed_tokens)
-    t1 = time.perf_counter()
-    ck, lk, count_k = O.kmeans(hi["k"], cfg.nK, cfg.iters, hi["uk"], seed_tokens=seed_tokens)
-    t2 = time.perf_counter()
-    w = O.select_weights(cq.astype(np.float32), ck.astype(np.float32), count_k, scale)
-    mask = O.topp(w, count_k, top_p)
-    pq, qo = O.permute(lq, cfg.nQ)
-    pk, ko = O.permute(lk, cfg.nK)
-    Qp, Kp, Vp = O.gather_rows(hi["q"], pq), O.gather_rows(hi["k"], pk), O.gather_rows(hi["v"], pk)
-    t3 = time.perf_counter()
-    sel = np.random.default_rng(1).choice(cfg.N, rows, replace=False)
-    O.sparse_attention_rows(Qp, Kp, Vp, qo, ko, mask, scale, sel)
-    t4 = time.perf_counter()
-    per_head = (t1 - t0) + (t2 - t1) + (t3 - t2) + (t4 - t3) * cfg.N / rows
-    return per_head * cfg.H * 1e3, {"kmeans_q_s": t1 - t0, "kmeans_k_s": t2 - t1, "select_permute_s": t3 - t2,
-                                     "attn_rows_s": t4 - t3, "wall_s": t4 - t0}
+    parts = {"kmeans_q_s": 0.0, "kmeans_k_s": 0.0, "select_permute_s": 0.0, "attn_rows_s": 0.0}
+    per_head = []
+    w0 = time.perf_counter()
+    for head in heads:
+        hi = I.head_inputs(cfg, 0, head)
+        t0 = time.perf_counter()
+        cq, lq, count_q = O.kmeans(hi["q"], cfg.nQ, cfg.iters, hi["uq"], seed_tokens=seed_tokens)
+        t1 = time.perf_counter()
+        ck, lk, count_k = O.kmeans(hi["k"], cfg.nK, cfg.iters, hi["uk"], seed_tokens=seed_tokens)
+        t2 = time.perf_counter()
+        w = O.select_weights(cq.astype(np.float32), ck.astype(np.float32), count_k, scale)
+        mask = O.topp(w, count_k, top_p)
+        pq, qo = O.permute(lq, cfg.nQ)
+        pk, ko = O.permute(lk, cfg.nK)
+        Qp, Kp, Vp = O.gather_rows(hi["q"], pq), O.gather_rows(hi["k"], pk), O.gather_rows(hi["v"], pk)
+        t3 = time.perf_counter()
+        sel = np.random.default_rng(1 + head).choice(cfg.N, rows, replace=False)
+        O.sparse_attention_rows(Qp, Kp, Vp, qo, ko, mask, scale, sel)
+        t4 = time.perf_counter()
+        for key, dt in zip(parts, (t1 - t0, t2 - t1, t3 - t2, t4 - t3)):
+            parts[key] += dt
+        per_head.append((t3 - t0) + (t4 - t3) * cfg.N / rows)
+    parts["wall_s"] = time.perf_counter() - w0
+    return float(np.mean(per_head)) * cfg.H * 1e3, parts
+
+
+def sample_text(cfg, rows, heads):
+    return (f"{len(heads)} of {cfg.H} heads: full k-means++ + {cfg.iters} Lloyd iterations on Q and K, selection, "
+            f"permutation, and attention for {rows} of {cfg.N} query rows per head; extrapolated "
+            f"x{cfg.N}/{rows} rows, mean head x{cfg.H} heads")
 
 
 def run_reference(args, cfg):
@@ -126,8 +139,7 @@ def run_reference(args, cfg):
         v, _ = oracle_sample(cfg, args.top_p, seed_tokens=args.seed_tokens)
         vals.append(v)
     value = statistics.median(vals)
-    sample = (f"one head of {cfg.H}: full k-means++ + {cfg.iters} Lloyd iterations on Q and K, selection, "
-              f"permutation, and attention for 96 of {cfg.N} query rows; extrapolated x{cfg.N}/96 rows, x{cfg.H} heads")
+    sample = sample_text(cfg, 96, (0,))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "ms", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -374,10 +386,10 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        v, parts = oracle_sample(cfg, args.top_p, seed_tokens=args.seed_tokens)
+        heads = tuple(range(min(8, cfg.H)))
+        v, parts = oracle_sample(cfg, args.top_p, rows=256, heads=heads, seed_tokens=args.seed_tokens)
         cpu = {"value": v, "unit": "ms", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-               "sample": (f"one head of {cfg.H}: full k-means (Q and K), selection, permutation, attention for 96 "
-                          f"of {cfg.N} rows; extrapolated to the layer"), "parts_s": parts}
+               "sample": sample_text(cfg, 256, heads), "parts_s": parts}
     launches = kernel_launches(cfg)
     line = {
         "metric": METRIC, "value": whole_job_ms_per_layer(ms_per_step, world), "unit": "ms", "n_gpus": world, "steps": args.steps,
