@@ -15,7 +15,9 @@
 //     computes their exact float64 D^2 (a sequential sum over the 128 coordinates, the reference's
 //     order, one candidate per thread) and the exact value decides;
 //   * a tile is skipped without being fetched when no candidate in it can move closer: with a the
-//     candidate's nearest seed, ||c_new - c_a||^2 >= 4 D^2 proves ||x - c_new|| >= ||x - c_a||.
+//     candidate's nearest seed, ||c_new - c_a||^2 >= 4 D^2 proves ||x - c_new|| >= ||x - c_a||;
+//   * late in the seeding that test leaves few candidates; when a CTA has at most two rounds of its
+//     threads' worth, the pass skips the stream and computes their exact D^2 directly.
 //
 // Per-tile sums of the fixed-point weights make the sampling search a scan over the tiles, then a
 // scan over one tile.  The D^2 values, and so the seeds, are the same as those of the sequential
@@ -40,6 +42,9 @@ constexpr int kSdMaxTiles = 48;
 constexpr int kSdMaxPerCta = kSdMaxTiles * kSdTile;   // 6144 candidates per CTA
 constexpr int kSdMaxCluster = 16;
 constexpr int kSdMaxK = 1024;
+// A pass whose pruning test leaves at most this many candidates in a CTA skips the tensor-core
+// stream and computes their exact D^2 directly (four rounds of the 320 threads).
+constexpr int kSdDirect = 4 * kSdThreads;
 
 struct SdBars {
   uint64_t full[kSdStages];
@@ -98,6 +103,9 @@ __global__ void __launch_bounds__(kSdThreads, 1)
   __shared__ int tlist[kSdMaxTiles];
   __shared__ int n_active;
   __shared__ int n_exact;
+  __shared__ int direct_sh;
+  __shared__ unsigned tmask[kSdMaxTiles][4];  // per tile: which candidates pass the pruning test
+  __shared__ int toff[kSdMaxTiles];           // their offsets in the direct route's list
   __shared__ int err_sh;
   __shared__ float cc_sh;
   __shared__ unsigned long long cta_tot[kSdMaxCluster];
@@ -273,6 +281,7 @@ __global__ void __launch_bounds__(kSdThreads, 1)
       for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
       if (lane == 0) cc_sh = a;
     }
+
     for (int a0 = warp * 32; a0 < s; a0 += 32 * kSdWarps) {
       uint2 raw[32];
 #pragma unroll
@@ -308,31 +317,58 @@ __global__ void __launch_bounds__(kSdThreads, 1)
       for (int i = threadIdx.x; i < n; i += kSdThreads) xlist[i] = static_cast<uint16_t>(i);
     }
     for (int t = warp; t < ntiles; t += kSdWarps) {
-      bool any = false;
+      unsigned any = 0u;
       if (s > 0) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int c = t * kSdTile + 32 * j + lane;
-          if (c < n) any |= static_cast<double>(ss[As[c]]) < 4.0001 * Ds[c];
+          const unsigned m = __ballot_sync(0xffffffffu, c < n && static_cast<double>(ss[As[c]]) < 4.0001 * Ds[c]);
+          if (lane == 0) tmask[t][j] = m;
+          any |= m;
         }
       }
-      any = __any_sync(0xffffffffu, any);
       if (lane == 0) tflag[t] = any ? 1 : 0;
     }
-    if (threadIdx.x == 0) n_exact = s == 0 ? n : 0;
     __syncthreads();
     if (warp == 0) {
-      int cnt = 0;
+      int cnt = 0, tot = 0;  // active tiles; candidates passing the test, with each tile's offset
       for (int t0 = 0; t0 < ntiles; t0 += 32) {
-        const bool f = t0 + lane < ntiles && tflag[t0 + lane] != 0;
+        const int t = t0 + lane;
+        const bool f = t < ntiles && tflag[t] != 0;
         const unsigned m = __ballot_sync(0xffffffffu, f);
-        if (f) tlist[cnt + __popc(m & ((1u << lane) - 1u))] = t0 + lane;
+        if (f) tlist[cnt + __popc(m & ((1u << lane) - 1u))] = t;
         cnt += __popc(m);
+        const int c = f ? __popc(tmask[t][0]) + __popc(tmask[t][1]) + __popc(tmask[t][2]) + __popc(tmask[t][3]) : 0;
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (t < ntiles) toff[t] = tot + incl - c;
+        tot += __shfl_sync(0xffffffffu, incl, 31);
       }
-      if (lane == 0) n_active = err_sh ? 0 : cnt;
+      if (lane == 0) {
+        const bool direct = s == 0 || tot <= kSdDirect;  // pass 0: every candidate, listed above
+        n_active = (err_sh || direct) ? 0 : cnt;
+        n_exact = s == 0 ? n : (direct ? tot : 0);
+        direct_sh = s > 0 && direct;
+      }
     }
     __syncthreads();
     const int na = n_active;
+    if (direct_sh) {  // the direct route: list the candidates that pass the test, in tile order
+      for (int t = warp; t < ntiles; t += kSdWarps) {
+        if (!tflag[t]) continue;
+        int off = toff[t];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const unsigned m = tmask[t][j];
+          if ((m >> lane) & 1u) xlist[off + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(t * kSdTile + 32 * j + lane);
+          off += __popc(m);
+        }
+      }
+    }
 
     // ---- stream the active tiles: TMA -> MMA (x . c) -> screen + exact D^2
     if (warp == 0) {
@@ -387,7 +423,6 @@ __global__ void __launch_bounds__(kSdThreads, 1)
       bool ok = true;
       for (int i = eg; i < na && ok; i += 2) {
         const unsigned long long g = gbase + i;
-        const int slot = static_cast<int>(g % kSdStages);
         const int a = static_cast<int>(g % kSdAcc);
         const int t = tlist[i];
         ok = mbar_wait(smem_u32(&bars.acc_full[a]), static_cast<uint32_t>((g / kSdAcc) & 1), st, kWhereSeedEpilogue);
