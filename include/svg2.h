@@ -206,8 +206,9 @@ SVG2_API int svg2_layer(const void* Q, const void* K, const void* V, int dtype, 
 
 /*
  * svg2_layer for inputs and output in host memory, with the transfers overlapped with the work:
- * on `copy_stream` Q, then K, then V are copied to the caller's device staging buffers while, on
- * `stream`, the k-means of Q starts as soon as Q has landed and that of K as soon as K has; the
+ * on `copy_stream` K, then Q, then V are copied to the caller's device staging buffers while, on
+ * `stream`, the k-means of K starts as soon as K has landed and that of Q as soon as Q has (K's
+ * k-means, with more clusters, is the longer one and hides Q's upload); the
  * attention then runs in groups of `heads_per_group` (b,h) planes (0 = all at once) and each
  * group's output is copied back while the next group is computed.  Host buffers must be
  * page-locked (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.  The copies

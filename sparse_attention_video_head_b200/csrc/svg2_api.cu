@@ -104,7 +104,7 @@ cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int
     e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, s.c_hi, seed_tokens, st, stream);
   if (e == cudaSuccess) e = launch_centroid_prep(C, BH, k, d, s.c_hi, s.c_lo, s.c_norm, stream);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-    e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, st, stream);
+    e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, s.rr_list, s.rr_count, st, stream);
     if (e == cudaSuccess) e = launch_sort(labels, BH, N, k, perm, offsets, counts, s.chunk_hist, st, stream);
     if (e == cudaSuccess) e = launch_update(X, f32, BH, N, d, k, perm, offsets, C, s.c_hi, s.c_lo, s.c_norm, stream);
   }
@@ -484,21 +484,22 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     };
     ok(cudaEventRecord(entry, s));
     ok(cudaStreamWaitEvent(cs, entry, 0));
-    // inputs in the order the computation needs them: Q, then K while Q is clustered, then V
-    ok(cudaMemcpyAsync(Qd, Qh, bytes_in, cudaMemcpyHostToDevice, cs));
-    ok(cudaEventRecord(q_in, cs));
+    // inputs in the order the computation needs them: K first (its k-means, with more clusters than
+    // Q's, is the longer of the two and hides the upload of Q), then Q, then V
     ok(cudaMemcpyAsync(Kd, Kh, bytes_in, cudaMemcpyHostToDevice, cs));
     ok(cudaEventRecord(k_in, cs));
+    ok(cudaMemcpyAsync(Qd, Qh, bytes_in, cudaMemcpyHostToDevice, cs));
+    ok(cudaEventRecord(q_in, cs));
     ok(cudaMemcpyAsync(Vd, Vh, bytes_in, cudaMemcpyHostToDevice, cs));
     ok(cudaEventRecord(v_in, cs));
-    ok(cudaStreamWaitEvent(s, q_in, 0));
-    if (e == cudaSuccess)
-      e = run_kmeans(Qd, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q,
-                     L.perm_q, L.q_off, L.kq, L.st, s);
     ok(cudaStreamWaitEvent(s, k_in, 0));
     if (e == cudaSuccess)
       e = run_kmeans(Kd, f32, BH, N, d, p->nK, p->iters, p->init, uk, p->seed_tokens, ck, L.labels_k, L.count_k,
                      L.perm_k, L.k_off, L.kk, L.st, s);
+    ok(cudaStreamWaitEvent(s, q_in, 0));
+    if (e == cudaSuccess)
+      e = run_kmeans(Qd, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q,
+                     L.perm_q, L.q_off, L.kq, L.st, s);
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, nullptr, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);

@@ -69,6 +69,8 @@ struct KmeansScratch {
   int32_t* chunk_hist;// [BH, kSortChunks, k]
   int32_t* perm;      // [BH, N] (if the caller passes none)
   int32_t* offsets;   // [BH, k+1]
+  uint4* rr_list;     // [BH * N] tokens whose assignment the exact re-rank decides: {bh, n, c0|c1, c2|c3}
+  uint32_t* rr_count; // entries in rr_list
 };
 
 inline void carve_kmeans(Carve& c, int BH, int N, int d, int k, KmeansScratch& s, bool need_perm) {
@@ -81,6 +83,8 @@ inline void carve_kmeans(Carve& c, int BH, int N, int d, int k, KmeansScratch& s
   s.chunk_hist = c.take<int32_t>(static_cast<size_t>(BH) * kSortChunks * k);
   s.perm = need_perm ? c.take<int32_t>(static_cast<size_t>(BH) * N) : nullptr;
   s.offsets = c.take<int32_t>(static_cast<size_t>(BH) * (k + 1));
+  s.rr_list = c.take<uint4>(static_cast<size_t>(BH) * N);
+  s.rr_count = c.take<uint32_t>(1);
 }
 
 // Attention work plan: one unit = up to two 128-row Q tiles of one Q cluster.
@@ -129,7 +133,7 @@ cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, u
                                  float* c_norm, cudaStream_t s);
 cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,
                           const uint16_t* c_hi, const uint16_t* c_lo, const float* c_norm, int32_t* labels,
-                          DeviceStatus* st, cudaStream_t s);
+                          uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, cudaStream_t s);
 cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
                           const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
                           float* c_norm, cudaStream_t s);

@@ -721,51 +721,6 @@ struct AsgBars {
   uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void top3_insert(float s, int j, float& s1, int& i1, float& s2, int& i2, float& s3,
-                                            int& i3) {
-  if (s < s3) {
-    if (s < s2) {
-      s3 = s2;
-      i3 = i2;
-      if (s < s1) {
-        s2 = s1;
-        i2 = i1;
-        s1 = s;
-        i1 = j;
-      } else {
-        s2 = s;
-        i2 = j;
-      }
-    } else {
-      s3 = s;
-      i3 = j;
-    }
-  }
-}
-
-// Exact float32 distance between the token row held in the swizzled X tile and centroid row c.
-__device__ __forceinline__ float tile_row_dist(const uint8_t* xt, int row, const float* __restrict__ c) {
-  float acc = 0.f;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const uint4 v = *reinterpret_cast<const uint4*>(xt + h * 16384 + sw128_offset(row, ch));
-      const float4 c0 = __ldg(reinterpret_cast<const float4*>(c + h * 64 + ch * 8));
-      const float4 c1 = __ldg(reinterpret_cast<const float4*>(c + h * 64 + ch * 8 + 4));
-      float x[8] = {bf16lo_to_f32(v.x), bf16hi_to_f32(v.x), bf16lo_to_f32(v.y), bf16hi_to_f32(v.y),
-                    bf16lo_to_f32(v.z), bf16hi_to_f32(v.z), bf16lo_to_f32(v.w), bf16hi_to_f32(v.w)};
-      const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float df = x[e] - cc[e];
-        acc = fmaf(df, df, acc);
-      }
-    }
-  }
-  return acc;
-}
-
 __device__ __forceinline__ float tile_row_norm(const uint8_t* xt, int row) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four chains: the sum is only used for the tolerance
 #pragma unroll
@@ -808,8 +763,8 @@ __device__ __forceinline__ void cand_insert(float val, int j, float (&cv)[4], in
 __global__ void __launch_bounds__(kAsgThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, int BH, int N, int k, int kpad,
-                     const float* __restrict__ C, const float* __restrict__ c_norm, int32_t* __restrict__ labels,
-                     DeviceStatus* st) {
+                     const float* __restrict__ c_norm, int32_t* __restrict__ labels, uint4* __restrict__ rr_list,
+                     uint32_t* __restrict__ rr_count, uint32_t rr_cap, DeviceStatus* st) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;                       // 2 stages
@@ -932,8 +887,9 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     // minimum, the columns within tau go into a 4-entry candidate list (the minimum itself and
     // near-ties).  tau = 2^-11 (||x||^2 + max(d_min, 0)) is >= 3x the bound on the split-bf16 score
     // error 2^-15 (5 ||x||^2 + 2 d_min), so the true argmin is always among the candidates.  The
-    // two warpgroups' lists are merged per token; when more than one candidate survives, exact
-    // float32 ||x - c||^2 decides (ties to the lower index).
+    // two warpgroups' lists are merged per token; when more than one candidate survives, the token
+    // goes on a list and rerank_kernel, launched next, decides by exact float32 ||x - c||^2 (ties
+    // to the lower index), so that the epilogue never waits on centroid rows.
     const int q = warp & 3;
     const int half = (warp - 4) >> 2;
     const int row = q * 32 + lane;
@@ -1036,6 +992,8 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
           if (j >= 0) cand_insert(mr[1 + r], j, cv, ci);  // higher indices than every own entry: ties keep own
         }
         const int n = tile * kAssignTileM + row;
+        bool defer = false;
+        uint32_t c01 = 0xffffffffu, c23 = 0xffffffffu;  // the candidates, 16 bits each (0xffff: none)
         if (n < N) {
           const float thr = gmin + (xn + fmaxf(gmin + xn, 0.f)) * 0x1p-11f;
           int best = -1, nc = 0;
@@ -1043,6 +1001,10 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             if (ci[r] >= 0 && cv[r] <= thr) {
+              const uint32_t sh = 16u * static_cast<uint32_t>(nc & 1);
+              const uint32_t idx = static_cast<uint32_t>(ci[r]) << sh, keep = ~(0xffffu << sh);
+              if (nc < 2) c01 = (c01 & keep) | idx;
+              else c23 = (c23 & keep) | idx;
               ++nc;
               if (cv[r] < bv || (cv[r] == bv && ci[r] < best)) {
                 bv = cv[r];
@@ -1050,23 +1012,19 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
               }
             }
           }
-          if (nc > 1) {
-            const float* Cb = C + static_cast<size_t>(bh) * k * 128;
-            float bd = INFINITY;
-            best = -1;
-#pragma unroll 1
-            for (int r = 0; r < 4; ++r) {
-              const float cvr = r == 0 ? cv[0] : r == 1 ? cv[1] : r == 2 ? cv[2] : cv[3];
-              const int cir = r == 0 ? ci[0] : r == 1 ? ci[1] : r == 2 ? ci[2] : ci[3];
-              if (cir < 0 || cvr > thr) continue;
-              const float dd = tile_row_dist(xt, row, Cb + static_cast<size_t>(cir) * 128);
-              if (dd < bd || (dd == bd && cir < best)) {
-                bd = dd;
-                best = cir;
-              }
-            }
-          }
+          defer = nc > 1;  // near-tie: the exact distances decide, in rerank_kernel
           labels[static_cast<size_t>(bh) * N + n] = best < 0 ? 0 : best;
+        }
+        const unsigned dm = __ballot_sync(0xffffffffu, defer);
+        if (dm) {
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(rr_count, static_cast<uint32_t>(__popc(dm)));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const uint32_t slot = base + static_cast<uint32_t>(__popc(dm & ((1u << lane) - 1u)));
+          if (defer && slot < rr_cap)
+            rr_list[slot] = make_uint4(static_cast<uint32_t>(bh), static_cast<uint32_t>(n), c01, c23);
+          else if (defer)  // only past 2^32 - 1 listed tokens in one launch
+            raise_status(st, kStatusDeviceBounds, kWhereAssign, slot, static_cast<uint32_t>(n));
         }
         __syncwarp();
         if (lane == 0) {
@@ -1082,6 +1040,53 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, kAsgTmemCols);
+  }
+}
+
+// Near-ties of the tensor-core assignment: one warp per listed token computes the exact float32
+// ||x - c||^2 of each candidate (lane l holds coordinates 4l .. 4l+3; the partial sums are then
+// added across the warp in a fixed butterfly order) and keeps the smallest, ties to the lower index.
+constexpr int kRrThreads = 256;
+
+__global__ void __launch_bounds__(kRrThreads) rerank_kernel(const uint16_t* __restrict__ X, int N, int k,
+                                                            const float* __restrict__ C,
+                                                            const uint4* __restrict__ rr_list,
+                                                            const uint32_t* __restrict__ rr_count, uint32_t cap,
+                                                            int32_t* __restrict__ labels) {
+  const uint32_t total = min(*rr_count, cap);
+  const int lane = threadIdx.x & 31;
+  const uint32_t warps = gridDim.x * (kRrThreads / 32);
+  for (uint32_t i = blockIdx.x * (kRrThreads / 32) + (threadIdx.x >> 5); i < total; i += warps) {
+    const uint4 e = rr_list[i];
+    const size_t tok = static_cast<size_t>(e.x) * N + e.y;
+    const uint2 xr = *reinterpret_cast<const uint2*>(X + tok * 128 + 4 * lane);
+    const float x0 = bf16lo_to_f32(xr.x), x1 = bf16hi_to_f32(xr.x), x2 = bf16lo_to_f32(xr.y), x3 = bf16hi_to_f32(xr.y);
+    int cid[4];
+    float4 cv4[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {  // all four rows requested at once (an empty slot reads row 0)
+      const uint32_t w = r < 2 ? e.z : e.w;
+      const int c = static_cast<int>((w >> (16 * (r & 1))) & 0xffffu);
+      cid[r] = c < k ? c : -1;
+      cv4[r] = __ldg(reinterpret_cast<const float4*>(C + (static_cast<size_t>(e.x) * k + (c < k ? c : 0)) * 128) + lane);
+    }
+    int best = -1;
+    float bd = INFINITY;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int c = cid[r];
+      if (c < 0) continue;  // uniform across the warp
+      const float4 cv = cv4[r];
+      const float d0 = x0 - cv.x, d1 = x1 - cv.y, d2 = x2 - cv.z, d3 = x3 - cv.w;
+      float part = fmaf(d3, d3, fmaf(d2, d2, fmaf(d1, d1, d0 * d0)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (part < bd || (part == bd && c < best)) {
+        bd = part;
+        best = c;
+      }
+    }
+    if (lane == 0 && best >= 0) labels[tok] = best;
   }
 }
 
@@ -1140,11 +1145,21 @@ __global__ void __launch_bounds__(kUpdThreads) update_kernel(const void* __restr
     if (tid < D) {
       const int nr = min(kUpdRows, cnt - b * kUpdRows);
       const uint8_t* src = buf[b & 1];
-      for (int r = 0; r < nr; ++r) {
-        float x;
-        if constexpr (F32) x = reinterpret_cast<const float*>(src + r * ROWB)[tid];
-        else x = bf16lo_to_f32(reinterpret_cast<const uint16_t*>(src + r * ROWB)[tid]);
-        acc = __dadd_rn(acc, static_cast<double>(x));
+      if (nr == kUpdRows) {  // a full batch: every load is issued ahead of the additions
+#pragma unroll
+        for (int r = 0; r < kUpdRows; ++r) {
+          float x;
+          if constexpr (F32) x = reinterpret_cast<const float*>(src + r * ROWB)[tid];
+          else x = bf16lo_to_f32(reinterpret_cast<const uint16_t*>(src + r * ROWB)[tid]);
+          acc = __dadd_rn(acc, static_cast<double>(x));
+        }
+      } else {
+        for (int r = 0; r < nr; ++r) {
+          float x;
+          if constexpr (F32) x = reinterpret_cast<const float*>(src + r * ROWB)[tid];
+          else x = bf16lo_to_f32(reinterpret_cast<const uint16_t*>(src + r * ROWB)[tid]);
+          acc = __dadd_rn(acc, static_cast<double>(x));
+        }
       }
     }
     __syncthreads();
@@ -1272,7 +1287,7 @@ cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, u
 
 cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,
                           const uint16_t* c_hi, const uint16_t* c_lo, const float* c_norm, int32_t* labels,
-                          DeviceStatus* st, cudaStream_t s) {
+                          uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, cudaStream_t s) {
   if (!x_f32 && d == 128) {
     alignas(64) CUtensorMap tx, th, tl;
     const int kp = kpad_of(k);
@@ -1282,9 +1297,19 @@ cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAsgSmem);
     if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(rr_count, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return e;
     const long long tiles = static_cast<long long>(BH) * ((N + kAssignTileM - 1) / kAssignTileM);
-    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-    assign_tc_kernel<<<grid, kAsgThreads, kAsgSmem, s>>>(tx, th, tl, BH, N, k, kp, centroids, c_norm, labels, st);
+    const int sms = num_sms();
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    const size_t bhn = static_cast<size_t>(BH) * N;  // rr_list holds one entry per token
+    const uint32_t cap = bhn < 0xffffffffu ? static_cast<uint32_t>(bhn) : 0xffffffffu;
+    assign_tc_kernel<<<grid, kAsgThreads, kAsgSmem, s>>>(tx, th, tl, BH, N, k, kp, c_norm, labels, rr_list, rr_count,
+                                                          cap, st);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    rerank_kernel<<<2 * sms, kRrThreads, 0, s>>>(static_cast<const uint16_t*>(X), N, k, centroids, rr_list, rr_count,
+                                                 cap, labels);
     return cudaGetLastError();
   }
   const dim3 grid((N + 127) / 128, BH);
