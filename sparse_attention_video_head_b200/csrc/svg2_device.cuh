@@ -92,6 +92,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceS
   }
 }
 
+// The bounded wait with acquire semantics at cluster scope, for phases that other CTAs of the
+// cluster complete (st_async_u64 below).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, DeviceStatus* st, uint32_t where,
+                                                  long long budget = kWaitBudgetCycles) {
+  auto poll = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (poll()) return true;
+  const long long t0 = clock64();
+  uint32_t spins = 0;
+  while (true) {
+    if (poll()) return true;
+    if ((++spins & 63u) == 0u) {
+      if (status_set(st)) return false;
+      if (clock64() - t0 > budget) {
+        raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
+        return false;
+      }
+    }
+  }
+}
+
 // The same wait for threads that are not on the critical path: between polls the thread sleeps,
 // leaving the scheduler (and the shared-memory pipe the polls use) to the warps that are.
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, DeviceStatus* st,
@@ -118,6 +148,17 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, D
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Orders this thread's generic-proxy global writes before later async-proxy (bulk copy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global
+// memory into this CTA's shared memory; completion is counted in bytes on the mbarrier `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -373,6 +414,15 @@ __device__ __forceinline__ void st_cluster_u64(void* local, uint32_t rank, unsig
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(remote), "l"(v) : "memory");
+}
+// Writes v into CTA `rank`'s copy of the shared variable `local` and counts its 8 bytes as
+// completed transactions on that CTA's copy of the mbarrier `bar` (which expects them).
+__device__ __forceinline__ void st_async_u64(void* local, uint64_t* bar, uint32_t rank, unsigned long long v) {
+  uint32_t ra, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_u32(bar)), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u64 [%0], %1, [%2];" ::"r"(ra), "l"(v), "r"(rb)
+               : "memory");
 }
 __device__ __forceinline__ void st_cluster_f64(void* local, uint32_t rank, double v) {
   st_cluster_u64(local, rank, static_cast<unsigned long long>(__double_as_longlong(v)));

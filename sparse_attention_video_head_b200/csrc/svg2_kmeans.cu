@@ -720,6 +720,7 @@ struct AsgBars {
   uint64_t merge_full[4], merge_empty[4];  // per warp quarter: warpgroup 1 -> warpgroup 0 handoff
   uint32_t tmem_base;
 };
+static_assert(sizeof(AsgBars) <= 256, "barrier block");
 
 __device__ __forceinline__ float tile_row_norm(const uint8_t* xt, int row) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four chains: the sum is only used for the tolerance
@@ -953,6 +954,10 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
             unsigned hits = 0;
 #pragma unroll
             for (int e = 0; e < 32; ++e) hits |= (sc[e] <= thr ? 1u : 0u) << e;
+            if (__popc(hits) == 1) {  // the usual case: the group's minimum is its only entry within tau
+              cand_insert(mloc, jb + __ffs(hits) - 1, cv, ci);
+              hits = 0u;
+            }
             while (hits) {
               const int e = __ffs(hits) - 1;
               hits &= hits - 1;

@@ -45,6 +45,7 @@ constexpr int kSdMaxK = 1024;
 // A pass whose pruning test leaves at most this many candidates in a CTA skips the tensor-core
 // stream and computes their exact D^2 directly (four rounds of the 320 threads).
 constexpr int kSdDirect = 4 * kSdThreads;
+constexpr int kSdRingRows = kSdStages * kSdStageBytes / 256;  // bf16 seed rows the ring holds: 384
 
 struct SdBars {
   uint64_t full[kSdStages];
@@ -52,6 +53,8 @@ struct SdBars {
   uint64_t acc_full[kSdAcc];
   uint64_t acc_empty[kSdAcc];
   uint64_t mma_done;
+  uint64_t rows;  // the earlier seeds' bf16 rows copied into the (idle) ring for the pruning table
+  uint64_t pick;  // the pass's pick, sent by the CTA that owns it to every CTA of the cluster
   uint32_t tmem_base;
 };
 
@@ -86,6 +89,12 @@ __device__ __forceinline__ void sd_bcast(unsigned long long* var, unsigned long 
   }
 }
 
+// The pick goes to every CTA of the cluster with its arrival on their `pick` barrier, so that no
+// cluster-wide barrier is needed: each CTA waits for the one message of the pass.
+__device__ __forceinline__ void sd_send_pick(unsigned long long* var, uint64_t* bar, unsigned long long v, int ncl) {
+  for (int r = 0; r < ncl; ++r) st_async_u64(var, bar, static_cast<uint32_t>(r), v);
+}
+
 __global__ void __launch_bounds__(kSdThreads, 1)
     seed_tc_kernel(const __grid_constant__ CUtensorMap tm, const uint16_t* __restrict__ X, int N, int stride, int S,
                    int k, const double* __restrict__ u, float* __restrict__ C, uint16_t* __restrict__ Sb,
@@ -108,7 +117,7 @@ __global__ void __launch_bounds__(kSdThreads, 1)
   __shared__ int toff[kSdMaxTiles];           // their offsets in the direct route's list
   __shared__ int err_sh;
   __shared__ float cc_sh;
-  __shared__ unsigned long long cta_tot[kSdMaxCluster];
+  __shared__ unsigned long long cta_tot[2][kSdMaxCluster];  // by pass parity: a CTA may run a pass ahead
   __shared__ unsigned long long cta_max[kSdMaxCluster];
   __shared__ unsigned long long pick_bcast;
   __shared__ unsigned long long wred[kSdWarps];
@@ -140,6 +149,8 @@ __global__ void __launch_bounds__(kSdThreads, 1)
       mbar_init(smem_u32(&bars.acc_empty[i]), 4);
     }
     mbar_init(smem_u32(&bars.mma_done), 1);
+    mbar_init(smem_u32(&bars.rows), 1);
+    mbar_init(smem_u32(&bars.pick), 1);
     fence_mbar_init();
     err_sh = 0;
   }
@@ -177,6 +188,7 @@ __global__ void __launch_bounds__(kSdThreads, 1)
         Ch[static_cast<size_t>(s) * 128 + i] = a;
         Ch[static_cast<size_t>(s) * 128 + i + 1] = b;
         *reinterpret_cast<uint32_t*>(Sbh + static_cast<size_t>(s) * 128 + i) = w;
+        fence_proxy_async_global();  // every CTA's later bulk copy of the seed rows reads this one
       }
     }
     fence_proxy_async_smem();  // the tensor core reads seedB through the async proxy
@@ -192,23 +204,34 @@ __global__ void __launch_bounds__(kSdThreads, 1)
   for (int s = 0; s < k; ++s) {
     if (s > 0) {
       // ---- D^2 sampling: CTA total, cluster totals, then the owning CTA scans tiles and one tile
+      if (threadIdx.x == 0) mbar_arrive_expect_tx(smem_u32(&bars.pick), 8u);  // this pass's message
       if (warp == 0) {
         unsigned long long t = 0;
         for (int i = lane; i < ntiles; i += 32) t += gtot[i];
         t = warp_sum_u64(t);
-        if (lane == 0) sd_bcast(&cta_tot[rank], t, CL);
+        if (lane == 0) sd_bcast(&cta_tot[s & 1][rank], t, CL);
       }
       sd_sync(CL);
+      // the seed rows 0 .. s-1 (the last one written in the previous pass, before the barrier) go
+      // into the ring now, so that the copy overlaps the pick; the ring is idle until the stream
+      if (threadIdx.x == 0 && s < k - 1) {  // (the last seed's pass ends before the table)
+        const int nrow = min(s, kSdRingRows);
+        const uint32_t bar = smem_u32(&bars.rows);
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nrow) * 256u);
+        for (int r0 = 0; r0 < nrow; r0 += kSdTile)
+          bulk_load(smem_u32(ring + r0 * 256), Sbh + static_cast<size_t>(r0) * 128,
+                    static_cast<uint32_t>(min(kSdTile, nrow - r0)) * 256u, bar);
+      }
       unsigned long long U = 0, base = 0;
       for (int r = 0; r < CL; ++r) {
-        if (r < static_cast<int>(rank)) base += cta_tot[r];
-        U += cta_tot[r];
+        if (r < static_cast<int>(rank)) base += cta_tot[s & 1][r];
+        U += cta_tot[s & 1][r];
       }
-      const unsigned long long mine = cta_tot[rank];
+      const unsigned long long mine = cta_tot[s & 1][rank];
       if (U == 0ull) {
         if (threadIdx.x == 0 && rank == 0) {
           const long long p = static_cast<long long>(floor(uh[s] * static_cast<double>(S)));
-          sd_bcast(&pick_bcast, static_cast<unsigned long long>(p >= S ? S - 1 : p), CL);
+          sd_send_pick(&pick_bcast, &bars.pick, static_cast<unsigned long long>(p >= S ? S - 1 : p), CL);
         }
       } else if (warp == 0) {
         unsigned long long target = static_cast<unsigned long long>(floor(uh[s] * static_cast<double>(U)));
@@ -260,11 +283,12 @@ __global__ void __launch_bounds__(kSdThreads, 1)
                 break;
               }
             }
-            sd_bcast(&pick_bcast, static_cast<unsigned long long>(lo + pk), CL);
+            sd_send_pick(&pick_bcast, &bars.pick, static_cast<unsigned long long>(lo + pk), CL);
           }
         }
       }
-      sd_sync(CL);
+      if (!mbar_wait_cluster(smem_u32(&bars.pick), static_cast<uint32_t>((s - 1) & 1), st, kWhereSeedEpilogue))
+        err_sh = 1;
       pick = static_cast<int>(min(pick_bcast, static_cast<unsigned long long>(S - 1)));
     }
     load_seed(pick, s);
@@ -282,52 +306,99 @@ __global__ void __launch_bounds__(kSdThreads, 1)
       if (lane == 0) cc_sh = a;
     }
 
-    for (int a0 = warp * 32; a0 < s; a0 += 32 * kSdWarps) {
-      uint2 raw[32];
+    const int nrow = min(s, kSdRingRows);  // rows 0 .. nrow-1 are in the ring
+    bool rows_ok = true;
+    if (s > 0 && warp * 8 < s)
+      rows_ok = mbar_wait(smem_u32(&bars.rows), static_cast<uint32_t>((s - 1) & 1), st, kWhereSeedEpilogue);
+    if (s > 0 && rows_ok) {
+      // a warp takes 8 seed rows per round: lane (rr, qd) = (lane / 4, lane % 4) sums the quarter
+      // qq of the coordinates of row rr, visiting its four 16-byte chunks from a lane-dependent
+      // start (rho) so that the ring reads spread over all banks; the new seed's coordinates of
+      // that quarter, in the same visiting order, stay in registers
+      const int rr = lane >> 2, qd = lane & 3, rho = rr & 3;
+      const int qq = (qd + rr) & 3;
+      float cq[32];
 #pragma unroll
-      for (int r = 0; r < 32; ++r)
-        if (a0 + r < s) raw[r] = *reinterpret_cast<const uint2*>(Sbh + static_cast<size_t>(a0 + r) * 128 + 4 * lane);
-      const float c0 = cs[4 * lane], c1 = cs[4 * lane + 1], c2 = cs[4 * lane + 2], c3 = cs[4 * lane + 3];
-      float pr[32];
+      for (int i = 0; i < 4; ++i) {
+        const int ch = (i + rho) & 3;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        pr[r] = 0.f;
-        if (a0 + r < s) {
-          const float d0 = bf16lo_to_f32(raw[r].x) - c0, d1 = bf16hi_to_f32(raw[r].x) - c1;
-          const float d2 = bf16lo_to_f32(raw[r].y) - c2, d3 = bf16hi_to_f32(raw[r].y) - c3;
-          pr[r] = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
-        }
+        for (int e = 0; e < 8; ++e) cq[8 * i + e] = cs[32 * qq + 8 * ch + e];
       }
+      for (int a0 = warp * 8; a0 < s; a0 += 8 * kSdWarps) {
+        const int a = a0 + rr;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (a < s) {
+          uint4 v[4];
 #pragma unroll
-      for (int o = 16, m = 16; o > 0; o >>= 1, m >>= 1) {
-        const bool upper = (lane & o) != 0;
+          for (int i = 0; i < 4; ++i) {
+            const int off = qq * 64 + ((i + rho) & 3) * 16;  // bytes within the row
+            v[i] = a < nrow ? *reinterpret_cast<const uint4*>(ring + a * 256 + off)
+                            : *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(Sbh) +
+                                                              static_cast<size_t>(a) * 256 + off);
+          }
 #pragma unroll
-        for (int q = 0; q < m; ++q) {
-          const float keep = upper ? pr[q + m] : pr[q];
-          const float send = upper ? pr[q] : pr[q + m];
-          pr[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float d0 = bf16lo_to_f32(w[e]) - cq[8 * i + 2 * e];
+              const float d1 = bf16hi_to_f32(w[e]) - cq[8 * i + 2 * e + 1];
+              acc[e] = fmaf(d0, d0, acc[e]);
+              acc[e] = fmaf(d1, d1, acc[e]);
+            }
+          }
         }
+        float t = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        if (qd == 0 && a < s) ss[a] = t;
       }
-      if (a0 + lane < s) ss[a0 + lane] = pr[0];
     }
+    if (!rows_ok) err_sh = 1;  // (the pruning table is incomplete: the pass streams nothing)
+    fence_proxy_async_smem();  // these generic reads of the ring come before the stream's TMA writes
     __syncthreads();
 
     // ---- tiles that may hold a candidate moving closer (all of them for the first seed)
     if (s == 0) {
       for (int i = threadIdx.x; i < n; i += kSdThreads) xlist[i] = static_cast<uint16_t>(i);
     }
-    for (int t = warp; t < ntiles; t += kSdWarps) {
-      unsigned any = 0u;
+    for (int t0 = warp; t0 < ntiles; t0 += 2 * kSdWarps) {
+      // two tiles (t0, t0 + kSdWarps) per round, every load issued before the tests
+      bool p[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) p[h][j] = false;
       if (s > 0) {
+        int ai[2][4];
+        double dv[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = (t0 + h * kSdWarps) * kSdTile + 32 * j + lane;
+            const bool in = t0 + h * kSdWarps < ntiles && c < n;
+            ai[h][j] = in ? As[c] : -1;
+            dv[h][j] = in ? Ds[c] : 0.0;
+          }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            p[h][j] = ai[h][j] >= 0 && static_cast<double>(ss[ai[h][j]]) < 4.0001 * dv[h][j];
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0 + h * kSdWarps;
+        unsigned any = 0u;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int c = t * kSdTile + 32 * j + lane;
-          const unsigned m = __ballot_sync(0xffffffffu, c < n && static_cast<double>(ss[As[c]]) < 4.0001 * Ds[c]);
-          if (lane == 0) tmask[t][j] = m;
+          const unsigned m = __ballot_sync(0xffffffffu, p[h][j]);
+          if (lane == 0 && t < ntiles) tmask[t][j] = m;
           any |= m;
         }
+        if (lane == 0 && t < ntiles) tflag[t] = any ? 1 : 0;
       }
-      if (lane == 0) tflag[t] = any ? 1 : 0;
     }
     __syncthreads();
     if (warp == 0) {
@@ -531,6 +602,9 @@ __global__ void __launch_bounds__(kSdThreads, 1)
       mbar_wait(smem_u32(&bars.full[g % kSdStages]), static_cast<uint32_t>((g / kSdStages) & 1), nullptr,
                 kWhereSeedDrain, kWaitBudgetCycles / 8);
   }
+  if (threadIdx.x == 0 && k > 2)  // the last copy of the seed rows (pass k-2) has landed
+    mbar_wait(smem_u32(&bars.rows), static_cast<uint32_t>((k - 3) & 1), nullptr, kWhereSeedDrain,
+              kWaitBudgetCycles / 8);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
