@@ -354,6 +354,31 @@ def main():
                              "layer_ms": kmeans_ms + ev[0].elapsed_time(ev[1]) + stage_ms["permute"] + a_ms}
         svg2.raise_on_device_error(ws)
 
+    # HBM stages against the measured copy bandwidth: the three row gathers (permutation) as timed
+    # in the step, and the stand-alone inverse permutation (fused into the attention in the step)
+    plane = BH * N * d * 2
+    perm_bytes = 3 * (2 * plane + BH * N * 4)
+    eu = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for _ in range(3):
+        svg2.svg2_unpermute(Qp, perm_q, Kp)  # (Kp is rebuilt by the next step's gathers)
+    eu[0].record(stream)
+    for _ in range(5):
+        svg2.svg2_unpermute(Qp, perm_q, Kp)
+    eu[1].record(stream)
+    torch.cuda.synchronize(dev)
+    unperm_ms = eu[0].elapsed_time(eu[1]) / 5
+    unperm_bytes = 2 * plane + BH * N * 4
+    hbm_stages = {
+        "peak_gbs": P["hbm_gbs"], "peak_source": P["source"] + " copy bandwidth",
+        "permute": {"kernel": "gather_rows_kernel x3", "ms": stage_ms["permute"], "bytes": perm_bytes,
+                    "gbs": perm_bytes / (stage_ms["permute"] * 1e-3) / 1e9,
+                    "frac": perm_bytes / (stage_ms["permute"] * 1e-3) / 1e9 / P["hbm_gbs"]},
+        "unpermute": {"kernel": "scatter_rows_kernel (stand-alone svg2_unpermute)", "ms": unperm_ms,
+                      "bytes": unperm_bytes, "gbs": unperm_bytes / (unperm_ms * 1e-3) / 1e9,
+                      "frac": unperm_bytes / (unperm_ms * 1e-3) / 1e9 / P["hbm_gbs"]},
+    }
+    svg2.svg2_gather(K, perm_k, Kp)
+
     # k-means with k-means++ over all tokens (seed_tokens = 0), for comparison with the sampled seeding
     full_seed = None
     if args.seed_tokens != 0:
@@ -407,6 +432,7 @@ def main():
         "attn_tflops_effective": dense_flops / (attn_ms * 1e-3) / 1e12,
         "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
         "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
+        "hbm_stages": hbm_stages,
         "dense_sdpa_ms": dense_ms, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
         "top_p_sweep": sweep,
     }
@@ -577,7 +603,7 @@ def fixed128_waste(q_off, k_off, mask, heads):
 
 
 def kernel_launches(cfg):
-    per_role = 1 + 1 + cfg.iters * (1 + 3 + 1)   # k-means++, split prep, per iteration: assign, 3 sort, update
+    per_role = 1 + 1 + cfg.iters * (2 + 3 + 1)   # k-means++, split prep, per iteration: assign + re-rank, 3 sort, update
     return 2 * per_role + 1 + 3 + 4               # select, 3 gathers, plan (3) + attention
 
 
