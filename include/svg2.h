@@ -209,8 +209,10 @@ SVG2_API int svg2_layer(const void* Q, const void* K, const void* V, int dtype, 
  * on `copy_stream` K, then Q, then V are copied to the caller's device staging buffers while, on
  * `stream`, the k-means of K starts as soon as K has landed and that of Q as soon as Q has (K's
  * k-means, with more clusters, is the longer one and hides Q's upload); the
- * attention then runs in groups of `heads_per_group` (b,h) planes (0 = all at once) and each
- * group's output is copied back while the next group is computed.  Host buffers must be
+ * attention then runs in groups of `heads_per_group` (b,h) planes (0 = all at once; the last
+ * `heads_per_group` planes go in halves, quarters, ... down to one plane, so that the one copy
+ * back that nothing overlaps is small) and each group's output is copied back while the next
+ * group is computed.  Host buffers must be
  * page-locked (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.  The copies
  * start only after the work already enqueued on `stream`; on return everything is enqueued and
  * `stream` waits for the last copy, so synchronising `stream` covers the whole call.

@@ -455,7 +455,25 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     r = check_ws(ws, ws_bytes, c.off);
     if (r != SVG2_OK) return r;
     const int G = heads_per_group == 0 ? BH : (heads_per_group < BH ? heads_per_group : BH);
-    const int ngroups = (BH + G - 1) / G;
+    // groups of G planes, except that the last G are split into halves, quarters, ... down to one
+    // plane, so that the copy back that nothing overlaps (the last group's) is small
+    std::vector<int> gsize;
+    if (heads_per_group == 0) {
+      gsize.push_back(BH);
+    } else {
+      int left = BH;
+      while (left > G) {
+        gsize.push_back(G);
+        left -= G;
+      }
+      while (left > 1) {
+        const int h = (left + 1) / 2;
+        gsize.push_back(h);
+        left -= h;
+      }
+      if (left == 1) gsize.push_back(1);
+    }
+    const int ngroups = static_cast<int>(gsize.size());
     const bool f32 = dtype == SVG2_F32;
     const size_t esz = f32 ? 4 : 2;
     const size_t bytes_in = static_cast<size_t>(BH) * N * d * esz;
@@ -508,9 +526,9 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     if (e == cudaSuccess) e = launch_gather2(Kd, Vd, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s);
     // attention by head groups; each group's output goes back while the next group runs
     const size_t plane_p = static_cast<size_t>(N) * d;  // elements of one permuted plane
-    for (int g = 0; g < ngroups && e == cudaSuccess; ++g) {
-      const size_t h0 = static_cast<size_t>(g) * G;
-      const int hn = (h0 + G <= static_cast<size_t>(BH)) ? G : BH - static_cast<int>(h0);
+    size_t h0 = 0;
+    for (int g = 0; g < ngroups && e == cudaSuccess; h0 += static_cast<size_t>(gsize[g]), ++g) {
+      const int hn = gsize[g];
       e = launch_sparse_attn(static_cast<const uint16_t*>(L.Qp) + h0 * plane_p,
                              static_cast<const uint16_t*>(L.Kp) + h0 * plane_p,
                              static_cast<const uint16_t*>(L.Vp) + h0 * plane_p, L.q_off + h0 * (p->nQ + 1),
