@@ -396,9 +396,10 @@ def main():
     if not args.no_e2e:
         e2e = measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist)
 
-    dense_ms = None
+    dense_ms = own_dense = None
     if not args.no_dense and rank == 0:
         dense_ms = time_dense(torch, Q, K, V, scale)
+        own_dense = time_own_dense(svg2, torch, Q, K, V, scale)
 
 
     warm = None
@@ -433,7 +434,7 @@ def main():
         "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
         "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
         "hbm_stages": hbm_stages,
-        "dense_sdpa_ms": dense_ms, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
+        "dense_sdpa_ms": dense_ms, "dense_svg2_dense_attn": own_dense, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
         "top_p_sweep": sweep,
     }
     print(json.dumps(line), flush=True)
@@ -576,6 +577,25 @@ def time_dense(torch, Q, K, V, scale, reps=3):
         return a.elapsed_time(b) / reps
     except Exception as e:  # library baseline only; never part of the product path
         return f"unavailable: {type(e).__name__}"
+
+
+def time_own_dense(svg2, torch, Q, K, V, scale, reps=3):
+    """This library's dense attention (the one-cluster case of the same tcgen05 kernel)."""
+    B, H, N, d = Q.shape
+    O = torch.empty_like(Q)
+    ws = svg2.dense_workspace(B, H, N, d, device=Q.device)
+    svg2.svg2_dense_attn(Q, K, V, scale, O, ws)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        svg2.svg2_dense_attn(Q, K, V, scale, O, ws)
+    b.record()
+    torch.cuda.synchronize()
+    svg2.raise_on_device_error(ws)
+    ms = a.elapsed_time(b) / reps
+    flops = 4.0 * N * N * d * B * H
+    return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
 
 
 def fixed128_waste(q_off, k_off, mask, heads):

@@ -168,6 +168,21 @@ SVG2_API int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, co
                      int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O, void* ws,
                      size_t ws_bytes, void* stream);
 
+/*
+ * Dense attention, O = softmax(scale * Q K^T) V per (b,h) over all N keys, on the same tcgen05
+ * kernel as svg2_sparse_attn: the one-cluster case (one Q cluster and one K cluster holding every
+ * token in its original order), so no permutation and no k-means.  This is the layer the pages run
+ * for the first denoising steps before the sparse one takes over (Method; the dense warm-up) and the
+ * reference the sparse layer is compared with at top-p = 1.
+ *   Q, K, V  bf16 [B,H,N,d] (d = 128 or 64), row-major; O bf16 [B,H,N,d], out (may not alias Q, K, V).
+ *   ws       at least svg2_dense_attn_workspace_size() bytes, 256-byte aligned; holds the status
+ *            word (read with svg2_check_status) and the work plan.
+ * Errors: SVG2_ERR_INVALID_ARG (null or unaligned pointers, non-finite scale), SVG2_ERR_UNSUPPORTED
+ * (sizes), SVG2_ERR_WORKSPACE, SVG2_ERR_CUDA (launch). */
+SVG2_API int svg2_dense_attn_workspace_size(int B, int H, int N, int d, size_t* bytes);
+SVG2_API int svg2_dense_attn(const void* Q, const void* K, const void* V, int B, int H, int N, int d, float scale,
+                             void* O, void* ws, size_t ws_bytes, void* stream);
+
 /* Inverse permutation of output rows (Method (2)): O[b,h,perm[b,h,j],:] = Op[b,h,j,:], bf16. */
 SVG2_API int svg2_unpermute(const void* Op, const int32_t* perm, int B, int H, int N, int d, void* O, void* stream);
 

@@ -358,6 +358,58 @@ int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32
   }
 }
 
+namespace {
+struct DenseCarve {
+  DeviceStatus* st;
+  int32_t *q_off, *k_off, *sel_count, *sel_idx;
+  AttnScratch attn;
+};
+void carve_dense(Carve& c, int BH, int N, DenseCarve& D) {
+  D.st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+  D.q_off = c.take<int32_t>(static_cast<size_t>(BH) * 2);
+  D.k_off = c.take<int32_t>(static_cast<size_t>(BH) * 2);
+  D.sel_count = c.take<int32_t>(BH);
+  D.sel_idx = c.take<int32_t>(BH);
+  carve_attn(c, BH, N, 1, D.attn);
+}
+}  // namespace
+
+int svg2_dense_attn_workspace_size(int B, int H, int N, int d, size_t* bytes) {
+  if (bytes == nullptr) return SVG2_ERR_INVALID_ARG;
+  const int r = check_sizes(B, H, N, d);
+  if (r != SVG2_OK) return r;
+  Carve c(nullptr);
+  DenseCarve D;
+  carve_dense(c, B * H, N, D);
+  *bytes = align_up(c.off, 256);
+  return SVG2_OK;
+}
+
+int svg2_dense_attn(const void* Q, const void* K, const void* V, int B, int H, int N, int d, float scale, void* O,
+                    void* ws, size_t ws_bytes, void* stream) {
+  try {
+    int r = check_sizes(B, H, N, d);
+    if (r != SVG2_OK) return r;
+    if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16)) return SVG2_ERR_INVALID_ARG;
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    DenseCarve D;
+    carve_dense(c, BH, N, D);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_dense_plan(BH, N, D.q_off, D.k_off, D.sel_count, D.sel_idx, s);
+    if (e == cudaSuccess)
+      e = launch_sparse_attn(Q, K, V, D.q_off, D.k_off, D.sel_count, D.sel_idx, BH, N, d, 1, 1, scale, nullptr, O,
+                             D.attn, D.st, s);
+    return to_status(e);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
 int svg2_unpermute(const void* Op, const int32_t* perm, int B, int H, int N, int d, void* O, void* stream) {
   try {
     const int r = check_sizes(B, H, N, d);

@@ -609,7 +609,27 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// Dense attention as the one-cluster case: per (b,h) one Q cluster and one K cluster holding all N
+// tokens in their original order, the K cluster selected.
+__global__ void dense_plan_kernel(int BH, int N, int32_t* __restrict__ q_off, int32_t* __restrict__ k_off,
+                                  int32_t* __restrict__ sel_count, int32_t* __restrict__ sel_idx) {
+  const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+  if (bh >= BH) return;
+  q_off[2 * bh] = 0;
+  q_off[2 * bh + 1] = N;
+  k_off[2 * bh] = 0;
+  k_off[2 * bh + 1] = N;
+  sel_count[bh] = 1;
+  sel_idx[bh] = 0;
+}
+
 }  // namespace
+
+cudaError_t launch_dense_plan(int BH, int N, int32_t* q_off, int32_t* k_off, int32_t* sel_count, int32_t* sel_idx,
+                              cudaStream_t s) {
+  dense_plan_kernel<<<(BH + 255) / 256, 256, 0, s>>>(BH, N, q_off, k_off, sel_count, sel_idx);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
                                const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int BH,

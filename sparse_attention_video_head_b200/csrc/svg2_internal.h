@@ -148,6 +148,9 @@ cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, c
                                int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
                                const AttnScratch& scratch, DeviceStatus* st, cudaStream_t s);
 
+cudaError_t launch_dense_plan(int BH, int N, int32_t* q_off, int32_t* k_off, int32_t* sel_count, int32_t* sel_idx,
+                              cudaStream_t s);
+
 cudaError_t launch_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O,
                                 DeviceStatus* st, cudaStream_t s);
 

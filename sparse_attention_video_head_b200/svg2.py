@@ -23,7 +23,8 @@ DEFAULT_SEED_TOKENS = 16384  # SVG2_DEFAULT_SEED_TOKENS
 
 _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeanspp", "svg2_kmeans", "svg2_select",
             "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
-            "svg2_unpermute", "svg2_layer", "svg2_layer_host", "svg2_selftest_mma", "svg2_sparse_attn_noalloc")
+            "svg2_unpermute", "svg2_layer", "svg2_layer_host", "svg2_selftest_mma", "svg2_sparse_attn_noalloc",
+            "svg2_dense_attn_workspace_size", "svg2_dense_attn")
 
 _lib = None
 
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
                                       I, P, S, P, P]
         L.svg2_selftest_mma.argtypes = [P, P, I, P, P, P, P, S, P]
         L.svg2_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
+        L.svg2_dense_attn_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
+        L.svg2_dense_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, S, P]
         for name in _EXPORTS:
             if name != "svg2_status_string":
                 getattr(L, name).restype = I
@@ -210,6 +213,24 @@ def svg2_sparse_attn(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off
     _check(lib().svg2_sparse_attn(_p(Qp), _p(Kp), _p(Vp), _p(q_off), _p(k_off), _p(sel_count), _p(sel_idx), B, H, N,
                                   d, nQ, nK, float(scale), _p(perm_q), _p(O), _p(ws), ws.numel(), _stream(stream)),
            "svg2_sparse_attn")
+
+
+def svg2_dense_attn_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().svg2_dense_attn_workspace_size(B, H, N, d, ctypes.byref(out)), "svg2_dense_attn_workspace_size")
+    return int(out.value)
+
+
+def dense_workspace(B: int, H: int, N: int, d: int, device=None) -> torch.Tensor:
+    """A workspace tensor for svg2_dense_attn (device memory from torch; the status word starts at 0)."""
+    return torch.zeros(svg2_dense_attn_workspace_size(B, H, N, d), dtype=torch.uint8, device=device or "cuda")
+
+
+def svg2_dense_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: float, O: torch.Tensor,
+                    ws: torch.Tensor, stream=None):
+    B, H, N, d = Q.shape
+    _check(lib().svg2_dense_attn(_p(Q), _p(K), _p(V), B, H, N, d, float(scale), _p(O), _p(ws), ws.numel(),
+                                 _stream(stream)), "svg2_dense_attn")
 
 
 def svg2_sparse_attn_noalloc(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off: torch.Tensor,

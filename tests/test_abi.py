@@ -176,3 +176,27 @@ def test_attention_and_layer_reject_bad_arguments(L):
     assert L.svg2_layer(*args[:9], None, *args[10:]) == INVALID          # k-means++ without uniforms
     assert L.svg2_layer(*args[:16], 1024, None) == WORKSPACE
     assert L.svg2_layer(*args[:8], None, *args[9:]) == INVALID
+
+
+def test_dense_attn_rejects_bad_arguments(L):
+    from sparse_attention_video_head_b200 import svg2
+    out = ctypes.c_size_t(0)
+    assert L.svg2_dense_attn_workspace_size(1, 2, 1000, 128, ctypes.byref(out)) == OK and out.value > 0
+    assert L.svg2_dense_attn_workspace_size(1, 2, 1000, 96, ctypes.byref(out)) == UNSUPPORTED
+    assert L.svg2_dense_attn_workspace_size(1, 2, 1000, 128, None) == INVALID
+    # much smaller than the layer's workspace: no permuted copies, one cluster
+    assert svg2.svg2_dense_attn_workspace_size(1, 40, 75600, 128) < svg2.svg2_workspace_size(1, 40, 75600, 128, 1, 1) // 100
+    ws_ok = 1 << 30
+    call = lambda **kw: L.svg2_dense_attn(*[dict(dict(Q=FAKE, K=FAKE, V=FAKE, B=1, H=2, N=1000, d=128, s=0.08, O=FAKE,
+                                                      ws=FAKE, wsb=ws_ok, st=None), **kw)[n]
+                                            for n in ("Q", "K", "V", "B", "H", "N", "d", "s", "O", "ws", "wsb", "st")])
+    assert call(Q=None) == INVALID
+    assert call(O=None) == INVALID
+    assert call(V=ctypes.c_void_p(0x10008)) == INVALID            # not 16-byte aligned
+    assert call(s=float("nan")) == INVALID
+    assert call(s=float("inf")) == INVALID
+    assert call(d=96) == UNSUPPORTED
+    assert call(N=0) == INVALID
+    assert call(ws=None) == WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x10010)) == WORKSPACE        # not 256-byte aligned
+    assert call(wsb=16) == WORKSPACE
