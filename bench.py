@@ -10,7 +10,8 @@ through the C ABI of libsvg2.  Prints one JSON line (rank 0).
   python bench.py --impl reference ...     # the CPU oracle, timed on a bounded sample
 
 With N > 1 (torchrun), every rank runs its own layer (replicas, weak scaling: the layer's heads
-are independent and there is no exchange on the path); the time is the max over ranks.
+are independent and there is no exchange on the path); the time is the max over ranks.  With
+--shard heads the ranks instead split the heads of one layer (strong scaling, still no exchange).
 """
 from __future__ import annotations
 
@@ -47,6 +48,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the top-p sweep (selection + attention per p)")
     ap.add_argument("--heads", type=int, default=0, help="run only this many heads of the layer (profiling cases)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: every rank runs its own layer (replicas, weak scaling) or the ranks split the "
+                         "heads of one layer (strong scaling)")
     ap.add_argument("--no-warm", action="store_true", help="skip the warm-start denoising-sequence measurement")
     ap.add_argument("--warm-steps", type=int, default=10)
     ap.add_argument("--seed-tokens", type=int, default=16384,
@@ -64,13 +68,16 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
-def gen_inputs(cfg, step=0):
+def gen_inputs(cfg, step=0, heads=None):
+    """The layer's synthetic inputs for `heads` (default: all of them), stacked as [1, len(heads), ...]."""
     import multiprocessing as mp
-    procs = max(1, min(cfg.H, len(os.sched_getaffinity(0))))
+    heads = list(range(cfg.H)) if heads is None else list(heads)
+    procs = max(1, min(len(heads), len(os.sched_getaffinity(0))))
     if procs == 1:
-        return I.layer_inputs(cfg, step)
-    with mp.get_context("spawn").Pool(procs) as pool:
-        parts = pool.starmap(I.head_inputs, [(cfg, 0, h, step) for h in range(cfg.H)])
+        parts = [I.head_inputs(cfg, 0, h, step) for h in heads]
+    else:
+        with mp.get_context("spawn").Pool(procs) as pool:
+            parts = pool.starmap(I.head_inputs, [(cfg, 0, h, step) for h in heads])
     return {k: np.stack([p[k] for p in parts])[None] for k in parts[0]}
 
 
@@ -149,13 +156,15 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(cfg, top_p, seed_tokens):
-    return {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "grid": list(cfg.grid), "d": cfg.d,
+def config_dict(cfg, top_p, seed_tokens, shard=None):
+    """`shard` = (layer heads, world) when the ranks split one layer's heads; cfg.H is then the rank's."""
+    heads, world = shard if shard else (cfg.H, 1)
+    return {"workload": cfg.name, "B": cfg.B, "H": heads, "N": cfg.N, "grid": list(cfg.grid), "d": cfg.d,
             "nQ": cfg.nQ, "nK": cfg.nK, "iters": cfg.iters, "init": "kmeans++", "top_p": top_p,
             "kmeanspp_seed_tokens": seed_tokens,
             "components": cfg.components, "sigma": cfg.sigma,
             "l2": "inputs larger than L2 (each of Q, K, V is %.0f MB)" % (cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6),
-            "parallelism": "replicas"}
+            "parallelism": f"heads/{world}" if shard else "replicas"}
 
 
 def max_over_ranks(value: float, world: int, dist, device) -> float:
@@ -168,9 +177,10 @@ def max_over_ranks(value: float, world: int, dist, device) -> float:
     return float(t.item())
 
 
-def whole_job_ms_per_layer(ms_per_step: float, world: int) -> float:
-    """Weak scaling with one layer per rank per step: the job finishes `world` layers per step."""
-    return ms_per_step / world
+def whole_job_ms_per_layer(ms_per_step: float, world: int, sharded: bool = False) -> float:
+    """Replicas (weak scaling, one layer per rank per step): the job finishes `world` layers per
+    step.  Heads split across the ranks (strong scaling): one layer per step."""
+    return ms_per_step if sharded else ms_per_step / world
 
 
 # ------------------------------------------------------------------------------------------ clocks
@@ -235,7 +245,19 @@ def main():
         if rank == 0:
             run_reference(args, cfg)
         return
-    data = gen_inputs(cfg)  # before CUDA initialisation
+    sharded = args.shard == "heads" and world > 1
+    shard_info = None
+    if sharded:
+        import dataclasses
+        from sparse_attention_video_head_b200.shard import head_range
+        h0, h1 = head_range(cfg.H, world, rank)
+        if h1 == h0:
+            raise SystemExit(f"--shard heads needs at least one head per rank ({cfg.H} heads, {world} ranks)")
+        data = gen_inputs(cfg, heads=range(h0, h1))  # this rank's block of the layer's heads
+        shard_info = (cfg.H, world)
+        cfg = dataclasses.replace(cfg, H=h1 - h0)
+    else:
+        data = gen_inputs(cfg)  # before CUDA initialisation
 
     import torch
     import torch.distributed as dist
@@ -418,9 +440,10 @@ def main():
                "sample": sample_text(cfg, 256, heads), "parts_s": parts}
     launches = kernel_launches(cfg)
     line = {
-        "metric": METRIC, "value": whole_job_ms_per_layer(ms_per_step, world), "unit": "ms", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.top_p, args.seed_tokens),
+        "metric": METRIC, "value": whole_job_ms_per_layer(ms_per_step, world, sharded), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
+        "scaling": "strong" if sharded else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.top_p, args.seed_tokens, shard_info),
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel", "achieved": achieved_tflops,
                      "peak": P["bf16_sustained"], "unit": "TFLOP/s",
                      "frac": achieved_tflops / P["bf16_sustained"],
@@ -481,7 +504,8 @@ def measure_e2e(svg2, torch, cfg, data, args, dev, ws, world, dist):
     svg2.raise_on_device_error(ws)
     ms = max_over_ranks(a.elapsed_time(b) / steps, world, dist, dev)
     h2d = 3 * hq.numel() * 2 + (huq.numel() + huk.numel()) * 8
-    return {"value": whole_job_ms_per_layer(ms, world), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
+    return {"value": whole_job_ms_per_layer(ms, world, args.shard == "heads" and world > 1), "unit": "ms",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2,
             "steps": steps, "api": "svg2_layer_host", "heads_per_group": args.e2e_heads_per_group}
 
 
