@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the top-p sweep (selection + attention per p)")
     ap.add_argument("--heads", type=int, default=0, help="run only this many heads of the layer (profiling cases)")
+    ap.add_argument("--no-denoise", action="store_true", help="skip the denoising-loop driver measurement")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N > 1: every rank runs its own layer (replicas, weak scaling) or the ranks split the "
                          "heads of one layer (strong scaling)")
@@ -424,6 +425,10 @@ def main():
         own_dense = time_own_dense(svg2, torch, Q, K, V, scale)
 
 
+    denoise = None
+    if not args.no_denoise and rank == 0:
+        denoise = measure_denoise(svg2, torch, cfg, args, dev, Q, K, V, scale)
+
     warm = None
     if not args.no_warm:
         warm = measure_warm(svg2, torch, cfg, args, dev, Q, K, V, ws, scale)
@@ -457,7 +462,7 @@ def main():
         "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
         "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
         "hbm_stages": hbm_stages,
-        "dense_sdpa_ms": dense_ms, "dense_svg2_dense_attn": own_dense, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
+        "dense_sdpa_ms": dense_ms, "dense_svg2_dense_attn": own_dense, "denoise_driver": denoise, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
         "top_p_sweep": sweep,
     }
     print(json.dumps(line), flush=True)
@@ -601,6 +606,44 @@ def time_dense(torch, Q, K, V, scale, reps=3):
         return a.elapsed_time(b) / reps
     except Exception as e:  # library baseline only; never part of the product path
         return f"unavailable: {type(e).__name__}"
+
+
+def measure_denoise(svg2, torch, cfg, args, dev, Q, K, V, scale, steps=6, dense_steps=1):
+    """The denoising-loop driver over a short schedule of one layer: `dense_steps` dense steps, then
+    a cold k-means step, then warm steps (2 iterations from the layer's cached centroids).  The
+    inputs are the step's tensors re-used each step (the k-means work per warm step is fixed at 2
+    iterations whatever the drift).  Reports ms per step kind and the schedule's mean per step."""
+    B, H, N, d = Q.shape
+    p = svg2.LayerParams(nQ=cfg.nQ, nK=cfg.nK, iters=cfg.iters, top_p=args.top_p, scale=scale,
+                         seed_tokens=args.seed_tokens)
+    drv = svg2.Driver(B, H, N, d, num_steps=steps, num_layers=1, dense_steps=dense_steps, warm_iters=2, params=p,
+                      device=dev)
+    rng = np.random.default_rng(4321)
+    uq = torch.from_numpy(rng.random((B, H, cfg.nQ))).to(dev)
+    uk = torch.from_numpy(rng.random((B, H, cfg.nK))).to(dev)
+    O = torch.empty_like(Q)
+    names = {svg2.SVG2_STEP_DENSE: "dense", svg2.SVG2_STEP_COLD: "cold", svg2.SVG2_STEP_WARM: "warm"}
+    for s in range(steps):  # warm-up pass over the schedule
+        drv.layer(s, 0, Q, K, V, O, uq, uk)
+    drv.reset()
+    per = {}
+    total = 0.0
+    for s in range(steps):
+        kind = names[drv.plan(s, 0)]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        drv.layer(s, 0, Q, K, V, O, uq, uk)
+        b.record()
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b)
+        per.setdefault(kind, []).append(ms)
+        total += ms
+    svg2.raise_on_device_error(drv.ws)
+    out = {"steps": steps, "dense_steps": dense_steps, "warm_iters": 2,
+           "ms": {k: statistics.mean(v) for k, v in per.items()}, "mean_ms_per_step": total / steps,
+           "api": "svg2_driver_layer"}
+    drv.close()
+    return out
 
 
 def time_own_dense(svg2, torch, Q, K, V, scale, reps=3):

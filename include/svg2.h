@@ -271,6 +271,47 @@ SVG2_API int svg2_sparse_attn_noalloc(const void* Qp, const void* Kp, const void
 SVG2_API int svg2_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O, void* ws,
                       size_t ws_bytes, void* stream);
 
+/*
+ * Denoising-loop driver: the schedule the pages run around the layer.  Over num_steps denoising
+ * steps and num_layers attention layers, steps 0 .. dense_steps-1 run dense attention
+ * (svg2_dense_attn; the pages keep full attention for the first steps); a layer's first sparse
+ * step starts its k-means cold (k-means++ seeding and layer.iters Lloyd iterations); its later
+ * steps start warm from the centroids it left at its previous sparse step, with warm_iters
+ * iterations (the centroid cache across steps of Key claims section 4.3, Fig. 7(a)).
+ * The driver holds host state only (the schedule, which layers' caches hold centroids) and does
+ * not touch the GPU except through the layer calls it makes.  Its centroid cache is caller-owned
+ * device memory: num_layers x [B,H,nQ,d] then [B,H,nK,d] float32, svg2_driver_cache_bytes()
+ * bytes, 16-byte aligned, bound with svg2_driver_bind_cache (binding marks every layer cold;
+ * svg2_driver_reset does the same for a new video).  One driver serves one stream at a time.
+ * Errors: SVG2_ERR_INVALID_ARG (null handle or pointers, step or layer out of range, bad config),
+ * SVG2_ERR_UNSUPPORTED (d), SVG2_ERR_WORKSPACE (no or too small cache, workspace), and the errors
+ * of the layer calls.
+ */
+typedef struct svg2_driver svg2_driver;
+typedef struct {
+  int num_steps, num_layers;
+  int dense_steps;    /* steps 0 .. dense_steps-1 run dense attention (0 <= dense_steps <= num_steps) */
+  int warm_iters;     /* Lloyd iterations of a warm-started k-means (>= 1; 2 in the pages) */
+  svg2_params layer;  /* the sparse layer; layer.iters is the cold start's, layer.init is ignored */
+} svg2_driver_config;
+typedef enum { SVG2_STEP_DENSE = 0, SVG2_STEP_COLD = 1, SVG2_STEP_WARM = 2 } svg2_step_kind;
+
+SVG2_API int svg2_driver_create(const svg2_driver_config* cfg, int B, int H, int N, int d, svg2_driver** out);
+SVG2_API int svg2_driver_destroy(svg2_driver* drv);
+SVG2_API int svg2_driver_cache_bytes(const svg2_driver* drv, size_t* bytes);
+SVG2_API int svg2_driver_bind_cache(svg2_driver* drv, float* cache, size_t bytes);
+SVG2_API int svg2_driver_reset(svg2_driver* drv);
+/* Bytes of workspace that both the dense and the sparse layer calls of this driver fit in. */
+SVG2_API int svg2_driver_workspace_size(const svg2_driver* drv, size_t* bytes);
+/* What svg2_driver_layer(step, layer) will run now: a svg2_step_kind in *kind. */
+SVG2_API int svg2_driver_plan(const svg2_driver* drv, int step, int layer, int* kind);
+/* Runs layer `layer` of step `step` on bf16 Q, K, V [B,H,N,d] into O (bf16, token order), on
+ * `stream`: dense, cold (uq, uk: the k-means++ uniforms as in svg2_layer) or warm, per
+ * svg2_driver_plan.  A sparse call that returns SVG2_OK leaves the layer's cache warm. */
+SVG2_API int svg2_driver_layer(svg2_driver* drv, int step, int layer, const void* Q, const void* K, const void* V,
+                               const double* uq, const double* uk, void* O, void* ws, size_t ws_bytes,
+                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,9 @@ DEFAULT_SEED_TOKENS = 16384  # SVG2_DEFAULT_SEED_TOKENS
 _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "svg2_kmeanspp", "svg2_kmeans", "svg2_select",
             "svg2_select_from_weights", "svg2_sort", "svg2_gather", "svg2_permute", "svg2_sparse_attn",
             "svg2_unpermute", "svg2_layer", "svg2_layer_host", "svg2_selftest_mma", "svg2_sparse_attn_noalloc",
-            "svg2_dense_attn_workspace_size", "svg2_dense_attn")
+            "svg2_dense_attn_workspace_size", "svg2_dense_attn", "svg2_driver_create", "svg2_driver_destroy",
+            "svg2_driver_cache_bytes", "svg2_driver_bind_cache", "svg2_driver_reset", "svg2_driver_workspace_size",
+            "svg2_driver_plan", "svg2_driver_layer")
 
 _lib = None
 
@@ -39,6 +41,11 @@ class SvgParams(ctypes.Structure):
     _fields_ = [("nQ", ctypes.c_int), ("nK", ctypes.c_int), ("iters", ctypes.c_int), ("init", ctypes.c_int),
                 ("top_p", ctypes.c_float), ("scale", ctypes.c_float), ("seed_tokens", ctypes.c_int),
                 ("fuse_unpermute", ctypes.c_int)]
+
+
+class SvgDriverConfig(ctypes.Structure):
+    _fields_ = [("num_steps", ctypes.c_int), ("num_layers", ctypes.c_int), ("dense_steps", ctypes.c_int),
+                ("warm_iters", ctypes.c_int), ("layer", SvgParams)]
 
 
 class SvgLayerOutputs(ctypes.Structure):
@@ -77,6 +84,14 @@ def lib() -> ctypes.CDLL:
         L.svg2_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
         L.svg2_dense_attn_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
         L.svg2_dense_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, S, P]
+        L.svg2_driver_create.argtypes = [ctypes.POINTER(SvgDriverConfig), I, I, I, I, ctypes.POINTER(P)]
+        L.svg2_driver_destroy.argtypes = [P]
+        L.svg2_driver_cache_bytes.argtypes = [P, ctypes.POINTER(S)]
+        L.svg2_driver_bind_cache.argtypes = [P, P, S]
+        L.svg2_driver_reset.argtypes = [P]
+        L.svg2_driver_workspace_size.argtypes = [P, ctypes.POINTER(S)]
+        L.svg2_driver_plan.argtypes = [P, I, I, ctypes.POINTER(I)]
+        L.svg2_driver_layer.argtypes = [P, I, I, P, P, P, P, P, P, P, S, P]
         for name in _EXPORTS:
             if name != "svg2_status_string":
                 getattr(L, name).restype = I
@@ -308,6 +323,61 @@ def svg2_layer_host(Qh: torch.Tensor, Kh: torch.Tensor, Vh: torch.Tensor, Oh: to
     _check(lib().svg2_layer_host(_hp(Qh), _hp(Kh), _hp(Vh), _hp(Oh), _p(Q), _p(K), _p(V), _p(O), _dtype(Qh), B, H, N, d,
                                  ctypes.byref(prm), _p(uq), _p(uk), _p(cq), _p(ck), int(heads_per_group), _p(ws),
                                  ws.numel(), _stream(stream), cs), "svg2_layer_host")
+
+
+SVG2_STEP_DENSE, SVG2_STEP_COLD, SVG2_STEP_WARM = 0, 1, 2
+
+
+class Driver:
+    """The denoising-loop driver (svg2_driver_*): dense attention for the first `dense_steps` steps,
+    then per layer a cold k-means at its first sparse step and warm starts from its own cached
+    centroids afterwards.  The cache and the workspace are torch device tensors owned here."""
+
+    def __init__(self, B: int, H: int, N: int, d: int, num_steps: int, num_layers: int, dense_steps: int,
+                 warm_iters: int, params: LayerParams, device="cuda", allocate: bool = True):
+        self._h = ctypes.c_void_p(None)
+        cfg = SvgDriverConfig(num_steps, num_layers, dense_steps, warm_iters, params.c())
+        _check(lib().svg2_driver_create(ctypes.byref(cfg), B, H, N, d, ctypes.byref(self._h)), "svg2_driver_create")
+        self.shape = (B, H, N, d)
+        self.cache = self.ws = None
+        if allocate:
+            self.cache = torch.zeros(self.cache_bytes() // 4, dtype=torch.float32, device=device)
+            _check(lib().svg2_driver_bind_cache(self._h, _p(self.cache), self.cache.numel() * 4), "svg2_driver_bind_cache")
+            self.ws = torch.zeros(self.workspace_bytes(), dtype=torch.uint8, device=device)
+
+    def cache_bytes(self) -> int:
+        out = ctypes.c_size_t(0)
+        _check(lib().svg2_driver_cache_bytes(self._h, ctypes.byref(out)), "svg2_driver_cache_bytes")
+        return int(out.value)
+
+    def workspace_bytes(self) -> int:
+        out = ctypes.c_size_t(0)
+        _check(lib().svg2_driver_workspace_size(self._h, ctypes.byref(out)), "svg2_driver_workspace_size")
+        return int(out.value)
+
+    def plan(self, step: int, layer: int) -> int:
+        kind = ctypes.c_int(-1)
+        _check(lib().svg2_driver_plan(self._h, step, layer, ctypes.byref(kind)), "svg2_driver_plan")
+        return int(kind.value)
+
+    def reset(self):
+        _check(lib().svg2_driver_reset(self._h), "svg2_driver_reset")
+
+    def layer(self, step: int, layer: int, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
+              uq: Optional[torch.Tensor] = None, uk: Optional[torch.Tensor] = None, stream=None):
+        _check(lib().svg2_driver_layer(self._h, step, layer, _p(Q), _p(K), _p(V), _p(uq), _p(uk), _p(O), _p(self.ws),
+                                       self.ws.numel(), _stream(stream)), "svg2_driver_layer")
+
+    def close(self):
+        if self._h:
+            lib().svg2_driver_destroy(self._h)
+            self._h = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def svg2_selftest_mma(A: torch.Tensor, Bm: torch.Tensor, V: torch.Tensor, ws: torch.Tensor, stream=None):
