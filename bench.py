@@ -83,10 +83,10 @@ def gen_inputs(cfg, step=0, heads=None):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 240.4 MB + 69.6 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 239.9 MB + 68.0 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "5417b3a76e68752364c031ffe180745c47cc2cd53d012c74c18184396a1c516b",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 240.430080e6 + 69.561600e6,
+ATTN_TRAFFIC = {"sha256": "63ea0eeb193d63e8934ca4adae42c4976e0f0c7ac761c89790ffe9b393c0790e",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 239.936000e6 + 67.964672e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 
