@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--config", default="wan720p", choices=sorted(I.CONFIGS))
     ap.add_argument("--top-p", type=float, default=0.9)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-heads-per-group", type=int, default=8,
+    ap.add_argument("--e2e-heads-per-group", type=int, default=12,
                     help="heads per transfer group in the end-to-end call (copies overlap the other groups' compute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")

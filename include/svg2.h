@@ -221,9 +221,10 @@ SVG2_API int svg2_layer(const void* Q, const void* K, const void* V, int dtype, 
 
 /*
  * svg2_layer for inputs and output in host memory, with the transfers overlapped with the work:
- * on `copy_stream` K, then Q, then V are copied to the caller's device staging buffers while, on
- * `stream`, the k-means of K starts as soon as K has landed and that of Q as soon as Q has (K's
- * k-means, with more clusters, is the longer one and hides Q's upload); the
+ * on `copy_stream` K (in two halves of the planes), then Q, then V (per attention group) are copied
+ * to the caller's device staging buffers while, on `stream`, the k-means of each half of K starts
+ * as soon as that half has landed and that of Q as soon as Q has (K's k-means, with more clusters,
+ * is the longer one and hides Q's upload), and each group's K/V gathers wait only for its own V; the
  * attention then runs in groups of `heads_per_group` (b,h) planes (0 = all at once; the last
  * `heads_per_group` planes go in halves, quarters, ... down to one plane, so that the one copy
  * back that nothing overlaps is small) and each group's output is copied back while the next

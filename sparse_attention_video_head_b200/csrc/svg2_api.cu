@@ -533,9 +533,14 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaStream_t cs = copy_stream != nullptr ? static_cast<cudaStream_t>(copy_stream) : s;
 
-    // events: entry (copies wait for prior work on `stream`), Q/K/V landed, each group's output
-    // ready, all copies done
-    std::vector<cudaEvent_t> ev(5 + ngroups, nullptr);
+    // K is uploaded, and clustered, in two halves of the planes, so that the first half's k-means
+    // starts while the second half is still in flight; V goes up per attention group, so that a
+    // group's gathers and attention need only its own planes.
+    const int nkc = BH >= 2 ? 2 : 1;
+    const int kc_split = (BH + 1) / 2;
+    // events: entry (copies wait for prior work on `stream`), Q landed, all copies done, each K
+    // half landed, each group's V landed, each group's output ready
+    std::vector<cudaEvent_t> ev(3 + nkc + 2 * ngroups, nullptr);
     cudaError_t e = cudaSuccess;
     for (auto& x : ev)
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
@@ -547,25 +552,53 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
       release();
       return SVG2_ERR_CUDA;
     }
-    cudaEvent_t entry = ev[0], q_in = ev[1], k_in = ev[2], v_in = ev[3], all_out = ev[4];
+    cudaEvent_t entry = ev[0], q_in = ev[1], all_out = ev[2];
+    cudaEvent_t* k_in = ev.data() + 3;
+    cudaEvent_t* v_in = k_in + nkc;
+    cudaEvent_t* o_out = v_in + ngroups;
     auto ok = [&](cudaError_t x) {
       if (e == cudaSuccess) e = x;
       return e == cudaSuccess;
+    };
+    const size_t plane_in = static_cast<size_t>(N) * d * esz;  // bytes of one input plane
+    auto kc_range = [&](int c, int& h0c, int& hnc) {
+      h0c = c == 0 ? 0 : kc_split;
+      hnc = nkc == 1 ? BH : (c == 0 ? kc_split : BH - kc_split);
     };
     ok(cudaEventRecord(entry, s));
     ok(cudaStreamWaitEvent(cs, entry, 0));
     // inputs in the order the computation needs them: K first (its k-means, with more clusters than
     // Q's, is the longer of the two and hides the upload of Q), then Q, then V
-    ok(cudaMemcpyAsync(Kd, Kh, bytes_in, cudaMemcpyHostToDevice, cs));
-    ok(cudaEventRecord(k_in, cs));
+    for (int c = 0; c < nkc; ++c) {
+      int h0c, hnc;
+      kc_range(c, h0c, hnc);
+      ok(cudaMemcpyAsync(static_cast<char*>(Kd) + h0c * plane_in, static_cast<const char*>(Kh) + h0c * plane_in,
+                         hnc * plane_in, cudaMemcpyHostToDevice, cs));
+      ok(cudaEventRecord(k_in[c], cs));
+    }
     ok(cudaMemcpyAsync(Qd, Qh, bytes_in, cudaMemcpyHostToDevice, cs));
     ok(cudaEventRecord(q_in, cs));
-    ok(cudaMemcpyAsync(Vd, Vh, bytes_in, cudaMemcpyHostToDevice, cs));
-    ok(cudaEventRecord(v_in, cs));
-    ok(cudaStreamWaitEvent(s, k_in, 0));
-    if (e == cudaSuccess)
-      e = run_kmeans(Kd, f32, BH, N, d, p->nK, p->iters, p->init, uk, p->seed_tokens, ck, L.labels_k, L.count_k,
-                     L.perm_k, L.k_off, L.kk, L.st, s);
+    {
+      size_t h0 = 0;
+      for (int g = 0; g < ngroups; h0 += static_cast<size_t>(gsize[g]), ++g) {
+        ok(cudaMemcpyAsync(static_cast<char*>(Vd) + h0 * plane_in, static_cast<const char*>(Vh) + h0 * plane_in,
+                           gsize[g] * plane_in, cudaMemcpyHostToDevice, cs));
+        ok(cudaEventRecord(v_in[g], cs));
+      }
+    }
+    // k-means of K, half by half (the planes are independent problems; the scratch serves the
+    // halves in turn on the one stream)
+    for (int c = 0; c < nkc && e == cudaSuccess; ++c) {
+      int h0c, hnc;
+      kc_range(c, h0c, hnc);
+      ok(cudaStreamWaitEvent(s, k_in[c], 0));
+      const size_t hb = static_cast<size_t>(h0c);
+      if (e == cudaSuccess)
+        e = run_kmeans(static_cast<const char*>(Kd) + hb * plane_in, f32, hnc, N, d, p->nK, p->iters, p->init,
+                       uk != nullptr ? uk + hb * p->nK : nullptr, p->seed_tokens, ck + hb * p->nK * d,
+                       L.labels_k + hb * N, L.count_k + hb * p->nK, L.perm_k + hb * N, L.k_off + hb * (p->nK + 1),
+                       L.kk, L.st, s);
+    }
     ok(cudaStreamWaitEvent(s, q_in, 0));
     if (e == cudaSuccess)
       e = run_kmeans(Qd, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q,
@@ -574,21 +607,26 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, nullptr, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);
     if (e == cudaSuccess) e = launch_gather(Qd, f32, L.perm_q, BH, N, d, L.Qp, s);
-    ok(cudaStreamWaitEvent(s, v_in, 0));
-    if (e == cudaSuccess) e = launch_gather2(Kd, Vd, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s);
-    // attention by head groups; each group's output goes back while the next group runs
+    // per head group: gather its K and V planes once its V has landed, attend, and copy the output
+    // back while the next group runs
     const size_t plane_p = static_cast<size_t>(N) * d;  // elements of one permuted plane
     size_t h0 = 0;
     for (int g = 0; g < ngroups && e == cudaSuccess; h0 += static_cast<size_t>(gsize[g]), ++g) {
       const int hn = gsize[g];
+      ok(cudaStreamWaitEvent(s, v_in[g], 0));
+      if (e == cudaSuccess)
+        e = launch_gather2(static_cast<const char*>(Kd) + h0 * plane_in, static_cast<const char*>(Vd) + h0 * plane_in,
+                           f32, L.perm_k + h0 * N, hn, N, d, static_cast<uint16_t*>(L.Kp) + h0 * plane_p,
+                           static_cast<uint16_t*>(L.Vp) + h0 * plane_p, s);
+      if (e != cudaSuccess) break;
       e = launch_sparse_attn(static_cast<const uint16_t*>(L.Qp) + h0 * plane_p,
                              static_cast<const uint16_t*>(L.Kp) + h0 * plane_p,
                              static_cast<const uint16_t*>(L.Vp) + h0 * plane_p, L.q_off + h0 * (p->nQ + 1),
                              L.k_off + h0 * (p->nK + 1), L.sel_count + h0 * p->nQ,
                              L.sel_idx + h0 * static_cast<size_t>(p->nQ) * p->nK, hn, N, d, p->nQ, p->nK, p->scale,
                              L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st, s);
-      ok(cudaEventRecord(ev[5 + g], s));
-      ok(cudaStreamWaitEvent(cs, ev[5 + g], 0));
+      ok(cudaEventRecord(o_out[g], s));
+      ok(cudaStreamWaitEvent(cs, o_out[g], 0));
       ok(cudaMemcpyAsync(static_cast<char*>(Oh) + h0 * plane_out, static_cast<const char*>(Od) + h0 * plane_out,
                          hn * plane_out, cudaMemcpyDeviceToHost, cs));
     }
