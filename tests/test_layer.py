@@ -186,3 +186,48 @@ def test_host_buffer_layer_matches_device_layer(heads_per_group, separate_copy_s
     assert torch.equal(ho.view(torch.int16), torch.from_numpy(ref["o"]).to(torch.bfloat16).view(torch.int16))
     np.testing.assert_array_equal(host(cq), ref["cq"])
     np.testing.assert_array_equal(host(ck), ref["ck"])
+
+
+def _mixture(rng, B, H, N, d, comps=8, sigma=0.3):
+    out = np.empty((B, H, N, d), np.float32)
+    for b in range(B):
+        for h in range(H):
+            centres = rng.standard_normal((comps, d), dtype=np.float32)
+            out[b, h] = centres[rng.integers(0, comps, N)] + sigma * rng.standard_normal((N, d), dtype=np.float32)
+    return I.round_to_bf16(out)
+
+
+def _run_and_check(oracle, B, H, N, nQ, nK, iters, top_p, seed_tokens, seed):
+    """svg2_layer on a (B, H) batch of mixtures, every (b, h) plane checked stage by stage."""
+    from types import SimpleNamespace
+    svg2 = require_gpu()
+    rng = np.random.default_rng(seed)
+    d = 128
+    data = {"q": _mixture(rng, B, H, N, d), "k": _mixture(rng, B, H, N, d),
+            "v": I.round_to_bf16(rng.standard_normal((B, H, N, d), dtype=np.float32)),
+            "uq": rng.random((B, H, nQ)), "uk": rng.random((B, H, nK))}
+    cfg = SimpleNamespace(nQ=nQ, nK=nK, iters=iters, scale=float(np.float32(1 / np.sqrt(d))), dtype="bf16")
+    res = run_layer(svg2, cfg, data, top_p, seed_tokens=seed_tokens)
+    stats = []
+    for b in range(B):
+        db = {key: val[b:b + 1] for key, val in data.items()}
+        rb = {key: val[b:b + 1] for key, val in res.items()}
+        for h in range(H):
+            stats.append(check_head(oracle, cfg, db, rb, h, top_p))
+    return stats
+
+
+@pytest.mark.gpu
+def test_layer_batch_of_two_ragged_length(oracle):
+    """B = 2 (every kernel indexes (b, h) planes), N = 1000 (ragged 128-row tiles and 256-row units),
+    k-means++ over strided candidates."""
+    stats = _run_and_check(oracle, B=2, H=3, N=1000, nQ=12, nK=40, iters=3, top_p=0.9, seed_tokens=400, seed=21)
+    print(stats)
+
+
+@pytest.mark.gpu
+def test_layer_degenerate_cluster_counts(oracle):
+    """One Q cluster holding every token, and as many K clusters as tokens (k-means++ then runs out of
+    positive D^2 and picks repeated seeds, so some K clusters stay empty)."""
+    stats = _run_and_check(oracle, B=1, H=2, N=300, nQ=1, nK=300, iters=2, top_p=0.5, seed_tokens=0, seed=22)
+    print(stats)
