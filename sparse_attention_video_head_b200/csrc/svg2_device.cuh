@@ -424,9 +424,6 @@ __device__ __forceinline__ void st_async_u64(void* local, uint64_t* bar, uint32_
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u64 [%0], %1, [%2];" ::"r"(ra), "l"(v), "r"(rb)
                : "memory");
 }
-__device__ __forceinline__ void st_cluster_f64(void* local, uint32_t rank, double v) {
-  st_cluster_u64(local, rank, static_cast<unsigned long long>(__double_as_longlong(v)));
-}
 
 // bf16 helpers
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -1125,23 +1125,44 @@ __global__ void __launch_bounds__(kUpdThreads) update_kernel(const void* __restr
   float* cj = C + (static_cast<size_t>(bh) * k + j) * D;
   const int32_t* pr = perm + static_cast<size_t>(bh) * N;
   const char* xb = static_cast<const char*>(X) + static_cast<size_t>(bh) * N * ROWB;
-  auto issue = [&](int batch, int b) {
+  // Each thread copies kPer 16-byte chunks of a batch.  The member indices of a batch are read one
+  // batch before its copies are issued, so a copy never waits for its index load.
+  constexpr int kPer = kUpdRows * CH / kUpdThreads;
+  static_assert(kPer * kUpdThreads == kUpdRows * CH, "chunks per thread");
+  auto load_idx = [&](int batch, int (&t)[kPer]) {
+    const int r0 = o0 + batch * kUpdRows;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int row = r0 + (tid + i * kUpdThreads) / CH;
+      t[i] = row < o1 ? __ldg(pr + row) : 0;
+    }
+  };
+  auto issue = [&](int batch, int b, const int (&t)[kPer]) {
     const int r0 = o0 + batch * kUpdRows;
     const int nr = min(kUpdRows, o1 - r0);
-    for (int q = tid; q < nr * CH; q += kUpdThreads) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int q = tid + i * kUpdThreads;
       const int r = q / CH, c = q - r * CH;
-      int t = __ldg(pr + r0 + r);
-      t = t < 0 ? 0 : (t >= N ? N - 1 : t);
-      cp_async16(smem_u32(&buf[b][r * ROWB + c * 16]), xb + static_cast<size_t>(t) * ROWB + c * 16);
+      if (r < nr) {
+        const int tk = t[i] < 0 ? 0 : (t[i] >= N ? N - 1 : t[i]);
+        cp_async16(smem_u32(&buf[b][r * ROWB + c * 16]), xb + static_cast<size_t>(tk) * ROWB + c * 16);
+      }
     }
     cp_async_commit();
   };
   double acc = 0.0;
   const int nb = (cnt + kUpdRows - 1) / kUpdRows;
-  if (nb > 0) issue(0, 0);
+  int tix[kPer];
+  if (nb > 0) {
+    load_idx(0, tix);
+    issue(0, 0, tix);
+  }
+  if (nb > 1) load_idx(1, tix);
   for (int b = 0; b < nb; ++b) {
     if (b + 1 < nb) {
-      issue(b + 1, (b + 1) & 1);
+      issue(b + 1, (b + 1) & 1, tix);
+      if (b + 2 < nb) load_idx(b + 2, tix);  // lands while batch b is summed
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
