@@ -357,7 +357,11 @@ def main():
     if not args.no_sweep:
         sweep = {}
         kmeans_ms = stage_ms["kmeans_q"] + stage_ms["kmeans_k"]
-        for p in sorted(set(cfg.top_p) | {args.top_p}):
+        # the configuration's top-p values, plus two labelled extension points: p = 0.5 (towards the
+        # pages' 25-35 % densities on these inputs) and p = 1 (every pair kept: dense attention through
+        # the sparse path)
+        extension = {0.5: "extension: lower density", 1.0: "extension: every pair kept (dense through the sparse path)"}
+        for p in sorted(set(cfg.top_p) | {args.top_p} | set(extension)):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             svg2.svg2_select(cq, ck, cnt_k, p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
             svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
@@ -375,6 +379,8 @@ def main():
                              "attn_ms": a_ms, "attn_tflops_actual": flops / (a_ms * 1e-3) / 1e12,
                              "attn_tflops_effective": dense_flops / (a_ms * 1e-3) / 1e12,
                              "layer_ms": kmeans_ms + ev[0].elapsed_time(ev[1]) + stage_ms["permute"] + a_ms}
+            if p in extension and p not in set(cfg.top_p) | {args.top_p}:
+                sweep[str(p)]["note"] = extension[p]
         svg2.raise_on_device_error(ws)
 
     # HBM stages against the measured copy bandwidth: the three row gathers (permutation) as timed
@@ -462,7 +468,8 @@ def main():
         "layer_tflops_effective": dense_flops / (ms_per_step * 1e-3) / 1e12,
         "executed_over_actual": executed_flops / actual_flops, "fixed128_padding_waste": waste128,
         "hbm_stages": hbm_stages,
-        "dense_sdpa_ms": dense_ms, "dense_svg2_dense_attn": own_dense, "denoise_driver": denoise, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
+        "dense_sdpa_ms": dense_ms, "dense_sdpa_backends_enabled": sdpa_backends(torch) if dense_ms is not None else None,
+        "dense_svg2_dense_attn": own_dense, "denoise_driver": denoise, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
         "top_p_sweep": sweep,
     }
     print(json.dumps(line), flush=True)
@@ -590,6 +597,14 @@ def measure_warm(svg2, torch, cfg, args, dev, Q0, K0, V0, ws, scale):
                       "kmeans_ms_cold": med(out["kmeans_ms_cold"]),
                       "kmeans_speedup": med(out["kmeans_ms_cold"]) / med(out["kmeans_ms_warm"])}
     return out
+
+
+def sdpa_backends(torch):
+    """The scaled_dot_product_attention backends torch has enabled (it picks among them per call)."""
+    b = torch.backends.cuda
+    names = {"flash": b.flash_sdp_enabled, "cudnn": getattr(b, "cudnn_sdp_enabled", None),
+             "mem_efficient": b.mem_efficient_sdp_enabled, "math": b.math_sdp_enabled}
+    return [n for n, f in names.items() if f is not None and f()]
 
 
 def time_dense(torch, Q, K, V, scale, reps=3):
