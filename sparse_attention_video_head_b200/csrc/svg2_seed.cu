@@ -12,16 +12,19 @@
 //     column 0, K = 128), giving x . c in TMEM;
 //   * the epilogue forms f = ||x||^2 + ||c||^2 - 2 x.c and lists the candidates where f, widened by
 //     a rigorous error bound, does not rule out an improvement; after the stream the whole CTA
-//     computes their exact float64 D^2 (a sequential sum over the 128 coordinates, the reference's
+//     computes their exact float64 D^2 (a sequential sum over the 128 coordinates, the definition's
 //     order, one candidate per thread) and the exact value decides;
 //   * a tile is skipped without being fetched when no candidate in it can move closer: with a the
-//     candidate's nearest seed, ||c_new - c_a||^2 >= 4 D^2 proves ||x - c_new|| >= ||x - c_a||;
-//   * late in the seeding that test leaves few candidates; when a CTA has at most two rounds of its
+//     candidate's nearest seed, ||c_new - c_a||^2 >= 4 D^2 proves ||x - c_new|| >= ||x - c_a||; the
+//     table of ||c_new - c_a||^2 is built from the earlier seeds' bf16 rows, which a bulk copy brings
+//     into the (then idle) TMA ring while the pick is made;
+//   * late in the seeding that test leaves few candidates; when a CTA has at most four rounds of its
 //     threads' worth, the pass skips the stream and computes their exact D^2 directly.
 //
 // Per-tile sums of the fixed-point weights make the sampling search a scan over the tiles, then a
-// scan over one tile.  The D^2 values, and so the seeds, are the same as those of the sequential
-// float64 definition.
+// scan over one tile: the CTA totals meet at a cluster barrier, and the CTA that owns the pick sends
+// it to every CTA of the cluster as an 8-byte message on an mbarrier.  The D^2 values, and so the
+// seeds, are the same as those of the sequential float64 definition.
 #include "svg2_internal.h"
 #include "svg2_device.cuh"
 
