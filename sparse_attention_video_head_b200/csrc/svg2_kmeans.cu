@@ -1334,7 +1334,8 @@ cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k
                                                           cap, st);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    rerank_kernel<<<2 * sms, kRrThreads, 0, s>>>(static_cast<const uint16_t*>(X), N, k, centroids, rr_list, rr_count,
+    // eight CTAs of 8 warps per SM: each warp waits on its token's rows, so many warps in flight
+    rerank_kernel<<<8 * sms, kRrThreads, 0, s>>>(static_cast<const uint16_t*>(X), N, k, centroids, rr_list, rr_count,
                                                  cap, labels);
     return cudaGetLastError();
   }
