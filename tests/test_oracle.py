@@ -326,3 +326,65 @@ def test_density_of_full_mask_is_one(oracle):
     count_k = np.array([2, 6], np.int32)
     assert oracle.density(np.ones((3, 2), np.uint8), count_q, count_k) == 1.0
     assert oracle.density(np.array([[1, 0], [1, 1], [0, 1]], np.uint8), count_q, count_k) == (3 * 2 + 5 * 6) / 64
+
+
+# ---------------------------------------------------------------- composition helpers
+
+def test_strided_seeding_draws_only_every_stride_th_token(oracle):
+    """seed_tokens caps the k-means++ candidates at every s-th token, s = ceil(N / seed_tokens)."""
+    assert oracle.seed_stride(75600, 16384) == 5
+    assert oracle.seed_stride(16384, 16384) == 1
+    assert oracle.seed_stride(16385, 16384) == 2
+    assert oracle.seed_stride(1000, 0) == 1
+    X, _ = _mixture(1003, 6, 12, 0.3, 21)
+    u = np.random.default_rng(22).random(12)
+    s = oracle.seed_stride(X.shape[0], 100)
+    assert s == 11
+    seeds, C0 = oracle.kmeanspp(np.ascontiguousarray(X[::s]), 12, u)
+    # the first seed is candidate floor(u0 * S) of the S = ceil(N / s) candidates, i.e. token s * that
+    assert seeds[0] == int(np.floor(u[0] * (-(-1003 // s))))
+    C, labels, counts = oracle.kmeans(X, 12, 4, u, seed_tokens=100)
+    Cl, ll, cl = oracle.lloyd(X, C0, 4)
+    np.testing.assert_array_equal(C, Cl)
+    np.testing.assert_array_equal(labels, ll)
+    # every seed is a row of X at a multiple of the stride
+    rows = {tuple(r) for r in X[::s].astype(np.float64)}
+    assert all(tuple(c) in rows for c in C0)
+
+
+def test_layer_rows_equal_the_full_layer_at_those_rows(oracle):
+    cfg = I.CONFIGS["tiny"]
+    hi = I.head_inputs(cfg, 0, 0)
+    q, k, v = hi["q"][:1500], hi["k"][:1500], hi["v"][:1500]
+    args = (q, k, v, 8, 16, 3, 0.7, cfg.scale, hi["uq"][:8], hi["uk"][:16])
+    full = oracle.layer_head(*args)
+    rows = np.array([0, 1, 17, 700, 1499])
+    part = oracle.layer_head(*args, rows=rows)
+    assert not full["mask"].all()                         # a real selection, not every pair
+    np.testing.assert_array_equal(part["o_rows"], full["o"][rows])
+
+
+def test_oracle_results_do_not_depend_on_the_thread_count(oracle, tmp_path):
+    """OpenMP only splits independent rows, so one thread and many give identical bits."""
+    import subprocess
+    import sys
+    script = tmp_path / "run.py"
+    script.write_text(
+        "import sys, numpy as np\n"
+        f"sys.path.insert(0, {repr(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))})\n"
+        "from oracle import oracle as O\n"
+        "from sparse_attention_video_head_b200 import inputs as I\n"
+        "cfg = I.CONFIGS['tiny']\n"
+        "hi = I.head_inputs(cfg, 0, 0)\n"
+        "out = O.layer_head(hi['q'][:2000], hi['k'][:2000], hi['v'][:2000], 8, 16, 3, 0.9, cfg.scale,\n"
+        "                   hi['uq'][:8], hi['uk'][:16])\n"
+        "np.savez(sys.argv[1], **out)\n")
+    outs = []
+    for threads in ("1", "4"):
+        path = tmp_path / f"out{threads}.npz"
+        env = {**os.environ, "OMP_NUM_THREADS": threads}
+        subprocess.check_call([sys.executable, str(script), str(path)], env=env, timeout=300)
+        outs.append(np.load(path))
+    assert set(outs[0].files) == set(outs[1].files)
+    for key in outs[0].files:
+        np.testing.assert_array_equal(outs[0][key], outs[1][key])
