@@ -3,6 +3,8 @@
 Every function here has the name of the C entry point it calls.  PyTorch supplies device memory
 and the current CUDA stream; all of the method's steps run in the library's sm_100a kernels.
 There is no fallback: if libsvg2.so is missing or a call fails, an exception is raised.
+The library sees only pointers, so each wrapper checks its tensors' dtypes and element counts
+against the sizes of the call (include/svg2.h) before it takes their pointers.
 """
 from __future__ import annotations
 
@@ -125,6 +127,36 @@ def _hp(t: torch.Tensor):
     return ctypes.c_void_p(t.data_ptr())
 
 
+_BF16, _F32, _F64, _I32, _U8 = (torch.bfloat16,), (torch.float32,), (torch.float64,), (torch.int32,), (torch.uint8,)
+_DATA = (torch.bfloat16, torch.float32)
+
+
+def _arg(t: Optional[torch.Tensor], name: str, dtypes, numel: int, optional: bool = False, host: bool = False):
+    """Pointer of a tensor argument after checking it against the header's contract: its dtype and
+    room for the `numel` elements the library reads or writes through it.  The library sees only a
+    pointer, so a smaller buffer would be read or written past its end on the device; these checks
+    run before the pointer is taken."""
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(x) for x in dtypes)}")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, the call uses {numel}")
+    return _hp(t) if host else _p(t)
+
+
+def _dims(t: torch.Tensor, name: str, ndim: int = 4):
+    if t is None or t.dim() != ndim:
+        raise ValueError(f"{name} must be a {ndim}-D tensor")
+    return tuple(int(x) for x in t.shape)
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
 def _stream(stream: Optional[torch.cuda.Stream] = None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -166,68 +198,105 @@ def raise_on_device_error(ws: torch.Tensor, stream=None):
 
 def svg2_kmeanspp(X: torch.Tensor, k: int, u: torch.Tensor, centroids: torch.Tensor, ws: torch.Tensor,
                   seed_tokens: int = DEFAULT_SEED_TOKENS, stream=None):
-    B, H, N, d = X.shape
-    _check(lib().svg2_kmeanspp(_p(X), _dtype(X), B, H, N, d, k, _p(u), int(seed_tokens), _p(centroids), _p(ws),
-                               ws.numel(), _stream(stream)), "svg2_kmeanspp")
+    B, H, N, d = _dims(X, "X")
+    BH = B * H
+    _check(lib().svg2_kmeanspp(_arg(X, "X", _DATA, 0), _dtype(X), B, H, N, d, k, _arg(u, "u", _F64, BH * k),
+                               int(seed_tokens), _arg(centroids, "centroids", _F32, BH * k * d), _p(ws),
+                               _nbytes(ws), _stream(stream)), "svg2_kmeanspp")
 
 
 def svg2_kmeans(X: torch.Tensor, k: int, iters: int, init: int, centroids: torch.Tensor, labels: torch.Tensor,
                 counts: torch.Tensor, ws: torch.Tensor, u: Optional[torch.Tensor] = None,
                 perm: Optional[torch.Tensor] = None, offsets: Optional[torch.Tensor] = None,
                 seed_tokens: int = DEFAULT_SEED_TOKENS, stream=None):
-    B, H, N, d = X.shape
-    _check(lib().svg2_kmeans(_p(X), _dtype(X), B, H, N, d, k, iters, init, _p(u), int(seed_tokens), _p(centroids),
-                             _p(labels),
-                             _p(counts), _p(perm), _p(offsets), _p(ws), ws.numel(), _stream(stream)), "svg2_kmeans")
+    B, H, N, d = _dims(X, "X")
+    BH = B * H
+    u_ptr = _arg(u, "u", _F64, BH * k) if init == SVG2_INIT_KMEANSPP else _p(u)
+    _check(lib().svg2_kmeans(_arg(X, "X", _DATA, 0), _dtype(X), B, H, N, d, k, iters, init, u_ptr, int(seed_tokens),
+                             _arg(centroids, "centroids", _F32, BH * k * d), _arg(labels, "labels", _I32, BH * N),
+                             _arg(counts, "counts", _I32, BH * k), _arg(perm, "perm", _I32, BH * N, optional=True),
+                             _arg(offsets, "offsets", _I32, BH * (k + 1), optional=True), _p(ws), _nbytes(ws),
+                             _stream(stream)), "svg2_kmeans")
 
 
 def svg2_select(cq: torch.Tensor, ck: torch.Tensor, count_k: torch.Tensor, top_p: float, scale: float,
                 mask: torch.Tensor, sel_count: torch.Tensor, sel_idx: torch.Tensor, ws: torch.Tensor,
                 weights: Optional[torch.Tensor] = None, stream_len: Optional[torch.Tensor] = None, stream=None):
-    B, H, nQ, d = cq.shape
-    nK = ck.shape[2]
-    _check(lib().svg2_select(_p(cq), _p(ck), _p(count_k), B, H, nQ, nK, d, float(top_p), float(scale), _p(weights),
-                             _p(mask), _p(sel_count), _p(sel_idx), _p(stream_len), _p(ws), ws.numel(),
+    B, H, nQ, d = _dims(cq, "cq")
+    nK = _dims(ck, "ck")[2]
+    BH = B * H
+    _check(lib().svg2_select(_arg(cq, "cq", _F32, 0), _arg(ck, "ck", _F32, BH * nK * d),
+                             _arg(count_k, "count_k", _I32, BH * nK), B, H, nQ, nK, d, float(top_p), float(scale),
+                             _arg(weights, "weights", _F32, BH * nQ * nK, optional=True),
+                             _arg(mask, "mask", _U8, BH * nQ * nK), _arg(sel_count, "sel_count", _I32, BH * nQ),
+                             _arg(sel_idx, "sel_idx", _I32, BH * nQ * nK),
+                             _arg(stream_len, "stream_len", _I32, BH * nQ, optional=True), _p(ws), _nbytes(ws),
                              _stream(stream)), "svg2_select")
 
 
 def svg2_select_from_weights(weights: torch.Tensor, count_k: torch.Tensor, top_p: float, mask: torch.Tensor,
                              sel_count: torch.Tensor, sel_idx: torch.Tensor, ws: torch.Tensor,
                              stream_len: Optional[torch.Tensor] = None, stream=None):
-    B, H, nQ, nK = weights.shape
-    _check(lib().svg2_select_from_weights(_p(weights), _p(count_k), B, H, nQ, nK, float(top_p), _p(mask),
-                                          _p(sel_count), _p(sel_idx), _p(stream_len), _p(ws), ws.numel(),
-                                          _stream(stream)), "svg2_select_from_weights")
+    B, H, nQ, nK = _dims(weights, "weights")
+    BH = B * H
+    _check(lib().svg2_select_from_weights(_arg(weights, "weights", _F32, 0), _arg(count_k, "count_k", _I32, BH * nK),
+                                          B, H, nQ, nK, float(top_p), _arg(mask, "mask", _U8, BH * nQ * nK),
+                                          _arg(sel_count, "sel_count", _I32, BH * nQ),
+                                          _arg(sel_idx, "sel_idx", _I32, BH * nQ * nK),
+                                          _arg(stream_len, "stream_len", _I32, BH * nQ, optional=True), _p(ws),
+                                          _nbytes(ws), _stream(stream)), "svg2_select_from_weights")
 
 
 def svg2_sort(labels: torch.Tensor, k: int, perm: torch.Tensor, offsets: torch.Tensor, counts: Optional[torch.Tensor],
               ws: torch.Tensor, stream=None):
-    B, H, N = labels.shape
-    _check(lib().svg2_sort(_p(labels), B, H, N, k, _p(perm), _p(offsets), _p(counts), _p(ws), ws.numel(),
+    B, H, N = _dims(labels, "labels", 3)
+    BH = B * H
+    _check(lib().svg2_sort(_arg(labels, "labels", _I32, 0), B, H, N, k, _arg(perm, "perm", _I32, BH * N),
+                           _arg(offsets, "offsets", _I32, BH * (k + 1)),
+                           _arg(counts, "counts", _I32, BH * k, optional=True), _p(ws), _nbytes(ws),
                            _stream(stream)), "svg2_sort")
 
 
 def svg2_gather(X: torch.Tensor, perm: torch.Tensor, Xp: torch.Tensor, stream=None):
-    B, H, N, d = X.shape
-    _check(lib().svg2_gather(_p(X), _dtype(X), _p(perm), B, H, N, d, _p(Xp), _stream(stream)), "svg2_gather")
+    B, H, N, d = _dims(X, "X")
+    BH = B * H
+    _check(lib().svg2_gather(_arg(X, "X", _DATA, 0), _dtype(X), _arg(perm, "perm", _I32, BH * N), B, H, N, d,
+                             _arg(Xp, "Xp", _BF16, BH * N * d), _stream(stream)), "svg2_gather")
 
 
 def svg2_permute(X: torch.Tensor, labels: torch.Tensor, k: int, Xp: torch.Tensor, perm: torch.Tensor,
                  offsets: torch.Tensor, counts: Optional[torch.Tensor], ws: torch.Tensor, stream=None):
-    B, H, N, d = X.shape
-    _check(lib().svg2_permute(_p(X), _dtype(X), _p(labels), B, H, N, d, k, _p(Xp), _p(perm), _p(offsets),
-                              _p(counts), _p(ws), ws.numel(), _stream(stream)), "svg2_permute")
+    B, H, N, d = _dims(X, "X")
+    BH = B * H
+    _check(lib().svg2_permute(_arg(X, "X", _DATA, 0), _dtype(X), _arg(labels, "labels", _I32, BH * N), B, H, N, d, k,
+                              _arg(Xp, "Xp", _BF16, BH * N * d), _arg(perm, "perm", _I32, BH * N),
+                              _arg(offsets, "offsets", _I32, BH * (k + 1)),
+                              _arg(counts, "counts", _I32, BH * k, optional=True), _p(ws), _nbytes(ws),
+                              _stream(stream)), "svg2_permute")
+
+
+def _attn_args(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, O, perm_q):
+    """Sizes and checked pointers (Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, O, perm_q) of an
+    attention call; nQ and nK come from the offsets' last dimension."""
+    B, H, N, d = _dims(Qp, "Qp")
+    if q_off is None or k_off is None or q_off.dim() < 1 or k_off.dim() < 1:
+        raise ValueError("q_off and k_off are required")
+    BH = B * H
+    nQ = int(q_off.shape[-1]) - 1
+    nK = int(k_off.shape[-1]) - 1
+    ptr = (_arg(Qp, "Qp", _BF16, 0), _arg(Kp, "Kp", _BF16, BH * N * d), _arg(Vp, "Vp", _BF16, BH * N * d),
+           _arg(q_off, "q_off", _I32, BH * (nQ + 1)), _arg(k_off, "k_off", _I32, BH * (nK + 1)),
+           _arg(sel_count, "sel_count", _I32, BH * nQ), _arg(sel_idx, "sel_idx", _I32, BH * nQ * nK),
+           _arg(O, "O", _BF16, BH * N * d), _arg(perm_q, "perm_q", _I32, BH * N, optional=True))
+    return B, H, N, d, nQ, nK, ptr
 
 
 def svg2_sparse_attn(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off: torch.Tensor, k_off: torch.Tensor,
                      sel_count: torch.Tensor, sel_idx: torch.Tensor, scale: float, O: torch.Tensor, ws: torch.Tensor,
                      perm_q: Optional[torch.Tensor] = None, stream=None):
-    B, H, N, d = Qp.shape
-    nQ = q_off.shape[-1] - 1
-    nK = k_off.shape[-1] - 1
-    _check(lib().svg2_sparse_attn(_p(Qp), _p(Kp), _p(Vp), _p(q_off), _p(k_off), _p(sel_count), _p(sel_idx), B, H, N,
-                                  d, nQ, nK, float(scale), _p(perm_q), _p(O), _p(ws), ws.numel(), _stream(stream)),
-           "svg2_sparse_attn")
+    B, H, N, d, nQ, nK, ptr = _attn_args(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, O, perm_q)
+    _check(lib().svg2_sparse_attn(*ptr[:7], B, H, N, d, nQ, nK, float(scale), ptr[8], ptr[7], _p(ws), _nbytes(ws),
+                                  _stream(stream)), "svg2_sparse_attn")
 
 
 def svg2_dense_attn_workspace_size(B: int, H: int, N: int, d: int) -> int:
@@ -243,9 +312,11 @@ def dense_workspace(B: int, H: int, N: int, d: int, device=None) -> torch.Tensor
 
 def svg2_dense_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: float, O: torch.Tensor,
                     ws: torch.Tensor, stream=None):
-    B, H, N, d = Q.shape
-    _check(lib().svg2_dense_attn(_p(Q), _p(K), _p(V), B, H, N, d, float(scale), _p(O), _p(ws), ws.numel(),
-                                 _stream(stream)), "svg2_dense_attn")
+    B, H, N, d = _dims(Q, "Q")
+    n = B * H * N * d
+    _check(lib().svg2_dense_attn(_arg(Q, "Q", _BF16, 0), _arg(K, "K", _BF16, n), _arg(V, "V", _BF16, n), B, H, N, d,
+                                 float(scale), _arg(O, "O", _BF16, n), _p(ws), _nbytes(ws), _stream(stream)),
+           "svg2_dense_attn")
 
 
 def svg2_sparse_attn_noalloc(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off: torch.Tensor,
@@ -253,17 +324,17 @@ def svg2_sparse_attn_noalloc(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tenso
                              O: torch.Tensor, perm_q: Optional[torch.Tensor] = None,
                              device_status: Optional[torch.Tensor] = None, stream=None):
     """svg2_sparse_attn for callers that cannot allocate: scratch is the library's fixed array."""
-    B, H, N, d = Qp.shape
-    nQ = q_off.shape[-1] - 1
-    nK = k_off.shape[-1] - 1
-    _check(lib().svg2_sparse_attn_noalloc(_p(Qp), _p(Kp), _p(Vp), _p(q_off), _p(k_off), _p(sel_count), _p(sel_idx),
-                                          B, H, N, d, nQ, nK, float(scale), _p(perm_q), _p(O), _p(device_status),
-                                          _stream(stream)), "svg2_sparse_attn_noalloc")
+    B, H, N, d, nQ, nK, ptr = _attn_args(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, O, perm_q)
+    if device_status is not None and _nbytes(device_status) < 16:
+        raise ValueError("device_status: the status word takes 16 bytes")
+    _check(lib().svg2_sparse_attn_noalloc(*ptr[:7], B, H, N, d, nQ, nK, float(scale), ptr[8], ptr[7],
+                                          _p(device_status), _stream(stream)), "svg2_sparse_attn_noalloc")
 
 
 def svg2_unpermute(Op: torch.Tensor, perm: torch.Tensor, O: torch.Tensor, stream=None):
-    B, H, N, d = Op.shape
-    _check(lib().svg2_unpermute(_p(Op), _p(perm), B, H, N, d, _p(O), _stream(stream)), "svg2_unpermute")
+    B, H, N, d = _dims(Op, "Op")
+    _check(lib().svg2_unpermute(_arg(Op, "Op", _BF16, 0), _arg(perm, "perm", _I32, B * H * N), B, H, N, d,
+                                _arg(O, "O", _BF16, B * H * N * d), _stream(stream)), "svg2_unpermute")
 
 
 @dataclass
@@ -297,18 +368,42 @@ def layer_output_buffers(B: int, H: int, N: int, nQ: int, nK: int, device="cuda"
     }
 
 
+# dtype and element count per (b, h) of each svg2_layer_outputs field
+def _layer_out_sizes(N: int, nQ: int, nK: int):
+    return {"labels_q": (_I32, N), "labels_k": (_I32, N), "count_q": (_I32, nQ), "count_k": (_I32, nK),
+            "perm_q": (_I32, N), "perm_k": (_I32, N), "q_off": (_I32, nQ + 1), "k_off": (_I32, nK + 1),
+            "weights": (_F32, nQ * nK), "mask": (_U8, nQ * nK), "sel_count": (_I32, nQ),
+            "sel_idx": (_I32, nQ * nK), "stream_len": (_I32, nQ)}
+
+
+def _layer_args(Q, K, V, params: "LayerParams", cq, ck, uq, uk, host: bool = False):
+    """Sizes and checked pointers (Q, K, V, uq, uk, cq, ck) of a layer call; Q, K, V are host tensors
+    when `host` is set (svg2_layer_host), everything else is on the device."""
+    B, H, N, d = _dims(Q, "Q")
+    BH = B * H
+    n = BH * N * d
+    cold = params.init == SVG2_INIT_KMEANSPP
+    ptr = (_arg(Q, "Q", _DATA, 0, host=host), _arg(K, "K", (Q.dtype,), n, host=host),
+           _arg(V, "V", (Q.dtype,), n, host=host),
+           _arg(uq, "uq", _F64, BH * params.nQ) if cold else _p(uq),
+           _arg(uk, "uk", _F64, BH * params.nK) if cold else _p(uk),
+           _arg(cq, "cq", _F32, BH * params.nQ * d), _arg(ck, "ck", _F32, BH * params.nK * d))
+    return B, H, N, d, ptr
+
+
 def svg2_layer(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, params: LayerParams, cq: torch.Tensor,
                ck: torch.Tensor, O: torch.Tensor, ws: torch.Tensor, uq: Optional[torch.Tensor] = None,
                uk: Optional[torch.Tensor] = None, outs: Optional[Dict[str, torch.Tensor]] = None, stream=None):
-    B, H, N, d = Q.shape
+    B, H, N, d, ptr = _layer_args(Q, K, V, params, cq, ck, uq, uk)
     prm = params.c()
     c_outs = None
     if outs is not None:
-        c_outs = SvgLayerOutputs(*[(_p(outs[n]).value if outs.get(n) is not None else None)
-                                   for n, _ in SvgLayerOutputs._fields_])
-    _check(lib().svg2_layer(_p(Q), _p(K), _p(V), _dtype(Q), B, H, N, d, ctypes.byref(prm), _p(uq), _p(uk), _p(cq),
-                            _p(ck), _p(O), ctypes.byref(c_outs) if c_outs is not None else None, _p(ws), ws.numel(),
-                            _stream(stream)), "svg2_layer")
+        sizes = _layer_out_sizes(N, params.nQ, params.nK)
+        c_outs = SvgLayerOutputs(*[(_arg(outs[n], n, sizes[n][0], B * H * sizes[n][1]).value
+                                    if outs.get(n) is not None else None) for n, _ in SvgLayerOutputs._fields_])
+    _check(lib().svg2_layer(*ptr[:3], _dtype(Q), B, H, N, d, ctypes.byref(prm), *ptr[3:],
+                            _arg(O, "O", _BF16, B * H * N * d), ctypes.byref(c_outs) if c_outs is not None else None,
+                            _p(ws), _nbytes(ws), _stream(stream)), "svg2_layer")
 
 
 def svg2_layer_host(Qh: torch.Tensor, Kh: torch.Tensor, Vh: torch.Tensor, Oh: torch.Tensor, Q: torch.Tensor,
@@ -317,12 +412,14 @@ def svg2_layer_host(Qh: torch.Tensor, Kh: torch.Tensor, Vh: torch.Tensor, Oh: to
                     uk: Optional[torch.Tensor] = None, heads_per_group: int = 0, stream=None, copy_stream=None):
     """The layer with Q, K, V and O in (page-locked) host memory; Q, K, V, O here are the device
     staging buffers.  Copies run on copy_stream, overlapped with the compute of other head groups."""
-    B, H, N, d = Qh.shape
+    B, H, N, d, ptr = _layer_args(Qh, Kh, Vh, params, cq, ck, uq, uk, host=True)
+    n = B * H * N * d
     prm = params.c()
     cs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
-    _check(lib().svg2_layer_host(_hp(Qh), _hp(Kh), _hp(Vh), _hp(Oh), _p(Q), _p(K), _p(V), _p(O), _dtype(Qh), B, H, N, d,
-                                 ctypes.byref(prm), _p(uq), _p(uk), _p(cq), _p(ck), int(heads_per_group), _p(ws),
-                                 ws.numel(), _stream(stream), cs), "svg2_layer_host")
+    _check(lib().svg2_layer_host(*ptr[:3], _arg(Oh, "Oh", _BF16, n, host=True), _arg(Q, "Q", (Qh.dtype,), n),
+                                 _arg(K, "K", (Qh.dtype,), n), _arg(V, "V", (Qh.dtype,), n), _arg(O, "O", _BF16, n),
+                                 _dtype(Qh), B, H, N, d, ctypes.byref(prm), *ptr[3:], int(heads_per_group), _p(ws),
+                                 _nbytes(ws), _stream(stream), cs), "svg2_layer_host")
 
 
 SVG2_STEP_DENSE, SVG2_STEP_COLD, SVG2_STEP_WARM = 0, 1, 2
@@ -339,6 +436,7 @@ class Driver:
         cfg = SvgDriverConfig(num_steps, num_layers, dense_steps, warm_iters, params.c())
         _check(lib().svg2_driver_create(ctypes.byref(cfg), B, H, N, d, ctypes.byref(self._h)), "svg2_driver_create")
         self.shape = (B, H, N, d)
+        self.nQ, self.nK = params.nQ, params.nK
         self.cache = self.ws = None
         if allocate:
             self.cache = torch.zeros(self.cache_bytes() // 4, dtype=torch.float32, device=device)
@@ -365,8 +463,14 @@ class Driver:
 
     def layer(self, step: int, layer: int, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
               uq: Optional[torch.Tensor] = None, uk: Optional[torch.Tensor] = None, stream=None):
-        _check(lib().svg2_driver_layer(self._h, step, layer, _p(Q), _p(K), _p(V), _p(uq), _p(uk), _p(O), _p(self.ws),
-                                       self.ws.numel(), _stream(stream)), "svg2_driver_layer")
+        if self.ws is None:
+            raise ValueError("this driver was created without a workspace (allocate=False)")
+        B, H, N, d = self.shape
+        n = B * H * N * d
+        _check(lib().svg2_driver_layer(self._h, step, layer, _arg(Q, "Q", _BF16, n), _arg(K, "K", _BF16, n),
+                                       _arg(V, "V", _BF16, n), _arg(uq, "uq", _F64, B * H * self.nQ, optional=True),
+                                       _arg(uk, "uk", _F64, B * H * self.nK, optional=True), _arg(O, "O", _BF16, n),
+                                       _p(self.ws), _nbytes(self.ws), _stream(stream)), "svg2_driver_layer")
 
     def close(self):
         if self._h:
@@ -381,9 +485,10 @@ class Driver:
 
 
 def svg2_selftest_mma(A: torch.Tensor, Bm: torch.Tensor, V: torch.Tensor, ws: torch.Tensor, stream=None):
-    n = Bm.shape[0]
+    n = _dims(Bm, "Bm", 2)[0]
     C = torch.empty(128, n, dtype=torch.float32, device=A.device)
     O = torch.empty(128, 128, dtype=torch.float32, device=A.device)
-    _check(lib().svg2_selftest_mma(_p(A), _p(Bm), n, _p(V), _p(C), _p(O), _p(ws), ws.numel(), _stream(stream)),
+    _check(lib().svg2_selftest_mma(_arg(A, "A", _BF16, 128 * 128), _arg(Bm, "Bm", _BF16, n * 128), n,
+                                   _arg(V, "V", _BF16, 128 * 128), _p(C), _p(O), _p(ws), _nbytes(ws), _stream(stream)),
            "svg2_selftest_mma")
     return C, O
