@@ -42,6 +42,8 @@ int check_sizes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1) return SVG2_ERR_INVALID_ARG;
   if (N > SVG2_MAX_TOKENS) return SVG2_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > (1 << 20)) return SVG2_ERR_UNSUPPORTED;
+  // token rows across all planes are indexed (and addressed by TMA) with 32-bit integers
+  if (static_cast<long long>(B) * H * N >= (1LL << 31)) return SVG2_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return SVG2_ERR_UNSUPPORTED;
   return SVG2_OK;
 }
