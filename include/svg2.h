@@ -21,8 +21,9 @@
  *     a failed launch returns SVG2_ERR_CUDA.  Device-side errors (a bounded wait that ran out,
  *     an out-of-range label) are latched in a status word at the start of `ws` and read with
  *     svg2_check_status.  No kernel traps or waits without a bound.
- *   - The library keeps no global state, is reentrant, and never lets a C++ exception cross the
- *     C boundary.  Return values are svg2_status codes.
+ *   - The library keeps no global state (the one exception is the fixed scratch array of
+ *     svg2_sparse_attn_noalloc, described there), is reentrant, and never lets a C++ exception
+ *     cross the C boundary.  Return values are svg2_status codes.
  */
 #ifndef SVG2_H_
 #define SVG2_H_
@@ -43,7 +44,7 @@ extern "C" {
 typedef enum {
   SVG2_OK = 0,
   SVG2_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, bad enum value */
-  SVG2_ERR_UNSUPPORTED = 2,   /* d / dtype / cluster count this build does not handle */
+  SVG2_ERR_UNSUPPORTED = 2,   /* d / dtype / sizes beyond the library's limits */
   SVG2_ERR_WORKSPACE = 3,     /* ws too small or misaligned */
   SVG2_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
   SVG2_ERR_DEVICE_TIMEOUT = 5,/* a bounded device wait ran out (read via svg2_check_status) */
@@ -62,7 +63,7 @@ typedef enum { SVG2_INIT_GIVEN = 0, SVG2_INIT_KMEANSPP = 1 } svg2_init;
  * This default keeps the seeding cheap on video-length layers. */
 #define SVG2_DEFAULT_SEED_TOKENS 16384
 
-/* Largest supported sizes of this build.  Besides these, B*H <= 2^20 and B*H*N < 2^31 (token rows
+/* Largest sizes the library supports.  Besides these, B*H <= 2^20 and B*H*N < 2^31 (token rows
  * across all planes are indexed with 32-bit integers); larger sizes return SVG2_ERR_UNSUPPORTED. */
 #define SVG2_MAX_CLUSTERS 1024
 #define SVG2_MAX_TOKENS (1 << 24)

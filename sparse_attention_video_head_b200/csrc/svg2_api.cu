@@ -155,7 +155,7 @@ const char* svg2_status_string(int status) {
   switch (status) {
     case SVG2_OK: return "SVG2_OK";
     case SVG2_ERR_INVALID_ARG: return "SVG2_ERR_INVALID_ARG: invalid argument";
-    case SVG2_ERR_UNSUPPORTED: return "SVG2_ERR_UNSUPPORTED: size or type not supported by this build";
+    case SVG2_ERR_UNSUPPORTED: return "SVG2_ERR_UNSUPPORTED: size or type not supported by the library";
     case SVG2_ERR_WORKSPACE: return "SVG2_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case SVG2_ERR_CUDA: return "SVG2_ERR_CUDA: a CUDA call failed";
     case SVG2_ERR_DEVICE_TIMEOUT: return "SVG2_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
