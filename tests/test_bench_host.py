@@ -60,3 +60,15 @@ def test_config_record_for_both_modes():
     import dataclasses
     c2 = bench.config_dict(dataclasses.replace(cfg, H=20), 0.9, 16384, shard=(40, 2))
     assert c2["H"] == 40 and c2["parallelism"] == "heads/2"
+
+
+def test_traffic_constant_matches_its_profile_summary():
+    """The attention's DRAM traffic that bench.py reports comes from the ncu summary it names; the
+    constant and the summary's read and write rows must agree (to the summary's rounding)."""
+    import re
+    path = os.path.join(ROOT, bench.ATTN_TRAFFIC["summary"])
+    text = open(path).read()
+    rd = float(re.search(r"dram__bytes_read\.sum \| ([0-9.]+) MB", text).group(1)) * 1e6
+    wr = float(re.search(r"dram__bytes_write\.sum \| ([0-9.]+) MB", text).group(1)) * 1e6
+    assert abs(bench.ATTN_TRAFFIC["bytes_captured"] - (rd + wr)) <= 0.1e6
+    assert f"{bench.ATTN_TRAFFIC['heads_captured']} heads" in text
