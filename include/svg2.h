@@ -80,6 +80,21 @@ SVG2_API int svg2_workspace_size(int B, int H, int N, int d, int nQ, int nK, siz
  * NULL) receive a kernel tag and two integers for diagnostics. */
 SVG2_API int svg2_check_status(void* ws, void* stream, int* device_status, uint32_t* where, uint32_t* info);
 
+/* Diagnostics: sets, stream-ordered on `stream`, the budget in SM clock cycles of the bounded
+ * waits inside the tensor-core attention (svg2_sparse_attn, svg2_dense_attn, the layer calls) and
+ * the tensor-core k-means assignment that later calls make with this workspace.  0 restores the
+ * default (about 0.5 s at the boost clock); values above the default are clamped to it, so the
+ * setting can only make a wait give up sooner.  A wait that runs out latches
+ * SVG2_ERR_DEVICE_TIMEOUT (read with svg2_check_status); the kernel then stops issuing work, waits
+ * for its own copies and tensor-core operations already in flight, frees its tensor memory and
+ * exits, so later calls on the same workspace run normally.  The value lives in the status area
+ * at the start of `ws` (bytes 16..23), which, like the status word, must be zero when the
+ * workspace is first used (torch.zeros / cudaMemset); svg2_check_status does not clear it.  The
+ * k-means++ seeding keeps the default budget whatever this says.  No counterpart on the pages:
+ * it exists so that the give-up path of those waits can be tested.
+ *   ws      256-byte aligned workspace; returns SVG2_ERR_INVALID_ARG if NULL or misaligned. */
+SVG2_API int svg2_set_wait_budget(void* ws, uint64_t cycles, void* stream);
+
 /*
  * Batched k-means (Method (1); Key claims section 4.1 and 4.3) on X [B, H, N, d] per (b, h):
  * `iters` >= 1 Lloyd iterations — assignment label_t = argmin_c ||x_t - c||^2 (ties to the lower

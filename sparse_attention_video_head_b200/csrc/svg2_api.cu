@@ -106,11 +106,20 @@ cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int
     e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, s.c_hi, seed_tokens, st, stream);
   if (e == cudaSuccess) e = launch_centroid_prep(C, BH, k, d, s.c_hi, s.c_lo, s.c_norm, stream);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-    e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, s.rr_list, s.rr_count, st, stream);
+    e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, s.rr_list, s.rr_count, st,
+                      wait_budget_of(st), stream);
     if (e == cudaSuccess) e = launch_sort(labels, BH, N, k, perm, offsets, counts, s.chunk_hist, st, stream);
     if (e == cudaSuccess) e = launch_update(X, f32, BH, N, d, k, perm, offsets, C, s.c_hi, s.c_lo, s.c_norm, stream);
   }
   return e;
+}
+
+// Stream-ordered store of one 64-bit value into device memory (the status area's wait budget).
+__global__ void store_u64_kernel(uint64_t* dst, uint64_t v) { *dst = v; }
+
+cudaError_t launch_store_u64(uint64_t* dst, uint64_t v, cudaStream_t s) {
+  store_u64_kernel<<<1, 1, 0, s>>>(dst, v);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -193,6 +202,13 @@ int svg2_check_status(void* ws, void* stream, int* device_status, uint32_t* wher
     info[1] = h.info1;
   }
   return SVG2_OK;
+}
+
+int svg2_set_wait_budget(void* ws, uint64_t cycles, void* stream) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SVG2_ERR_INVALID_ARG;
+  const cudaError_t e = launch_store_u64(reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kWaitBudgetOffset),
+                                         cycles, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SVG2_OK : SVG2_ERR_CUDA;
 }
 
 int svg2_kmeanspp(const void* X, int dtype, int B, int H, int N, int d, int k, const double* u, int seed_tokens,
@@ -354,7 +370,7 @@ int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32
     r = check_ws(ws, ws_bytes, c.off);
     if (r != SVG2_OK) return r;
     return to_status(launch_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, BH, N, d, nQ, nK, scale, perm_q,
-                                        O, a, st, static_cast<cudaStream_t>(stream)));
+                                        O, a, st, wait_budget_of(st), static_cast<cudaStream_t>(stream)));
   } catch (...) {
     return SVG2_ERR_CUDA;
   }
@@ -405,7 +421,7 @@ int svg2_dense_attn(const void* Q, const void* K, const void* V, int B, int H, i
     cudaError_t e = launch_dense_plan(BH, N, D.q_off, D.k_off, D.sel_count, D.sel_idx, s);
     if (e == cudaSuccess)
       e = launch_sparse_attn(Q, K, V, D.q_off, D.k_off, D.sel_count, D.sel_idx, BH, N, d, 1, 1, scale, nullptr, O,
-                             D.attn, D.st, s);
+                             D.attn, D.st, wait_budget_of(D.st), s);
     return to_status(e);
   } catch (...) {
     return SVG2_ERR_CUDA;
@@ -476,10 +492,10 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
     if (e == cudaSuccess) {
       if (p->fuse_unpermute) {
         e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
-                               p->scale, L.perm_q, O, L.attn, L.st, s);
+                               p->scale, L.perm_q, O, L.attn, L.st, wait_budget_of(L.st), s);
       } else {
         e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
-                               p->scale, nullptr, L.Op, L.attn, L.st, s);
+                               p->scale, nullptr, L.Op, L.attn, L.st, wait_budget_of(L.st), s);
         if (e == cudaSuccess) e = launch_unpermute(L.Op, L.perm_q, BH, N, d, O, s);
       }
     }
@@ -626,7 +642,8 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
                              static_cast<const uint16_t*>(L.Vp) + h0 * plane_p, L.q_off + h0 * (p->nQ + 1),
                              L.k_off + h0 * (p->nK + 1), L.sel_count + h0 * p->nQ,
                              L.sel_idx + h0 * static_cast<size_t>(p->nQ) * p->nK, hn, N, d, p->nQ, p->nK, p->scale,
-                             L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st, s);
+                             L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st,
+                             wait_budget_of(L.st), s);
       ok(cudaEventRecord(o_out[g], s));
       ok(cudaStreamWaitEvent(cs, o_out[g], 0));
       ok(cudaMemcpyAsync(static_cast<char*>(Oh) + h0 * plane_out, static_cast<const char*>(Od) + h0 * plane_out,

@@ -112,10 +112,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_idx, int N, int nQ,
                        int nK, float scale, const int32_t* __restrict__ perm_q, __nv_bfloat16* __restrict__ O,
                        const AttnUnit* __restrict__ units, const int32_t* __restrict__ head_base, int BH,
-                       DeviceStatus* st) {
+                       DeviceStatus* st, const uint64_t* __restrict__ wait_budget) {
   const int total_units = head_base[BH];
   if (static_cast<int>(blockIdx.x) >= total_units) return;
   if (status_set(st)) return;
+  const long long wb = effective_wait_budget(wait_budget);
   const AttnUnit un = units[blockIdx.x];
 
   constexpr uint32_t kTile = tile_bytes<D>();
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tma_load_2d(qa + hf * 16384, &tm_q, hf * 64, y, qbar);
         if (has_b) tma_load_2d(qb + hf * 16384, &tm_q, hf * 64, y + 128, qbar);
       }
-      bool ok = mbar_wait(qbar, 0, st, kWhereAttnMma);
+      bool ok = mbar_wait(qbar, 0, st, kWhereAttnMma, wb);
       const uint32_t id_s = idesc_bf16_f32(128, 64, 0);
       const uint32_t id_o = idesc_bf16_f32(128, D, 1);
       const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int T = (L + 63) / 64;  // 64-key sub-tiles; S slots alternate, so S(k+1) and S(k+2)
                                     // are computed while the softmax of k runs
       if (ok && T > 0) {
-        ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma);
+        ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma, wb);
         if (ok) {
           fence_proxy_async_smem();  // the key rows were written by cp.async (generic proxy)
           tc_fence_after();
@@ -273,8 +274,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       for (int k = 0; k < T && ok; ++k) {
         const int h = k & 1, j = k >> 1, stage = j & 1;
-        ok = mbar_wait(smem_u32(&bars->p_full[0][h]), j & 1, st, kWhereAttnMma);
-        if (ok && h == 0) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma);
+        ok = mbar_wait(smem_u32(&bars->p_full[0][h]), j & 1, st, kWhereAttnMma, wb);
+        if (ok && h == 0) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma, wb);
         if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_after();
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int j2 = k2 >> 1, stage2 = j2 & 1;
         if (k2 < T) {
           if ((k2 & 1) == 0) {
-            ok = mbar_wait(smem_u32(&bars->k_full[stage2]), (j2 >> 1) & 1, st, kWhereAttnMma);
+            ok = mbar_wait(smem_u32(&bars->k_full[stage2]), (j2 >> 1) & 1, st, kWhereAttnMma, wb);
             if (!ok) break;
             fence_proxy_async_smem();
             tc_fence_after();
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           issue_s(0, k2);
         }
         if (has_b) {
-          ok = mbar_wait(smem_u32(&bars->p_full[1][h]), j & 1, st, kWhereAttnMma);
+          ok = mbar_wait(smem_u32(&bars->p_full[1][h]), j & 1, st, kWhereAttnMma, wb);
           if (!ok) break;
           tc_fence_after();
           issue_pv(1, k);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // K(j) may land as soon as the last S product of K(j-2) is done, V(j) once PV of V(j-2) is;
       // each lands asynchronously and counts itself on its full barrier
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->k_empty[stage]), ((j >> 1) - 1) & 1, st,
-                                                             kWhereAttnProducer)))
+                                                             kWhereAttnProducer, 128, wb)))
         break;
 #pragma unroll
       for (int it = 0; it < 32 / RPI; ++it) {
@@ -346,7 +347,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->v_empty[stage]), ((j >> 1) - 1) & 1, st,
-                                                             kWhereAttnProducer)))
+                                                             kWhereAttnProducer, 128, wb)))
         break;
 #pragma unroll
       for (int it = 0; it < 32 / RPI; ++it) {
@@ -378,7 +379,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int T = (L + 63) / 64;
       for (int k = 0; k < T; ++k) {
         const int h = k & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x][h]), (k >> 1) & 1, st, kWhereAttnSoftmax));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x][h]), (k >> 1) & 1, st, kWhereAttnSoftmax, wb));
         if (!ok) break;
         tc_fence_after();
         const uint32_t t_sk = t_s + h * 64;
@@ -411,7 +412,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (k > 0 && __any_sync(0xffffffffu, grow)) {
           // O must hold every PV product up to k-1 before it is rescaled; rows that keep their
           // max multiply by 1.
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->pv_done[x]), (k - 1) & 1, st, kWhereAttnSoftmax));
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->pv_done[x]), (k - 1) & 1, st, kWhereAttnSoftmax, wb));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x][h]));
       }
       if (ok && T > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0, st, kWhereAttnSoftmax));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0, st, kWhereAttnSoftmax, wb));
       if (ok) {
         tc_fence_after();
         const int prow = un.row0 + x * 128 + row;
@@ -635,7 +636,8 @@ cudaError_t launch_dense_plan(int BH, int N, int32_t* q_off, int32_t* k_off, int
 cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
                                const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int BH,
                                int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
-                               const AttnScratch& sc, DeviceStatus* st, cudaStream_t s) {
+                               const AttnScratch& sc, DeviceStatus* st, const uint64_t* wait_budget,
+                               cudaStream_t s) {
   plan_count_kernel<<<BH, 256, 0, s>>>(q_off, nQ, N, sc.head_units);
   plan_scan_kernel<<<1, 32, 0, s>>>(sc.head_units, BH, sc.head_base);
   plan_write_kernel<<<BH, 32, 0, s>>>(q_off, nQ, N, sc.head_base, sc.units);
@@ -650,13 +652,13 @@ cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, c
     if (e != cudaSuccess) return e;
     sparse_attn_kernel<128><<<static_cast<unsigned>(grid), kAttnThreads, attn_smem<128>(), s>>>(
         tq, static_cast<const __nv_bfloat16*>(Kp), static_cast<const __nv_bfloat16*>(Vp), k_off, sel_count, sel_idx,
-        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st);
+        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st, wait_budget);
   } else {
     e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<64>());
     if (e != cudaSuccess) return e;
     sparse_attn_kernel<64><<<static_cast<unsigned>(grid), kAttnThreads, attn_smem<64>(), s>>>(
         tq, static_cast<const __nv_bfloat16*>(Kp), static_cast<const __nv_bfloat16*>(Vp), k_off, sel_count, sel_idx,
-        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st);
+        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st, wait_budget);
   }
   return cudaGetLastError();
 }

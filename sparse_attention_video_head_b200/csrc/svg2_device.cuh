@@ -35,6 +35,14 @@ __device__ __forceinline__ bool status_set(const DeviceStatus* st) {
   return *reinterpret_cast<const volatile uint32_t*>(&st->code) != 0u;
 }
 
+// The budget of a kernel's bounded waits: the status area's wait-budget field when the launch
+// passes one (0 there selects the default; larger values are clamped to it), else the default.
+__device__ __forceinline__ long long effective_wait_budget(const uint64_t* field) {
+  if (field == nullptr) return kWaitBudgetCycles;
+  const uint64_t b = *reinterpret_cast<const volatile uint64_t*>(field);
+  return (b == 0 || b > static_cast<uint64_t>(kWaitBudgetCycles)) ? kWaitBudgetCycles : static_cast<long long>(b);
+}
+
 // ------------------------------------------------------------------------------------------------
 // Shared-memory addresses and mbarriers
 // ------------------------------------------------------------------------------------------------

@@ -21,6 +21,12 @@ constexpr uint32_t kStatusDeviceBounds = 6;   // == SVG2_ERR_DEVICE_BOUNDS
 // About 0.5 s at the B200's boost clock: far above any legitimate wait inside one tile step.
 constexpr long long kWaitBudgetCycles = 1000LL * 1000LL * 1000LL;
 
+// The status area (kStatusBytes at the start of a workspace) holds the DeviceStatus word at offset
+// 0 and, at this offset, a uint64 wait budget in clock cycles for the attention and assignment
+// kernels' bounded waits: 0 (the value of a zeroed workspace) means kWaitBudgetCycles, and a value
+// above kWaitBudgetCycles is clamped to it, so the field can only shorten a wait.
+constexpr size_t kWaitBudgetOffset = 16;
+
 // Kernel tags for DeviceStatus::where.
 enum : uint32_t {
   kWhereSort = 1,
@@ -38,6 +44,12 @@ enum : uint32_t {
 };
 
 constexpr int kStatusBytes = 256;
+static_assert(kWaitBudgetOffset >= sizeof(DeviceStatus) && kWaitBudgetOffset + 8 <= kStatusBytes, "status area");
+
+// The wait-budget field of the status area that starts at st (a workspace's first bytes).
+inline const uint64_t* wait_budget_of(const DeviceStatus* st) {
+  return reinterpret_cast<const uint64_t*>(reinterpret_cast<const char*>(st) + kWaitBudgetOffset);
+}
 constexpr int kSortChunks = 32;  // token chunks per (b,h) in the stable counting sort
 constexpr int kAssignTileM = 128;
 constexpr int kAssignChunkN = 128;  // centroids per MMA chunk
@@ -133,7 +145,8 @@ cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, u
                                  float* c_norm, cudaStream_t s);
 cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,
                           const uint16_t* c_hi, const uint16_t* c_lo, const float* c_norm, int32_t* labels,
-                          uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, cudaStream_t s);
+                          uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, const uint64_t* wait_budget,
+                          cudaStream_t s);
 cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
                           const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
                           float* c_norm, cudaStream_t s);
@@ -146,7 +159,8 @@ cudaError_t launch_select(const float* cq, const float* ck, const float* weights
 cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
                                const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int BH,
                                int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
-                               const AttnScratch& scratch, DeviceStatus* st, cudaStream_t s);
+                               const AttnScratch& scratch, DeviceStatus* st, const uint64_t* wait_budget,
+                               cudaStream_t s);
 
 cudaError_t launch_dense_plan(int BH, int N, int32_t* q_off, int32_t* k_off, int32_t* sel_count, int32_t* sel_idx,
                               cudaStream_t s);

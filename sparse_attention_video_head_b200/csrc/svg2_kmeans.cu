@@ -6,13 +6,17 @@
 //    A token is skipped when the triangle inequality proves the new seed cannot be closer
 //    (||c_new - c_near||^2 >= 4.0001 D^2), and screened in float32 before the exact recompute.
 //  * assignment: tcgen05 GEMM X * C^T on the tensor cores with the centroids split into two bf16
-//    terms (hi + lo, residual ~2^-16 |c|), accumulated in TMEM, fused with an argmin epilogue that
-//    keeps the best three scores ||c||^2 - 2 x.c per token; when the top scores are closer than the
-//    error bound the candidates are re-ranked by exact float32 ||x - c||^2.  A CUDA-core kernel
-//    computes exact float32 distances for float32 inputs and d = 64.
-//  * update: one warp per cluster sums its members in ascending token order (the stable sort's
-//    order) in float64 and divides by the count; an empty cluster keeps its centroid.  It also
-//    emits the hi/lo split and ||c||^2 for the next assignment.
+//    terms (hi + lo, residual ~2^-16 |c|), accumulated in TMEM, fused with an argmin epilogue over
+//    the scores ||c||^2 - 2 x.c.  Per token the epilogue keeps the 4 smallest scores that lie
+//    within the error tolerance tau of the running minimum; a token left with one candidate is
+//    labelled there, a token with several (a near-tie) goes on a list that rerank_kernel decides
+//    by exact float32 ||x - c||^2, and a token whose 4-entry list overflowed (a fifth score within
+//    tau was dropped) goes on the same list with a flag that makes the re-rank scan all k
+//    centroids.  A CUDA-core kernel computes exact float32 distances for float32 inputs and d = 64.
+//  * update: one CTA per cluster stages its members' rows (ascending token order, the stable
+//    sort's) through shared memory and sums each dimension sequentially in float64, then divides by
+//    the count; an empty cluster keeps its centroid.  It also emits the hi/lo split and ||c||^2
+//    for the next assignment.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -712,8 +716,11 @@ constexpr int kAsgThreads = 384;
 constexpr uint32_t kAsgXStage = 32768;   // 128 tokens x 128 d bf16 (two 16 KB halves)
 constexpr uint32_t kAsgCStage = 65536;   // 128 centroids x 128 d x {hi, lo}
 constexpr uint32_t kAsgSmem = 2 * kAsgXStage + 2 * kAsgCStage + 1024 /*align*/ + 256 /*barriers*/ +
-                               128 * 9 * 4 /*half merge*/;
+                               128 * 10 * 4 /*half merge*/;
 constexpr uint32_t kAsgTmemCols = 512;   // 4 accumulators of 128 columns
+// Flag in the head field of a re-rank entry: the token's candidate list overflowed, so the re-rank
+// scans every centroid (heads are below 2^31 because B*H*N is).
+constexpr uint32_t kRrFullScan = 0x80000000u;
 
 struct AsgBars {
   uint64_t x_full[2], x_empty[2], c_full[2], c_empty[2], acc_full[4], acc_empty[4], mma_done;
@@ -741,8 +748,10 @@ __device__ __forceinline__ float tile_row_norm(const uint8_t* xt, int row) {
 }
 
 // Keep the 4 smallest (score, index) pairs: replace the worst entry if this one is better
-// (strictly: among equal scores the one seen first, i.e. the lower index, stays).
-__device__ __forceinline__ void cand_insert(float val, int j, float (&cv)[4], int (&ci)[4]) {
+// (strictly: among equal scores the one seen first, i.e. the lower index, stays).  `dropped` is the
+// smallest score that ever left the list or was refused by it; when it ends up within the final
+// tolerance, more than four centroids were candidates and the list alone cannot decide.
+__device__ __forceinline__ void cand_insert(float val, int j, float (&cv)[4], int (&ci)[4], float& dropped) {
   int wi = 0;
   float wv = cv[0];
 #pragma unroll
@@ -752,12 +761,15 @@ __device__ __forceinline__ void cand_insert(float val, int j, float (&cv)[4], in
       wi = r;
     }
   if (val < wv) {
+    dropped = fminf(dropped, wv);  // an empty slot holds +inf
 #pragma unroll
     for (int r = 0; r < 4; ++r)
       if (r == wi) {
         cv[r] = val;
         ci[r] = j;
       }
+  } else {
+    dropped = fminf(dropped, val);
   }
 }
 
@@ -765,7 +777,9 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, int BH, int N, int k, int kpad,
                      const float* __restrict__ c_norm, int32_t* __restrict__ labels, uint4* __restrict__ rr_list,
-                     uint32_t* __restrict__ rr_count, uint32_t rr_cap, DeviceStatus* st) {
+                     uint32_t* __restrict__ rr_count, uint32_t rr_cap, DeviceStatus* st,
+                     const uint64_t* __restrict__ wait_budget) {
+  const long long wb = effective_wait_budget(wait_budget);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;                       // 2 stages
@@ -814,7 +828,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
         const int bh = static_cast<int>(w / ntiles), tile = static_cast<int>(w % ntiles);
         const int xsI = it & 1;
-        if (it >= 2) ok = mbar_wait(smem_u32(&bars->x_empty[xsI]), ((it >> 1) - 1) & 1, st, kWhereAssign);
+        if (it >= 2) ok = mbar_wait(smem_u32(&bars->x_empty[xsI]), ((it >> 1) - 1) & 1, st, kWhereAssign, wb);
         if (!ok) break;
         const uint32_t xdst = smem_u32(xs + xsI * kAsgXStage);
         mbar_arrive_expect_tx(smem_u32(&bars->x_full[xsI]), kAsgXStage);
@@ -823,7 +837,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         tma_load_2d(xdst + 16384, &tm_x, 64, y, smem_u32(&bars->x_full[xsI]));
         for (int c = 0; c < nchunks; ++c, ++g) {
           const int cs = static_cast<int>(g & 1);
-          if (g >= 2) ok = mbar_wait(smem_u32(&bars->c_empty[cs]), ((g >> 1) - 1) & 1, st, kWhereAssign);
+          if (g >= 2) ok = mbar_wait(smem_u32(&bars->c_empty[cs]), ((g >> 1) - 1) & 1, st, kWhereAssign, wb);
           if (!ok) break;
           const uint32_t cdst = smem_u32(cstg + cs * kAsgCStage);
           const uint32_t bar = smem_u32(&bars->c_full[cs]);
@@ -851,14 +865,14 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
       bool ok = true;
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
         const int xsI = it & 1;
-        ok = mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssign);
+        ok = mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssign, wb);
         if (!ok) break;
         const uint32_t xa = smem_u32(xs + xsI * kAsgXStage);
         for (int c = 0; c < nchunks; ++c, ++g) {
           const int cs = static_cast<int>(g & 1);
           const int a = static_cast<int>(g & 3);
-          ok = mbar_wait(smem_u32(&bars->c_full[cs]), (g >> 1) & 1, st, kWhereAssign);
-          if (ok && g >= 4) ok = mbar_wait(smem_u32(&bars->acc_empty[a]), ((g >> 2) - 1) & 1, st, kWhereAssign);
+          ok = mbar_wait(smem_u32(&bars->c_full[cs]), (g >> 1) & 1, st, kWhereAssign, wb);
+          if (ok && g >= 4) ok = mbar_wait(smem_u32(&bars->acc_empty[a]), ((g >> 2) - 1) & 1, st, kWhereAssign, wb);
           if (!ok) break;
           tc_fence_after();
           const uint32_t cb = smem_u32(cstg + cs * kAsgCStage);
@@ -894,7 +908,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 4) >> 2;
     const int row = q * 32 + lane;
-    float* mrg = reinterpret_cast<float*>(bars + 1);  // [128][9]: warpgroup 1's minimum and list
+    float* mrg = reinterpret_cast<float*>(bars + 1);  // [128][10]: warpgroup 1's minimum, list, dropped
     long long g = 0;
     int it = 0;
     bool ok = true;
@@ -902,16 +916,17 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
       const int bh = static_cast<int>(w / ntiles), tile = static_cast<int>(w % ntiles);
       const int xsI = it & 1;
       const float* cn = c_norm + static_cast<size_t>(bh) * kpad;  // 4 KB at most: stays in L1
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssignTail));
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->x_full[xsI]), (it >> 1) & 1, st, kWhereAssignTail, wb));
       if (!ok) break;
       const uint8_t* xt = xs + xsI * kAsgXStage;
       const float xn = tile_row_norm(xt, row);
       float gmin = INFINITY;
       float cv[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
       int ci[4] = {-1, -1, -1, -1};
+      float dropped = INFINITY;
       for (int c = 0; c < nchunks; ++c, ++g) {
         const int a = static_cast<int>(g & 3);
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full[a]), (g >> 2) & 1, st, kWhereAssign));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full[a]), (g >> 2) & 1, st, kWhereAssign, wb));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -955,7 +970,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) hits |= (sc[e] <= thr ? 1u : 0u) << e;
             if (__popc(hits) == 1) {  // the usual case: the group's minimum is its only entry within tau
-              cand_insert(mloc, jb + __ffs(hits) - 1, cv, ci);
+              cand_insert(mloc, jb + __ffs(hits) - 1, cv, ci, dropped);
               hits = 0u;
             }
             while (hits) {
@@ -964,7 +979,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
               float val = sc[0];
 #pragma unroll
               for (int r = 1; r < 32; ++r) val = r == e ? sc[r] : val;
-              cand_insert(val, jb + e, cv, ci);
+              cand_insert(val, jb + e, cv, ci, dropped);
             }
           }
         }
@@ -974,12 +989,13 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
       }
       if (!ok) break;
       // merge: warpgroup 1 hands its minimum and list to warpgroup 0 (per token)
-      float* mr = mrg + row * 9;
+      float* mr = mrg + row * 10;
       if (half == 1) {
         if (it > 0)
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->merge_empty[q]), (it - 1) & 1, st, kWhereAssign));
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->merge_empty[q]), (it - 1) & 1, st, kWhereAssign, wb));
         if (!ok) break;
         mr[0] = gmin;
+        mr[9] = dropped;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           mr[1 + r] = cv[r];
@@ -988,16 +1004,17 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->merge_full[q]));
       } else {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->merge_full[q]), it & 1, st, kWhereAssign));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->merge_full[q]), it & 1, st, kWhereAssign, wb));
         if (!ok) break;
         gmin = fminf(gmin, mr[0]);
+        dropped = fminf(dropped, mr[9]);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int j = __float_as_int(mr[5 + r]);
-          if (j >= 0) cand_insert(mr[1 + r], j, cv, ci);  // higher indices than every own entry: ties keep own
+          if (j >= 0) cand_insert(mr[1 + r], j, cv, ci, dropped);  // higher indices than every own entry: ties keep own
         }
         const int n = tile * kAssignTileM + row;
-        bool defer = false;
+        bool defer = false, full_scan = false;
         uint32_t c01 = 0xffffffffu, c23 = 0xffffffffu;  // the candidates, 16 bits each (0xffff: none)
         if (n < N) {
           const float thr = gmin + (xn + fmaxf(gmin + xn, 0.f)) * 0x1p-11f;
@@ -1017,7 +1034,10 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
               }
             }
           }
-          defer = nc > 1;  // near-tie: the exact distances decide, in rerank_kernel
+          // near-tie: the exact distances decide, in rerank_kernel; a list that overflowed (a fifth
+          // score within tau was dropped) sends the token to an exact scan over every centroid there
+          full_scan = dropped <= thr;
+          defer = nc > 1 || full_scan;
           labels[static_cast<size_t>(bh) * N + n] = best < 0 ? 0 : best;
         }
         const unsigned dm = __ballot_sync(0xffffffffu, defer);
@@ -1027,7 +1047,8 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
           base = __shfl_sync(0xffffffffu, base, 0);
           const uint32_t slot = base + static_cast<uint32_t>(__popc(dm & ((1u << lane) - 1u)));
           if (defer && slot < rr_cap)
-            rr_list[slot] = make_uint4(static_cast<uint32_t>(bh), static_cast<uint32_t>(n), c01, c23);
+            rr_list[slot] = make_uint4(static_cast<uint32_t>(bh) | (full_scan ? kRrFullScan : 0u),
+                                       static_cast<uint32_t>(n), c01, c23);
           else if (defer)  // only past 2^32 - 1 listed tokens in one launch
             raise_status(st, kStatusDeviceBounds, kWhereAssign, slot, static_cast<uint32_t>(n));
         }
@@ -1051,7 +1072,16 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
 // Near-ties of the tensor-core assignment: one warp per listed token computes the exact float32
 // ||x - c||^2 of each candidate (lane l holds coordinates 4l .. 4l+3; the partial sums are then
 // added across the warp in a fixed butterfly order) and keeps the smallest, ties to the lower index.
+// A token whose candidate list overflowed is decided the same way over all k centroids.
 constexpr int kRrThreads = 256;
+
+__device__ __forceinline__ float rr_dist(float x0, float x1, float x2, float x3, float4 cv) {
+  const float d0 = x0 - cv.x, d1 = x1 - cv.y, d2 = x2 - cv.z, d3 = x3 - cv.w;
+  float part = fmaf(d3, d3, fmaf(d2, d2, fmaf(d1, d1, d0 * d0)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  return part;
+}
 
 __global__ void __launch_bounds__(kRrThreads) rerank_kernel(const uint16_t* __restrict__ X, int N, int k,
                                                             const float* __restrict__ C,
@@ -1063,9 +1093,24 @@ __global__ void __launch_bounds__(kRrThreads) rerank_kernel(const uint16_t* __re
   const uint32_t warps = gridDim.x * (kRrThreads / 32);
   for (uint32_t i = blockIdx.x * (kRrThreads / 32) + (threadIdx.x >> 5); i < total; i += warps) {
     const uint4 e = rr_list[i];
-    const size_t tok = static_cast<size_t>(e.x) * N + e.y;
+    const uint32_t hd = e.x & ~kRrFullScan;
+    const size_t tok = static_cast<size_t>(hd) * N + e.y;
     const uint2 xr = *reinterpret_cast<const uint2*>(X + tok * 128 + 4 * lane);
     const float x0 = bf16lo_to_f32(xr.x), x1 = bf16hi_to_f32(xr.x), x2 = bf16lo_to_f32(xr.y), x3 = bf16hi_to_f32(xr.y);
+    if (e.x & kRrFullScan) {  // uniform across the warp
+      const float4* cr = reinterpret_cast<const float4*>(C + static_cast<size_t>(hd) * k * 128) + lane;
+      int best = 0;
+      float bd = rr_dist(x0, x1, x2, x3, __ldg(cr));
+      for (int c = 1; c < k; ++c) {
+        const float part = rr_dist(x0, x1, x2, x3, __ldg(cr + static_cast<size_t>(c) * 32));
+        if (part < bd) {  // strict: ties keep the lower index
+          bd = part;
+          best = c;
+        }
+      }
+      if (lane == 0) labels[tok] = best;
+      continue;
+    }
     int cid[4];
     float4 cv4[4];
 #pragma unroll
@@ -1073,7 +1118,7 @@ __global__ void __launch_bounds__(kRrThreads) rerank_kernel(const uint16_t* __re
       const uint32_t w = r < 2 ? e.z : e.w;
       const int c = static_cast<int>((w >> (16 * (r & 1))) & 0xffffu);
       cid[r] = c < k ? c : -1;
-      cv4[r] = __ldg(reinterpret_cast<const float4*>(C + (static_cast<size_t>(e.x) * k + (c < k ? c : 0)) * 128) + lane);
+      cv4[r] = __ldg(reinterpret_cast<const float4*>(C + (static_cast<size_t>(hd) * k + (c < k ? c : 0)) * 128) + lane);
     }
     int best = -1;
     float bd = INFINITY;
@@ -1081,11 +1126,7 @@ __global__ void __launch_bounds__(kRrThreads) rerank_kernel(const uint16_t* __re
     for (int r = 0; r < 4; ++r) {
       const int c = cid[r];
       if (c < 0) continue;  // uniform across the warp
-      const float4 cv = cv4[r];
-      const float d0 = x0 - cv.x, d1 = x1 - cv.y, d2 = x2 - cv.z, d3 = x3 - cv.w;
-      float part = fmaf(d3, d3, fmaf(d2, d2, fmaf(d1, d1, d0 * d0)));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      const float part = rr_dist(x0, x1, x2, x3, cv4[r]);
       if (part < bd || (part == bd && c < best)) {
         bd = part;
         best = c;
@@ -1313,7 +1354,8 @@ cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, u
 
 cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,
                           const uint16_t* c_hi, const uint16_t* c_lo, const float* c_norm, int32_t* labels,
-                          uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, cudaStream_t s) {
+                          uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, const uint64_t* wait_budget,
+                          cudaStream_t s) {
   if (!x_f32 && d == 128) {
     alignas(64) CUtensorMap tx, th, tl;
     const int kp = kpad_of(k);
@@ -1331,7 +1373,7 @@ cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k
     const size_t bhn = static_cast<size_t>(BH) * N;  // rr_list holds one entry per token
     const uint32_t cap = bhn < 0xffffffffu ? static_cast<uint32_t>(bhn) : 0xffffffffu;
     assign_tc_kernel<<<grid, kAsgThreads, kAsgSmem, s>>>(tx, th, tl, BH, N, k, kp, c_norm, labels, rr_list, rr_count,
-                                                          cap, st);
+                                                          cap, st, wait_budget);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // eight CTAs of 8 warps per SM: each warp waits on its token's rows, so many warps in flight

@@ -77,7 +77,7 @@ extern "C" SVG2_API int svg2_sparse_attn_noalloc(const void* Qp, const void* Kp,
       return SVG2_ERR_CUDA;  // the library's own word is cleared so an old error cannot stop this call
     }
     const cudaError_t e = launch_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, static_cast<int>(BH), N,
-                                             d, nQ, nK, scale, perm_q, O, a, st, s);
+                                             d, nQ, nK, scale, perm_q, O, a, st, nullptr, s);
     return e == cudaSuccess ? SVG2_OK : SVG2_ERR_CUDA;
   } catch (...) {
     return SVG2_ERR_CUDA;

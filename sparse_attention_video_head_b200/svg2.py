@@ -28,7 +28,7 @@ _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "s
             "svg2_unpermute", "svg2_layer", "svg2_layer_host", "svg2_selftest_mma", "svg2_sparse_attn_noalloc",
             "svg2_dense_attn_workspace_size", "svg2_dense_attn", "svg2_driver_create", "svg2_driver_destroy",
             "svg2_driver_cache_bytes", "svg2_driver_bind_cache", "svg2_driver_reset", "svg2_driver_workspace_size",
-            "svg2_driver_plan", "svg2_driver_layer")
+            "svg2_driver_plan", "svg2_driver_layer", "svg2_set_wait_budget")
 
 _lib = None
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.svg2_workspace_size.argtypes = [I, I, I, I, I, I, ctypes.POINTER(S)]
         L.svg2_check_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_uint32),
                                         ctypes.POINTER(ctypes.c_uint32)]
+        L.svg2_set_wait_budget.argtypes = [P, ctypes.c_uint64, P]
         L.svg2_kmeanspp.argtypes = [P, I, I, I, I, I, I, P, I, P, P, S, P]
         L.svg2_kmeans.argtypes = [P, I, I, I, I, I, I, I, I, P, I, P, P, P, P, P, P, S, P]
         L.svg2_select.argtypes = [P, P, P, I, I, I, I, I, F, F, P, P, P, P, P, P, S, P]
@@ -188,6 +189,15 @@ def svg2_check_status(ws: torch.Tensor, stream=None):
     _check(lib().svg2_check_status(_p(ws), _stream(stream), ctypes.byref(code), ctypes.byref(where), info),
            "svg2_check_status")
     return int(code.value), int(where.value), (int(info[0]), int(info[1]))
+
+
+def svg2_set_wait_budget(ws: torch.Tensor, cycles: int, stream=None):
+    """Budget (SM clock cycles) of the bounded waits in the attention and assignment kernels for later
+    calls with this workspace; 0 restores the default.  Diagnostics only."""
+    if cycles < 0:
+        raise ValueError("cycles must be >= 0")
+    _check(lib().svg2_set_wait_budget(_arg(ws, "ws", _U8, 256), int(cycles), _stream(stream)),
+           "svg2_set_wait_budget")
 
 
 def raise_on_device_error(ws: torch.Tensor, stream=None):

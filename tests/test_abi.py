@@ -204,3 +204,8 @@ def test_dense_attn_rejects_bad_arguments(L):
     assert call(ws=None) == WORKSPACE
     assert call(ws=ctypes.c_void_p(0x10010)) == WORKSPACE        # not 256-byte aligned
     assert call(wsb=16) == WORKSPACE
+
+
+def test_set_wait_budget_rejects_a_missing_or_misaligned_workspace(L):
+    assert L.svg2_set_wait_budget(None, 100, None) == INVALID
+    assert L.svg2_set_wait_budget(ctypes.c_void_p(0x10010), 100, None) == INVALID  # not 256-byte aligned

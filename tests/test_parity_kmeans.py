@@ -164,3 +164,61 @@ def test_full_run_matches_oracle(oracle, cfg_name, role):
         print(f"{cfg_name}/{role} head {heads[h]}: label agreement {agree:.6f}, centroid rel err {err:.2e}")
         assert agree >= 0.99
         assert cnt[0, h].sum() == X.shape[2]
+
+
+def overflow_case(seed=21, H=4, groups=40, per_group=12, N=4096, gap=3e-4, offset=8.0):
+    """Tokens with more than four centroids inside the assignment's tolerance band.
+
+    Per head, `groups` base points x_g with coordinates near +-offset (so ||x||^2 ~ 128 offset^2 and
+    float32 scores ||c||^2 - 2 x.c carry rounding errors far larger than the spacing below), and
+    per base point `per_group` float32 centroids at squared distance (1 + gap*i) from it, i = 0..,
+    in shuffled index order.  Every token is a copy of one base point.  Its nearest centroid is then
+    ahead of the next by a relative gap of `gap` (not a near-tie), while all `per_group` centroids lie
+    within 2^-11 (||x||^2 + d_min) of the nearest, so a short candidate list kept by approximate
+    score can miss the nearest one.
+    """
+    rng = np.random.default_rng(seed)
+    d, k = 128, groups * per_group
+    X = np.empty((1, H, N, d), np.float32)
+    C = np.empty((1, H, k, d), np.float32)
+    for h in range(H):
+        base = offset * rng.choice([-1.0, 1.0], size=(groups, d)) + 0.5 * rng.standard_normal((groups, d))
+        base = I.round_to_bf16(base.astype(np.float32)).astype(np.float64)
+        for g in range(groups):
+            u = rng.standard_normal((per_group, d))
+            u /= np.linalg.norm(u, axis=1, keepdims=True)
+            r = np.sqrt(1.0 + gap * np.arange(per_group))
+            idx = g * per_group + rng.permutation(per_group)
+            C[0, h, idx] = (base[g] + r[:, None] * u).astype(np.float32)
+        X[0, h] = base[rng.integers(0, groups, size=N)].astype(np.float32)
+    return X, C
+
+
+def test_overflow_case_has_crowded_candidates_and_no_near_ties(oracle):
+    """The construction itself (CPU): nearest centroid unique by >= 1e-4 relative, and at least
+    eight centroids within 2^-11 (||x||^2 + d_min) of the nearest for every token."""
+    X, C = overflow_case(H=1, N=256)
+    x, c = X[0, 0].astype(np.float64), C[0, 0].astype(np.float64)
+    lab, d1, d2 = oracle.assign(X[0, 0], c)
+    assert not near_tie(d1, d2).any()
+    dist = ((x[:, None, :] - c[None, :, :]) ** 2).sum(-1)
+    band = 2.0 ** -11 * ((x * x).sum(1) + d1)
+    crowd = (dist <= (d1 + band)[:, None]).sum(1)
+    assert crowd.min() >= 8, crowd.min()
+    np.testing.assert_array_equal(lab, dist.argmin(1))
+
+
+@pytest.mark.gpu
+def test_assign_candidate_list_overflow(oracle):
+    """A token whose tolerance band holds more centroids than the epilogue's candidate list must
+    still get its exact nearest centroid: 0 mismatches away from near-ties (there are none here)."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS["small"]          # bf16, d = 128: the tensor-core assignment and its re-rank
+    X, C0 = overflow_case()
+    k = C0.shape[2]
+    _, lab, _ = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_GIVEN, C0=C0.astype(np.float64))
+    for h in range(X.shape[1]):
+        ref_lab, d1, d2 = oracle.assign(X[0, h], C0[0, h].astype(np.float64))
+        assert not near_tie(d1, d2).any()
+        bad = int((lab[0, h] != ref_lab).sum())
+        assert bad == 0, f"head {h}: {bad} of {X.shape[2]} tokens not at their nearest centroid"
