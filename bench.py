@@ -54,6 +54,9 @@ def parse():
                          "heads of one layer (strong scaling)")
     ap.add_argument("--no-warm", action="store_true", help="skip the warm-start denoising-sequence measurement")
     ap.add_argument("--warm-steps", type=int, default=10)
+    ap.add_argument("--no-layer-call", action="store_true", help="skip the single svg2_layer call at top-p 0.5")
+    ap.add_argument("--second", default="hunyuan720p", choices=["none"] + sorted(I.CONFIGS),
+                    help="a second configuration measured after the first (stages, top-p sweep, dense attention)")
     ap.add_argument("--seed-tokens", type=int, default=16384,
                     help="k-means++ candidates per (b,h): every ceil(N/seed_tokens)-th token (0 = all tokens)")
     return ap.parse_args()
@@ -138,16 +141,23 @@ def sample_text(cfg, rows, heads):
             f"x{cfg.N}/{rows} rows, mean head x{cfg.H} heads")
 
 
+# One sample definition for both CPU legs (the reference arm and cpu_baseline): the first
+# ORACLE_HEADS heads in full (k-means, selection, permutation) and ORACLE_ROWS query rows of attention
+# per head, extrapolated to the layer.
+ORACLE_HEADS, ORACLE_ROWS = 2, 128
+
+
 def run_reference(args, cfg):
     cores = len(os.sched_getaffinity(0))
+    heads = tuple(range(min(ORACLE_HEADS, cfg.H)))
     for _ in range(args.warmup):
-        oracle_sample(cfg, args.top_p, rows=16, seed_tokens=args.seed_tokens)
+        oracle_sample(cfg, args.top_p, rows=16, heads=heads[:1], seed_tokens=args.seed_tokens)
     vals = []
     for _ in range(args.steps):
-        v, _ = oracle_sample(cfg, args.top_p, seed_tokens=args.seed_tokens)
+        v, _ = oracle_sample(cfg, args.top_p, rows=ORACLE_ROWS, heads=heads, seed_tokens=args.seed_tokens)
         vals.append(v)
     value = statistics.median(vals)
-    sample = sample_text(cfg, 96, (0,))
+    sample = sample_text(cfg, ORACLE_ROWS, heads)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "ms", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -232,6 +242,174 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------------------------------------ one layer
+class LayerBench:
+    """Device buffers and the timed step of one layer configuration, every stage through the C ABI:
+    k-means of Q and of K, selection, the three row gathers, the attention with the inverse
+    permutation fused into its epilogue."""
+
+    names = ["kmeans_q", "kmeans_k", "select", "permute", "sparse_attn"]
+
+    def __init__(self, svg2, torch, cfg, data, dev, seed_tokens, top_p):
+        self.svg2, self.torch, self.cfg, self.dev = svg2, torch, cfg, dev
+        self.seed_tokens, self.top_p = seed_tokens, top_p
+        B, H, N, d = 1, cfg.H, cfg.N, cfg.d
+        self.scale = float(np.float32(cfg.scale))
+        self.Q = torch.from_numpy(data["q"]).to(torch.bfloat16).to(dev)
+        self.K = torch.from_numpy(data["k"]).to(torch.bfloat16).to(dev)
+        self.V = torch.from_numpy(data["v"]).to(torch.bfloat16).to(dev)
+        self.uq = torch.from_numpy(data["uq"]).to(dev)
+        self.uk = torch.from_numpy(data["uk"]).to(dev)
+        self.cq = torch.zeros(B, H, cfg.nQ, d, device=dev)
+        self.ck = torch.zeros(B, H, cfg.nK, d, device=dev)
+        self.O = torch.empty_like(self.Q)
+        self.ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK, device=dev)
+        self.Qp, self.Kp, self.Vp = torch.empty_like(self.Q), torch.empty_like(self.K), torch.empty_like(self.V)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.lab_q, self.lab_k = torch.empty(B, H, N, **i32), torch.empty(B, H, N, **i32)
+        self.cnt_q, self.cnt_k = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nK, **i32)
+        self.perm_q, self.perm_k = torch.empty(B, H, N, **i32), torch.empty(B, H, N, **i32)
+        self.q_off, self.k_off = torch.empty(B, H, cfg.nQ + 1, **i32), torch.empty(B, H, cfg.nK + 1, **i32)
+        self.mask = torch.empty(B, H, cfg.nQ, cfg.nK, dtype=torch.uint8, device=dev)
+        self.sel_count, self.sel_idx = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nQ, cfg.nK, **i32)
+        self.stream_len = torch.empty(B, H, cfg.nQ, **i32)
+        self.stream = torch.cuda.current_stream(dev)
+
+    def step(self, ev=None, top_p=None):
+        svg2, cfg, KPP = self.svg2, self.cfg, self.svg2.SVG2_INIT_KMEANSPP
+
+        def mark(i):
+            if ev is not None:
+                ev[i].record(self.stream)
+        mark(0)
+        svg2.svg2_kmeans(self.Q, cfg.nQ, cfg.iters, KPP, self.cq, self.lab_q, self.cnt_q, self.ws, u=self.uq,
+                         perm=self.perm_q, offsets=self.q_off, seed_tokens=self.seed_tokens)
+        mark(1)
+        svg2.svg2_kmeans(self.K, cfg.nK, cfg.iters, KPP, self.ck, self.lab_k, self.cnt_k, self.ws, u=self.uk,
+                         perm=self.perm_k, offsets=self.k_off, seed_tokens=self.seed_tokens)
+        mark(2)
+        self.select(self.top_p if top_p is None else top_p)
+        mark(3)
+        svg2.svg2_gather(self.Q, self.perm_q, self.Qp)
+        svg2.svg2_gather(self.K, self.perm_k, self.Kp)
+        svg2.svg2_gather(self.V, self.perm_k, self.Vp)
+        mark(4)
+        self.attend()
+        mark(5)
+
+    def select(self, p):
+        self.svg2.svg2_select(self.cq, self.ck, self.cnt_k, p, self.scale, self.mask, self.sel_count, self.sel_idx,
+                              self.ws, stream_len=self.stream_len)
+
+    def attend(self):
+        self.svg2.svg2_sparse_attn(self.Qp, self.Kp, self.Vp, self.q_off, self.k_off, self.sel_count, self.sel_idx,
+                                   self.scale, self.O, self.ws, perm_q=self.perm_q)
+
+    def flops(self):
+        """(actual, dense-equivalent, executed) attention FLOPs of the current selection."""
+        cfg, d = self.cfg, self.cfg.d
+        cq_h = self.cnt_q.cpu().numpy().astype(np.float64)
+        sl_h = self.stream_len.cpu().numpy().astype(np.float64)
+        actual = 4.0 * d * float((cq_h * sl_h).sum())
+        dense = 4.0 * d * cfg.N * cfg.N * cfg.B * cfg.H
+        executed = 4.0 * d * float((np.ceil(cq_h / 128.0) * 128.0 * np.ceil(sl_h / 128.0) * 128.0).sum())
+        return actual, dense, executed
+
+    def time_steps(self, steps):
+        torch = self.torch
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_start.record(self.stream)
+        for i in range(steps):
+            self.step(evs[i])
+        t_end.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(self.names)}
+        return t_start.elapsed_time(t_end), stage_ms
+
+    def sweep(self, stage_ms, extra=(0.5, 1.0)):
+        """Selection + attention per top-p on the step's clusters: the configuration's values plus
+        labelled extension points (p = 0.5 towards the pages' 25-35 % densities on these inputs, p = 1
+        every pair kept: dense attention through the sparse path)."""
+        torch = self.torch
+        notes = {0.5: "extension: lower density", 1.0: "extension: every pair kept (dense through the sparse path)"}
+        kmeans_ms = stage_ms["kmeans_q"] + stage_ms["kmeans_k"]
+        out = {}
+        for p in sorted(set(self.cfg.top_p) | {self.top_p} | set(extra)):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            self.select(p)
+            self.attend()
+            torch.cuda.synchronize(self.dev)
+            ev[0].record(self.stream)
+            self.select(p)
+            ev[1].record(self.stream)
+            self.attend()
+            ev[2].record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            flops, dense, _ = self.flops()
+            a_ms = ev[1].elapsed_time(ev[2])
+            out[str(p)] = {"density": flops / dense, "select_ms": ev[0].elapsed_time(ev[1]), "attn_ms": a_ms,
+                           "attn_tflops_actual": flops / (a_ms * 1e-3) / 1e12,
+                           "attn_tflops_effective": dense / (a_ms * 1e-3) / 1e12,
+                           "layer_ms": kmeans_ms + ev[0].elapsed_time(ev[1]) + stage_ms["permute"] + a_ms}
+            if p in notes and p not in set(self.cfg.top_p) | {self.top_p}:
+                out[str(p)]["note"] = notes[p]
+        self.select(self.top_p)
+        return out
+
+
+def time_layer_call(svg2, torch, lb, top_p, dense_ms, reps=3):
+    """The whole layer as one svg2_layer call (k-means++ and Lloyd on Q and K, selection,
+    permutation, attention with the fused inverse permutation) at `top_p`, timed with CUDA events."""
+    cfg = lb.cfg
+    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, top_p, lb.scale, 1, lb.seed_tokens)
+    cq, ck = torch.zeros_like(lb.cq), torch.zeros_like(lb.ck)
+    outs = svg2.layer_output_buffers(1, cfg.H, cfg.N, cfg.nQ, cfg.nK, device=lb.dev)
+    svg2.svg2_layer(lb.Q, lb.K, lb.V, prm, cq, ck, lb.O, lb.ws, lb.uq, lb.uk, outs)
+    torch.cuda.synchronize(lb.dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(lb.stream)
+    for _ in range(reps):
+        svg2.svg2_layer(lb.Q, lb.K, lb.V, prm, cq, ck, lb.O, lb.ws, lb.uq, lb.uk, outs)
+    b.record(lb.stream)
+    torch.cuda.synchronize(lb.dev)
+    svg2.raise_on_device_error(lb.ws)
+    ms = a.elapsed_time(b) / reps
+    cnt_q = outs["count_q"].cpu().numpy().astype(np.float64)
+    sl = outs["stream_len"].cpu().numpy().astype(np.float64)
+    density = float((cnt_q * sl).sum()) / (cfg.N * cfg.N * cfg.B * cfg.H)
+    out = {"api": "svg2_layer", "top_p": top_p, "density": density, "ms": ms, "reps": reps}
+    if isinstance(dense_ms, float):
+        out["dense_sdpa_ms"] = dense_ms
+        out["speedup_vs_dense"] = dense_ms / ms
+    return out
+
+
+def measure_second_config(svg2, torch, cfg, args, dev, P, steps=3, warmup=2):
+    """A second configuration (by default the Hunyuan-720p layer): stage times of the step, density
+    and attention throughput per top-p, and dense attention on the same tensors."""
+    data = gen_inputs(cfg)
+    lb = LayerBench(svg2, torch, cfg, data, dev, args.seed_tokens, args.top_p)
+    del data
+    for _ in range(warmup):
+        lb.step()
+    torch.cuda.synchronize(dev)
+    svg2.raise_on_device_error(lb.ws)
+    actual, dense, executed = lb.flops()
+    total_ms, stage_ms = lb.time_steps(steps)
+    svg2.raise_on_device_error(lb.ws)
+    attn_tflops = actual / (stage_ms["sparse_attn"] * 1e-3) / 1e12
+    out = {"workload": cfg.name, "H": cfg.H, "N": cfg.N, "nQ": cfg.nQ, "nK": cfg.nK, "iters": cfg.iters,
+           "top_p": args.top_p, "steps": steps, "ms_per_step": total_ms / steps, "stages_ms": stage_ms,
+           "density": actual / dense, "attn_tflops_actual": attn_tflops,
+           "attn_frac_of_sustained_peak": attn_tflops / P["bf16_sustained"],
+           "executed_over_actual": executed / actual, "top_p_sweep": lb.sweep(stage_ms, extra=(0.5,))}
+    out["dense_sdpa_ms"] = time_dense(torch, lb.Q, lb.K, lb.V, lb.scale)
+    out["layer_call_low_density"] = time_layer_call(svg2, torch, lb, 0.5, out["dense_sdpa_ms"])
+    svg2.raise_on_device_error(lb.ws)
+    return out
+
+
 # ------------------------------------------------------------------------------------------ GPU arm
 def main():
     args = parse()
@@ -273,114 +451,41 @@ def main():
     B, H, N, d = 1, cfg.H, cfg.N, cfg.d
     BH = B * H
     scale = float(np.float32(cfg.scale))
-    Q = torch.from_numpy(data["q"]).to(torch.bfloat16).to(dev)
-    K = torch.from_numpy(data["k"]).to(torch.bfloat16).to(dev)
-    V = torch.from_numpy(data["v"]).to(torch.bfloat16).to(dev)
-    uq = torch.from_numpy(data["uq"]).to(dev)
-    uk = torch.from_numpy(data["uk"]).to(dev)
-    cq = torch.zeros(B, H, cfg.nQ, d, device=dev)
-    ck = torch.zeros(B, H, cfg.nK, d, device=dev)
-    O = torch.empty_like(Q)
-    outs = svg2.layer_output_buffers(B, H, N, cfg.nQ, cfg.nK, device=dev)
-    ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK, device=dev)
-    Qp, Kp, Vp = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
-    i32 = dict(dtype=torch.int32, device=dev)
-    lab_q, lab_k = torch.empty(B, H, N, **i32), torch.empty(B, H, N, **i32)
-    cnt_q, cnt_k = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nK, **i32)
-    perm_q, perm_k = torch.empty(B, H, N, **i32), torch.empty(B, H, N, **i32)
-    q_off, k_off = torch.empty(B, H, cfg.nQ + 1, **i32), torch.empty(B, H, cfg.nK + 1, **i32)
-    mask = torch.empty(B, H, cfg.nQ, cfg.nK, dtype=torch.uint8, device=dev)
-    sel_count, sel_idx = torch.empty(B, H, cfg.nQ, **i32), torch.empty(B, H, cfg.nQ, cfg.nK, **i32)
-    stream_len = torch.empty(B, H, cfg.nQ, **i32)
+    lb = LayerBench(svg2, torch, cfg, data, dev, args.seed_tokens, args.top_p)
+    Q, K, V, O, ws = lb.Q, lb.K, lb.V, lb.O, lb.ws
+    Qp, Kp, Vp = lb.Qp, lb.Kp, lb.Vp
+    perm_q, perm_k, q_off, k_off = lb.perm_q, lb.perm_k, lb.q_off, lb.k_off
+    cq, ck, lab_q, lab_k, cnt_q, cnt_k, uq, uk = lb.cq, lb.ck, lb.lab_q, lb.lab_k, lb.cnt_q, lb.cnt_k, lb.uq, lb.uk
     KPP = svg2.SVG2_INIT_KMEANSPP
     stream = torch.cuda.current_stream(dev)
-    names = ["kmeans_q", "kmeans_k", "select", "permute", "sparse_attn"]
-
-    def step(ev=None):
-        def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
-        mark(0)
-        svg2.svg2_kmeans(Q, cfg.nQ, cfg.iters, KPP, cq, lab_q, cnt_q, ws, u=uq, perm=perm_q, offsets=q_off,
-                         seed_tokens=args.seed_tokens)
-        mark(1)
-        svg2.svg2_kmeans(K, cfg.nK, cfg.iters, KPP, ck, lab_k, cnt_k, ws, u=uk, perm=perm_k, offsets=k_off,
-                         seed_tokens=args.seed_tokens)
-        mark(2)
-        svg2.svg2_select(cq, ck, cnt_k, args.top_p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
-        mark(3)
-        svg2.svg2_gather(Q, perm_q, Qp)
-        svg2.svg2_gather(K, perm_k, Kp)
-        svg2.svg2_gather(V, perm_k, Vp)
-        mark(4)
-        svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
-        mark(5)
 
     for _ in range(args.warmup):
-        step()
+        lb.step()
     torch.cuda.synchronize(dev)
     svg2.raise_on_device_error(ws)
 
     # algorithmic work of the attention (actual = kept pairs only, no padding)
-    cq_h = cnt_q.cpu().numpy().astype(np.float64)
-    sl_h = stream_len.cpu().numpy().astype(np.float64)
-    actual_flops = 4.0 * d * float((cq_h * sl_h).sum())
-    dense_flops = 4.0 * d * N * N * BH
+    actual_flops, dense_flops, executed_flops = lb.flops()
     density = actual_flops / dense_flops
-    tiles_q = np.ceil(cq_h / 128.0)
-    executed_flops = 4.0 * d * float((tiles_q * 128.0 * np.ceil(sl_h / 128.0) * 128.0).sum())
-    waste128 = fixed128_waste(q_off.cpu().numpy(), k_off.cpu().numpy(), mask.cpu().numpy(), heads=range(min(4, H)))
+    waste128 = fixed128_waste(q_off.cpu().numpy(), k_off.cpu().numpy(), lb.mask.cpu().numpy(), heads=range(min(4, H)))
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
+        total_ms, stage_ms = lb.time_steps(args.steps)
     if world > 1:
         dist.barrier()
     svg2.raise_on_device_error(ws)
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dist, dev)
+    total_ms = max_over_ranks(total_ms, world, dist, dev)
     ms_per_step = total_ms / args.steps
-    stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
     attn_ms = stage_ms["sparse_attn"]
     achieved_tflops = actual_flops / (attn_ms * 1e-3) / 1e12
 
     # the configuration's top-p sweep on the same clusters: selection + attention per p
     sweep = None
     if not args.no_sweep:
-        sweep = {}
-        kmeans_ms = stage_ms["kmeans_q"] + stage_ms["kmeans_k"]
-        # the configuration's top-p values, plus two labelled extension points: p = 0.5 (towards the
-        # pages' 25-35 % densities on these inputs) and p = 1 (every pair kept: dense attention through
-        # the sparse path)
-        extension = {0.5: "extension: lower density", 1.0: "extension: every pair kept (dense through the sparse path)"}
-        for p in sorted(set(cfg.top_p) | {args.top_p} | set(extension)):
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-            svg2.svg2_select(cq, ck, cnt_k, p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
-            svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
-            torch.cuda.synchronize(dev)
-            ev[0].record(stream)
-            svg2.svg2_select(cq, ck, cnt_k, p, scale, mask, sel_count, sel_idx, ws, stream_len=stream_len)
-            ev[1].record(stream)
-            svg2.svg2_sparse_attn(Qp, Kp, Vp, q_off, k_off, sel_count, sel_idx, scale, O, ws, perm_q=perm_q)
-            ev[2].record(stream)
-            torch.cuda.synchronize(dev)
-            sl = stream_len.cpu().numpy().astype(np.float64)
-            flops = 4.0 * d * float((cq_h * sl).sum())
-            a_ms = ev[1].elapsed_time(ev[2])
-            sweep[str(p)] = {"density": flops / dense_flops, "select_ms": ev[0].elapsed_time(ev[1]),
-                             "attn_ms": a_ms, "attn_tflops_actual": flops / (a_ms * 1e-3) / 1e12,
-                             "attn_tflops_effective": dense_flops / (a_ms * 1e-3) / 1e12,
-                             "layer_ms": kmeans_ms + ev[0].elapsed_time(ev[1]) + stage_ms["permute"] + a_ms}
-            if p in extension and p not in set(cfg.top_p) | {args.top_p}:
-                sweep[str(p)]["note"] = extension[p]
+        sweep = lb.sweep(stage_ms)
         svg2.raise_on_device_error(ws)
 
     # HBM stages against the measured copy bandwidth: the three row gathers (permutation) as timed
@@ -439,16 +544,26 @@ def main():
     if not args.no_warm:
         warm = measure_warm(svg2, torch, cfg, args, dev, Q, K, V, ws, scale)
 
+    # the whole layer as one svg2_layer call at a low top-p (the pages' 25-35 % densities on these
+    # inputs), beside dense attention on the same tensors
+    layer_call = None
+    if not args.no_layer_call and rank == 0:
+        layer_call = time_layer_call(svg2, torch, lb, 0.5, dense_ms)
+
+    second = None
+    if args.second not in ("none", cfg.name) and not args.heads and rank == 0 and world == 1:
+        second = measure_second_config(svg2, torch, I.CONFIGS[args.second], args, dev, P)
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        heads = tuple(range(min(8, cfg.H)))
-        v, parts = oracle_sample(cfg, args.top_p, rows=256, heads=heads, seed_tokens=args.seed_tokens)
+        heads = tuple(range(min(ORACLE_HEADS, cfg.H)))
+        v, parts = oracle_sample(cfg, args.top_p, rows=ORACLE_ROWS, heads=heads, seed_tokens=args.seed_tokens)
         cpu = {"value": v, "unit": "ms", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-               "sample": sample_text(cfg, 256, heads), "parts_s": parts}
+               "sample": sample_text(cfg, ORACLE_ROWS, heads), "parts_s": parts}
     launches = kernel_launches(cfg)
     line = {
         "metric": METRIC, "value": whole_job_ms_per_layer(ms_per_step, world, sharded), "unit": "ms", "n_gpus": world,
@@ -470,7 +585,7 @@ def main():
         "hbm_stages": hbm_stages,
         "dense_sdpa_ms": dense_ms, "dense_sdpa_backends_enabled": sdpa_backends(torch) if dense_ms is not None else None,
         "dense_svg2_dense_attn": own_dense, "denoise_driver": denoise, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
-        "top_p_sweep": sweep,
+        "top_p_sweep": sweep, "layer_call_low_density": layer_call, "second_config": second,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -5,19 +5,20 @@
 // kept K clusters, concatenated into one packed key stream and cut into 128-key tiles, so a
 // cluster boundary costs nothing; only the stream's last tile is masked.  The design follows the
 // Blackwell execution model rather than the pages' FlashInfer-derived kernel:
-//   warps 0-3   softmax + correction + epilogue for Q tile A (TMEM lanes = query rows)
+//   warps 0-3   softmax + lazy O rescale + epilogue for Q tile A (TMEM lanes = query rows)
 //   warps 4-7   the same for Q tile B
-//   warps 8-11  key/value producer: thread r gathers row r of each key tile with cp.async into
-//               the 128-byte-swizzled layout the tensor core reads (two stages)
-//   warp 12     Q tiles by TMA, then the single-thread MMA issuer
-//   warp 13     TMEM allocator (512 columns: S_A, S_B, O_A, O_B)
-// Registers are re-split after set-up: the softmax warpgroups take 192 per thread, the producer 40,
-// the MMA group 88.  S is computed in 64-key sub-tiles into a two-slot ring inside each Q tile's
-// 128 S columns, and P (bf16) overwrites the first 32 columns of its slot as the A operand of the
-// PV product, so per Q tile the chain is: softmax(k) -> PV(k) -> S(k+2) into the freed slot,
-// while the softmax of k+1 runs on the other slot.  MMA order per sub-tile k: PV_A(k), S_A(k+2),
-// PV_B(k), S_B(k+2).  The softmax rescales O in TMEM (only when the row max grows by more than
-// 2^8) after PV(k-1) has landed.  Softmax is exact: p = 2^(s*scale*log2e - m), O / l at the end,
+//   warps 8-9   key/value producer: each thread gathers two rows of each key tile with cp.async
+//               into the 128-byte-swizzled layout the tensor core reads (two stages)
+//   warp 10     TMEM allocator (512 columns: S_A, S_B, O_A, O_B), Q tiles by TMA, then the
+//               single-thread MMA issuer; warp 11 idles (setmaxnreg acts on whole warpgroups)
+// After set-up the softmax warps take 184 registers per thread and the rest 120.  Each Q tile has one
+// 128-column S slot: S = Q K^T is one N = 128 product per key tile (full rate; a 64-key product is
+// bound by the shared-memory reads of its operands), and P (bf16) overwrites the slot's first 64
+// columns as the A operand of the PV product.  MMA order per key tile j: PV_A(j), S_A(j+1),
+// PV_B(j), S_B(j+1), so the two tiles' softmaxes run half a period apart and each one's
+// exponentials overlap the other's products.  The commit that announces S_x(j+1) also covers
+// PV_x(j), so the softmax may rescale O_x in TMEM (only when the row max grows by more than 2^8)
+// as soon as it sees S_x(j+1).  Softmax is exact: p = 2^(s*scale*log2e - m), O / l at the end,
 // with l summed over the float32 p whose bf16 rounding the PV product uses.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -29,7 +30,18 @@ namespace svg2 {
 
 namespace {
 
-constexpr int kAttnThreads = 512;
+// 12 warps in three warpgroups: 8 softmax warps, 2 key/value producer warps, the MMA issuer and
+// one idle warp (setmaxnreg acts on whole warpgroups).
+constexpr int kAttnThreads = 384;
+constexpr int kProducerWarp0 = 8, kProducerWarps = 2;
+constexpr int kProducerThreads = 32 * kProducerWarps;
+constexpr int kMmaWarp = 10;
+// Register split after set-up (setmaxnreg): 256 x 184 + 128 x 120 = 62464 <= 384 x 168, the launch's
+// allocation under __launch_bounds__(384, 1) (ptxas gives 168 registers per thread).
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 184;
+constexpr int kOtherRegs = 120;
+static_assert(256 * kSoftmaxRegs + (kAttnThreads - 256) * kOtherRegs <= kAttnThreads * kLaunchRegs, "register split");
 constexpr int kMaxRanges = 1024;
 // bytes of one 128-row tile of d bf16 values (d/64 swizzled 16 KB halves)
 template <int D>
@@ -38,15 +50,13 @@ template <int D>
 constexpr uint32_t attn_smem() { return 6 * tile_bytes<D>() + 1024 /*align*/ + 4096 /*ranges*/ + 4096 + 64 /*cum*/ + 256; }
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Of every 32 scores of a row, this many (the last ones) get 2^x from a polynomial on the FMA pipe
-// instead of the MUFU.  0: every exponential on the MUFU, the fastest setting measured here (4 of 32
-// was no faster, 8 and 12 slower: the polynomial's issue slots cost more than the MUFU time saved).
-constexpr int kEmuPerChunk = 0;
+// Of every 16 key pairs of a row, this many (the last ones) get 2^x from the cubic on the FMA pipe;
+// the rest use the MUFU, whose 16 exponentials per clock per SM would otherwise bound the softmax.
+constexpr int kCubicPairs = 4;
 
 struct AttnBars {
   uint64_t q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], o_full, mma_done;
-  uint64_t s_full[2][2], p_full[2][2];  // [Q tile][S slot]
-  uint64_t pv_done[2];                  // one phase per PV product of each Q tile
+  uint64_t s_full[2], p_full[2][2];  // per Q tile; P in two 64-key halves
   uint32_t tmem_base;
   int32_t L;
   int32_t nranges;
@@ -138,33 +148,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars->k_full[i]), 128);
-      mbar_init(smem_u32(&bars->v_full[i]), 128);
+      mbar_init(smem_u32(&bars->k_full[i]), kProducerThreads);
+      mbar_init(smem_u32(&bars->v_full[i]), kProducerThreads);
       mbar_init(smem_u32(&bars->k_empty[i]), 1);
       mbar_init(smem_u32(&bars->v_empty[i]), 1);
-      for (int t = 0; t < 2; ++t) {
-        mbar_init(smem_u32(&bars->s_full[i][t]), 1);
-        mbar_init(smem_u32(&bars->p_full[i][t]), 4);
-      }
-      mbar_init(smem_u32(&bars->pv_done[i]), 1);
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->p_full[i][0]), 4);
+      mbar_init(smem_u32(&bars->p_full[i][1]), 4);
     }
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->mma_done), 1);
     fence_mbar_init();
   }
-  if (warp == 13) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
-  if (warp >= 8 && warp < 12) {
+  if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
     // key-stream range table: start row and stream offset of every kept K cluster
-    const int pt = threadIdx.x - 256;
+    const int pt = threadIdx.x - 32 * kProducerWarp0;
     const size_t row = static_cast<size_t>(bh) * nQ + un.cluster;
     int cnt = sel_count[row];
     cnt = cnt < 0 ? 0 : (cnt > nK ? nK : cnt);
     const int32_t* ko = k_off + static_cast<size_t>(bh) * (nK + 1);
-    // each thread handles a contiguous block of entries, then a scan over the 128 block sums
-    const int per = (cnt + 127) / 128;
+    // each thread handles a contiguous block of entries, then a scan over the block sums
+    const int per = (cnt + kProducerThreads - 1) / kProducerThreads;
     const int e0 = min(cnt, pt * per), e1 = min(cnt, e0 + per);
     int local = 0;
     for (int e = e0; e < e1; ++e) {
@@ -175,26 +183,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       r_cum[e] = len;  // temporarily the length
       local += len;
     }
-    // scan of `local` across the 128 producer threads (4 warps) via shuffles + shared
+    // scan of `local` across the producer threads via shuffles + shared
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    int32_t* wsum = r_cum + kMaxRanges + 1;  // 4 scratch ints (inside the 16-int gap)
-    if (lane == 31) wsum[warp - 8] = incl;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int32_t* wsum = r_cum + kMaxRanges + 1;  // one scratch int per producer warp (inside the 16-int gap)
+    if (lane == 31) wsum[warp - kProducerWarp0] = incl;
+    asm volatile("bar.sync 1, %0;" ::"n"(kProducerThreads) : "memory");
     int wbase = 0;
-    for (int w = 0; w < warp - 8; ++w) wbase += wsum[w];
+    for (int w = 0; w < warp - kProducerWarp0; ++w) wbase += wsum[w];
     int run = wbase + incl - local;
     for (int e = e0; e < e1; ++e) {
       const int len = r_cum[e];
       r_cum[e] = run;
       run += len;
     }
-    if (pt == 127) {
-      bars->L = run;  // thread 127 holds the last block
+    if (pt == kProducerThreads - 1) {
+      bars->L = run;  // the last producer thread holds the last block
       bars->nranges = cnt;
       r_cum[cnt] = run;
     }
@@ -205,14 +213,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   const int L = bars->L;
   const int nranges = bars->nranges;
-  const int nt = (L + 127) / 128;
+  const int T = (L + 127) / 128;  // 128-key tiles of the packed key stream
 
-  // Warpgroups 0-1 (softmax) take registers from warpgroups 2-3 (producer; MMA, allocator):
-  // 256 x 192 + 128 x 40 + 128 x 88 = 512 x 128, the launch's allocation.
-  if (warp >= 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+  // The softmax warpgroups take registers from the producer/MMA warpgroup.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs) : "memory");
+  }
+  if (warp == kMmaWarp) {
     // ---------------- Q by TMA, then MMA issue ----------------
-    if (warp == 12 && elect_one()) {
+    if (elect_one()) {
       prefetch_tensormap(&tm_q);
       const uint32_t qbar = smem_u32(&bars->q_full);
       const uint32_t qa = smem_u32(q_s), qb = smem_u32(q_s + kTile);
@@ -224,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (has_b) tma_load_2d(qb + hf * 16384, &tm_q, hf * 64, y + 128, qbar);
       }
       bool ok = mbar_wait(qbar, 0, st, kWhereAttnMma, wb);
-      const uint32_t id_s = idesc_bf16_f32(128, 64, 0);
+      const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t id_o = idesc_bf16_f32(128, D, 1);
       const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
       // Descriptors of every operand tile, built once: stepping along K only moves the start
@@ -232,75 +241,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = sdesc_sw128(qa, 16, 1024), dq1 = sdesc_sw128(qb, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(kb, 16, 1024), dk1 = sdesc_sw128(kb + kTile, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(vb, 16384, 1024), dv1 = sdesc_sw128(vb + kTile, 16384, 1024);
-      // S for sub-tile k of Q tile x: 64 keys (rows 64h.. of K tile k/2) into S slot k%2
-      auto issue_s = [&](int x, int k) {
-        const int h = k & 1, stage = (k >> 1) & 1;
-        const uint32_t d_tmem = tmem + x * 128 + h * 64;
+      // S_x = Q_x K(j)^T over the 128 keys of stage j%2 into Q tile x's 128 S columns
+      auto issue_s = [&](int x, int stage) {
+        const uint32_t d_tmem = tmem + x * 128;
         const uint64_t aq = x == 0 ? dq0 : dq1;
-        const uint64_t bk = (stage == 0 ? dk0 : dk1) + static_cast<uint64_t>((h * 64 * 128) >> 4);
+        const uint64_t bk = stage == 0 ? dk0 : dk1;
 #pragma unroll
         for (int ks = 0; ks < kSteps; ++ks) {
           const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
           mma_ss(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
         }
-        mma_commit(smem_u32(&bars->s_full[x][h]));
+        mma_commit(smem_u32(&bars->s_full[x]));
       };
-      // O_x += P(k) V(k): P is the bf16 pair-packed first 32 columns of S slot k%2
-      auto issue_pv = [&](int x, int k) {
-        const int h = k & 1, stage = (k >> 1) & 1;
+      // O_x += P_x(j) V(j) over keys 64h .. 64h+63: P is bf16 pair-packed in the first 64 columns
+      // of S_x, the keys of half h in columns 32h .. 32h+31
+      auto issue_pv = [&](int x, int stage, int h, bool acc) {
         const uint32_t d_tmem = tmem + 256 + x * 128;
-        const uint32_t p_tmem = tmem + x * 128 + h * 64;
+        const uint32_t p_tmem = tmem + x * 128;
         const uint64_t bv = stage == 0 ? dv0 : dv1;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          mma_ts(d_tmem, p_tmem + ks * 8, bv + static_cast<uint64_t>(((h * 4 + ks) * 2048) >> 4), id_o,
-                 (k > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&bars->pv_done[x]));
+        for (int ks = 4 * h; ks < 4 * h + 4; ++ks)
+          mma_ts(d_tmem, p_tmem + ks * 8, bv + static_cast<uint64_t>((ks * 2048) >> 4), id_o,
+                 (acc || ks > 0) ? 1u : 0u);
       };
-      const int T = (L + 63) / 64;  // 64-key sub-tiles; S slots alternate, so S(k+1) and S(k+2)
-                                    // are computed while the softmax of k runs
       if (ok && T > 0) {
         ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma, wb);
         if (ok) {
           fence_proxy_async_smem();  // the key rows were written by cp.async (generic proxy)
           tc_fence_after();
-          for (int k = 0; k < 2 && k < T; ++k) {
-            issue_s(0, k);
-            if (has_b) issue_s(1, k);
-          }
+          issue_s(0, 0);
+          if (has_b) issue_s(1, 0);
           mma_commit(smem_u32(&bars->k_empty[0]));  // K(0) is not read again
         }
       }
-      for (int k = 0; k < T && ok; ++k) {
-        const int h = k & 1, j = k >> 1, stage = j & 1;
-        ok = mbar_wait(smem_u32(&bars->p_full[0][h]), j & 1, st, kWhereAttnMma, wb);
-        if (ok && h == 0) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma, wb);
+      // Per tile j: PV_A(j) in two halves as the softmax hands them over, S_A(j+1), then the same
+      // for B.  The commit after S_x(j+1) also covers PV_x(j), so when the softmax of x sees
+      // S_x(j+1) it may rescale O_x and reuse its S columns.
+      for (int j = 0; j < T && ok; ++j) {
+        const int stage = j & 1, nstage = (j + 1) & 1;
+        const bool more = j + 1 < T;
+        ok = mbar_wait(smem_u32(&bars->p_full[0][0]), j & 1, st, kWhereAttnMma, wb);
+        if (ok) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma, wb);
         if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_after();
-        issue_pv(0, k);
-        const int k2 = k + 2;
-        const int j2 = k2 >> 1, stage2 = j2 & 1;
-        if (k2 < T) {
-          if ((k2 & 1) == 0) {
-            ok = mbar_wait(smem_u32(&bars->k_full[stage2]), (j2 >> 1) & 1, st, kWhereAttnMma, wb);
-            if (!ok) break;
-            fence_proxy_async_smem();
-            tc_fence_after();
-          }
-          issue_s(0, k2);
+        issue_pv(0, stage, 0, j > 0);
+        ok = mbar_wait(smem_u32(&bars->p_full[0][1]), j & 1, st, kWhereAttnMma, wb);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, stage, 1, true);
+        if (more) {
+          ok = mbar_wait(smem_u32(&bars->k_full[nstage]), ((j + 1) >> 1) & 1, st, kWhereAttnMma, wb);
+          if (!ok) break;
+          fence_proxy_async_smem();
+          tc_fence_after();
+          issue_s(0, nstage);
         }
         if (has_b) {
-          ok = mbar_wait(smem_u32(&bars->p_full[1][h]), j & 1, st, kWhereAttnMma, wb);
+          ok = mbar_wait(smem_u32(&bars->p_full[1][0]), j & 1, st, kWhereAttnMma, wb);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(1, k);
+          issue_pv(1, stage, 0, j > 0);
+          ok = mbar_wait(smem_u32(&bars->p_full[1][1]), j & 1, st, kWhereAttnMma, wb);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, stage, 1, true);
         }
-        if (h == 1 || k == T - 1) mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
-        if (k2 < T) {
-          if (has_b) issue_s(1, k2);
-          if ((k2 & 1) == 1 || k2 == T - 1) mma_commit(smem_u32(&bars->k_empty[stage2]));  // nor K(j2)
+        mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
+        if (more) {
+          if (has_b) issue_s(1, nstage);
+          mma_commit(smem_u32(&bars->k_empty[nstage]));  // nor K(j+1)
         }
       }
       if (ok) mma_commit(smem_u32(&bars->o_full));
@@ -308,41 +318,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(smem_u32(&bars->mma_done), 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
       if (!ok) mbar_wait(qbar, 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
     }
-  } else if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+  } else if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
     // ---------------- key/value gather producer ----------------
-    // Warp w fills rows 32w..32w+31 of each key tile.  Each lane first finds the source row of one
-    // stream position; then every cp.async instruction moves whole rows (16 lanes x 16 bytes per
-    // row at d = 128), so one instruction touches 2 rows instead of 32.
+    // Warp w fills rows 64w'..64w'+63 of each key tile (w' = w - first producer warp).  Each lane
+    // first finds the source rows of two stream positions; then every cp.async instruction moves
+    // whole rows (16 lanes x 16 bytes per row at d = 128), so one instruction touches 2 rows.
     constexpr int CPR = D / 8;       // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;    // rows per warp instruction
-    const int wr0 = (warp - 8) * 32;
+    const int wr0 = (warp - kProducerWarp0) * 64;
     const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
     const size_t head_row0 = static_cast<size_t>(bh) * N;
     const int my_chunk = lane % CPR, my_sub = lane / CPR;
     const int hf = my_chunk >> 3, cc = my_chunk & 7;
-    for (int j = 0; j < nt; ++j) {
-      const int stage = j & 1;
-      int p = j * 128 + wr0 + lane;
+    // source row of stream position p: the largest e with r_cum[e] <= p, then the offset inside it
+    auto src_row = [&](int p) {
       if (p >= L) p = L - 1;
-      // largest e with r_cum[e] <= p
       int lo = 0, hi = nranges - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (r_cum[mid] <= p) lo = mid; else hi = mid - 1;
       }
-      int krow = r_start[lo] + (p - r_cum[lo]);
-      krow = krow < 0 ? 0 : (krow >= N ? N - 1 : krow);
+      const int r = r_start[lo] + (p - r_cum[lo]);
+      return r < 0 ? 0 : (r >= N ? N - 1 : r);
+    };
+    for (int j = 0; j < T; ++j) {
+      const int stage = j & 1;
+      const int krow0 = src_row(j * 128 + wr0 + lane), krow1 = src_row(j * 128 + wr0 + 32 + lane);
       const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
-      // K(j) may land as soon as the last S product of K(j-2) is done, V(j) once PV of V(j-2) is;
-      // each lands asynchronously and counts itself on its full barrier
+      // K(j) may land as soon as both S products of K(j-2) are done, V(j) once both PV products of
+      // V(j-2) are; each lands asynchronously and counts itself on its full barrier
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->k_empty[stage]), ((j >> 1) - 1) & 1, st,
                                                              kWhereAttnProducer, 128, wb)))
         break;
 #pragma unroll
-      for (int it = 0; it < 32 / RPI; ++it) {
-        const int rr = it * RPI + my_sub;  // row within the warp's 32
-        const int src = __shfl_sync(0xffffffffu, krow, rr);
+      for (int it = 0; it < 64 / RPI; ++it) {
+        const int rr = it * RPI + my_sub;  // row within the warp's 64
+        const int src = __shfl_sync(0xffffffffu, rr < 32 ? krow0 : krow1, rr & 31);
         cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * D + my_chunk * 8);
       }
       cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
@@ -350,16 +361,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                                              kWhereAttnProducer, 128, wb)))
         break;
 #pragma unroll
-      for (int it = 0; it < 32 / RPI; ++it) {
+      for (int it = 0; it < 64 / RPI; ++it) {
         const int rr = it * RPI + my_sub;
-        const int src = __shfl_sync(0xffffffffu, krow, rr);
+        const int src = __shfl_sync(0xffffffffu, rr < 32 ? krow0 : krow1, rr & 31);
         cp_async16(vdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Vp + (head_row0 + src) * D + my_chunk * 8);
       }
       cp_async_mbar_arrive(smem_u32(&bars->v_full[stage]));
     }
     cp_async_wait<0>();
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs) : "memory");
     // ---------------- softmax / correction / epilogue for tile X ----------------
     const int x = warp >> 2;
     const int q = warp & 3;
@@ -376,45 +387,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // runs under warp-uniform control flow; per-row decisions only select values.
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
-      const int T = (L + 63) / 64;
-      for (int k = 0; k < T; ++k) {
-        const int h = k & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x][h]), (k >> 1) & 1, st, kWhereAttnSoftmax, wb));
+      for (int j = 0; j < T; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x]), j & 1, st, kWhereAttnSoftmax, wb));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t t_sk = t_s + h * 64;
-        const int valid = min(64, L - k * 64);
-        uint32_t sv[64];
-        tmem_ld32p(t_sk, sv);
-        tmem_ld32p(t_sk + 32, sv + 32);
+        uint32_t sv[128];
+        tmem_ld32p(t_s, sv);
+        tmem_ld32p(t_s + 32, sv + 32);
+        tmem_ld32p(t_s + 64, sv + 64);
+        tmem_ld32p(t_s + 96, sv + 96);
         tmem_wait_ld();
-        if (valid < 64) {  // the key stream's last sub-tile: columns past its end become -inf (p = 0)
+        const int valid = L - j * 128;
+        if (valid < 128) {  // the key stream's last tile: columns past its end become -inf (p = 0)
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
+          for (int e = 0; e < 128; ++e)
             if (e >= valid) sv[e] = __float_as_uint(-INFINITY);
         }
-        // four independent chains of three-input maxima
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // eight independent chains of three-input maxima
+        float m8[8];
 #pragma unroll
-        for (int e = 0; e < 64; e += 8)
+        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            m4[c] = fmax3(m4[c], __uint_as_float(sv[e + 2 * c]), __uint_as_float(sv[e + 2 * c + 1]));
-        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        for (int e = 16; e < 128; e += 16)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            m8[c] = fmax3(m8[c], __uint_as_float(sv[e + 2 * c]), __uint_as_float(sv[e + 2 * c + 1]));
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         const float m_new = fmaxf(m_used, mx * sl2);
         const bool grow = m_new > m_used + kRescaleThreshold;
         float f = 1.f;
         if (grow) {
-          if (k > 0) f = fast_exp2(m_used - m_new);
+          if (j > 0) f = fast_exp2(m_used - m_new);
           l *= f;
           m_used = m_new;
         }
-        if (k > 0 && __any_sync(0xffffffffu, grow)) {
-          // O must hold every PV product up to k-1 before it is rescaled; rows that keep their
-          // max multiply by 1.
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->pv_done[x]), (k - 1) & 1, st, kWhereAttnSoftmax, wb));
-          if (!ok) break;
-          tc_fence_after();
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // S_x(j) has landed, and its commit covers PV_x(j-1): O_x holds every product up to
+          // j-1 and no MMA writes it until this warpgroup hands over P_x(j).  Rows that keep
+          // their max multiply by 1.
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -431,24 +441,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float2 lsum4[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) lsum4[c] = make_float2(0.f, 0.f);
-        uint32_t pk[32];
+        // P goes over in two 64-key halves, so that the first half's PV product runs while the
+        // second half's exponentials are computed
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = 2 * e;
-          const float2 t = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), scl, negm);
-          float2 pe;
-          if ((e & 15) >= 16 - kEmuPerChunk / 2) pe = exp2_poly2(t);
-          else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-          pk[e] = pack_bf16x2(pe.x, pe.y);
-          lsum4[e & 3] = add2(lsum4[e & 3], pe);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = hh * 64 + 2 * e;
+            const float2 t = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), scl, negm);
+            float2 pe;
+            if ((e & 15) >= 16 - kCubicPairs) pe = exp2_cubic2(t);
+            else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            pk[e] = pack_bf16x2(pe.x, pe.y);
+            lsum4[e & 3] = add2(lsum4[e & 3], pe);
+          }
+          tmem_st32(t_s + hh * 32, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x][hh]));
         }
-        tmem_st32(t_sk, pk);
         const float2 ls = add2(add2(lsum4[0], lsum4[1]), add2(lsum4[2], lsum4[3]));
         l += ls.x + ls.y;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x][h]));
       }
       if (ok && T > 0)
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0, st, kWhereAttnSoftmax, wb));
@@ -491,7 +506,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

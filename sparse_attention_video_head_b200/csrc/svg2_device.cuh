@@ -81,8 +81,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on the phase with the given parity.  Gives up (returns false) after `budget`
-// clock cycles, or as soon as the status word shows an error raised anywhere in the grid.
+// Bounded wait on the phase with the given parity.  Gives up (returns false) once `budget` clock
+// cycles have passed since the first unsuccessful poll (checked after every poll), or as soon as
+// the status word, read every 64 polls, shows an error raised anywhere in the grid.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceStatus* st,
                                           uint32_t where, long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -90,13 +91,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceS
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 63u) == 0u) {
-      if (status_set(st)) return false;
-      if (clock64() - t0 > budget) {
-        raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
-        return false;
-      }
+    if (clock64() - t0 > budget) {
+      raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
+      return false;
     }
+    if ((++spins & 63u) == 0u && status_set(st)) return false;
   }
 }
 
@@ -120,13 +119,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   uint32_t spins = 0;
   while (true) {
     if (poll()) return true;
-    if ((++spins & 63u) == 0u) {
-      if (status_set(st)) return false;
-      if (clock64() - t0 > budget) {
-        raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
-        return false;
-      }
+    if (clock64() - t0 > budget) {
+      raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
+      return false;
     }
+    if ((++spins & 63u) == 0u && status_set(st)) return false;
   }
 }
 
@@ -141,13 +138,11 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, D
   while (true) {
     __nanosleep(ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 15u) == 0) {
-      if (status_set(st)) return false;
-      if (clock64() - t0 > budget) {
-        raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
-        return false;
-      }
+    if (clock64() - t0 > budget) {
+      raise_status(st, kStatusDeviceTimeout, where, blockIdx.x, threadIdx.x);
+      return false;
     }
+    if ((++spins & 15u) == 0 && status_set(st)) return false;
   }
 }
 
@@ -299,23 +294,24 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x for a pair of floats on the FMA/ALU pipes (no MUFU).  Range reduction x = n + f with
-// n = round(x) (by adding 1.5 * 2^23), f in [-1/2, 1/2]; 2^f from a cubic fitted here for minimum
-// relative error on [-1/2, 1/2] (max 7.5e-5, far below bf16's 2^-9); 2^n is added to the
-// exponent field.  x is clamped at -125, where the result (~2e-38) is zero for the softmax.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 j = add2(x, magic);
-  const float2 n = add2(j, make_float2(-12582912.0f, -12582912.0f));
+// 2^x for a pair of floats on the FMA and ALU pipes instead of the MUFU.  x = n + f with n the
+// nearest integer (the rounding of x + 1.5 * 2^23 puts it in the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f is the cubic of least maximum relative error on that interval (fitted here by
+// iteratively reweighted least squares: 7.5e-5 in float32, far below the bf16 rounding of P), and
+// 2^n enters by adding n to the exponent field.  x is clamped at -126, where 2^x is below every
+// other term of a softmax row.
+__device__ __forceinline__ float2 exp2_cubic2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = add2(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = add2(t, make_float2(-12582912.f, -12582912.f));
   const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = fma2(make_float2(0.0551716610789299f, 0.0551716610789299f), f,
-                  make_float2(0.2426111400127411f, 0.2426111400127411f));
+  float2 p = fma2(make_float2(0.05517150089144707f, 0.05517150089144707f), f,
+                  make_float2(0.24261096119880676f, 0.24261096119880676f));
   p = fma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
   p = fma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
+  return make_float2(__uint_as_float(__float_as_uint(t.x) * 8388608u + __float_as_uint(p.x)),
+                     __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(p.y)));
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
