@@ -58,9 +58,12 @@ typedef enum { SVG2_BF16 = 0, SVG2_F32 = 1 } svg2_dtype;
  * previous denoising step's centroids.  KMEANSPP: k-means++ seeding from the data (Method (1)). */
 typedef enum { SVG2_INIT_GIVEN = 0, SVG2_INIT_KMEANSPP = 1 } svg2_init;
 
-/* k-means++ seeding looks at every stride-th token, stride = ceil(N / seed_tokens), so that at most
- * seed_tokens tokens are candidates (0 = all tokens).  The Lloyd iterations always use all tokens.
- * This default keeps the seeding cheap on video-length layers. */
+/* k-means++ seeding looks at S = seed_tokens candidate tokens (0, or seed_tokens >= N: all N tokens):
+ * one per stratum of the token order, stratum j = [floor(j N / S), floor((j + 1) N / S)), at offset
+ * floor(r_j w_j / 2^32) inside it, w_j its width and r_j = (j * 2654435769) mod 2^32.  The offsets
+ * vary from stratum to stratum, so the candidates do not line up with the rows and columns of the
+ * video grid the tokens come from.  The Lloyd iterations always use all tokens.  This default keeps
+ * the seeding cheap on video-length layers. */
 #define SVG2_DEFAULT_SEED_TOKENS 16384
 
 /* Largest sizes the library supports.  Besides these, B*H <= 2^20 and B*H*N < 2^31 (token rows
@@ -104,8 +107,8 @@ SVG2_API int svg2_set_wait_budget(void* ws, uint64_t cycles, void* stream);
  *   init       SVG2_INIT_GIVEN (centroids holds the start, e.g. the previous step's cache) or
  *              SVG2_INIT_KMEANSPP (seeding from the data; `u` must then hold B*H*k uniforms in
  *              [0,1), float64, one per seed, and seeds are chosen by fixed-point D^2 sampling).
- *   seed_tokens  k-means++ candidates: every ceil(N / seed_tokens)-th token (0 = all tokens; see
- *              SVG2_DEFAULT_SEED_TOKENS); the candidate count must be >= k.
+ *   seed_tokens  k-means++ candidates: seed_tokens tokens, one per stratum of the token order (0 =
+ *              all tokens; see SVG2_DEFAULT_SEED_TOKENS); the candidate count must be >= k.
  *   centroids  float32 [B, H, k, d], in (GIVEN) and out (final centroids).
  *   labels     int32 [B, H, N], out: labels of the last assignment (the ones the final centroids
  *              were computed from).
@@ -123,7 +126,7 @@ SVG2_API int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, i
  * Per (b, h): seed 0 is candidate floor(u_0 * S); seed s is the first candidate whose running sum
  * of floor(D^2 / M0 * 2^32) exceeds floor(u_s * U), where D^2 is the float64 squared distance to
  * the nearest earlier seed, M0 the largest D^2 after seed 0 and U the sum of all weights (a
- * uniform pick when U = 0).  Candidates are every ceil(N / seed_tokens)-th token (0 = all).
+ * uniform pick when U = 0).  Candidates as in SVG2_DEFAULT_SEED_TOKENS's note (0 = all tokens).
  *   u          float64 [B, H, k] uniforms in [0, 1).
  *   centroids  float32 [B, H, k, d], out: the seed rows.
  * Same sizes, dtype and workspace rules as svg2_kmeans; the candidate count must be >= k. */

@@ -171,19 +171,32 @@ def dense_attention_rows(Q, K, V, scale, rows=None):
     return out
 
 
-def seed_stride(N: int, seed_tokens: int) -> int:
-    """k-means++ candidates are every stride-th token so that at most seed_tokens are used (0 = all)."""
+def seed_candidates(N: int, seed_tokens: int) -> np.ndarray:
+    """Token indices of the k-means++ candidates, ascending.
+
+    0 or seed_tokens >= N: every token.  Otherwise S = seed_tokens candidates, one per stratum:
+    stratum j covers tokens [floor(j N / S), floor((j + 1) N / S)) and its candidate sits at offset
+    floor(r_j w_j / 2^32) inside it, w_j its width and r_j = (j * 2654435769) mod 2^32 (a
+    multiplicative hash by the golden ratio), all in exact integer arithmetic.  The spacing thus
+    varies from stratum to stratum, so the candidates cannot line up with the rows or columns of
+    the video grid the tokens are flattened from (a fixed stride that divides the row length would
+    see only some columns)."""
     if seed_tokens <= 0 or seed_tokens >= N:
-        return 1
-    return -(-N // seed_tokens)
+        return np.arange(N, dtype=np.int64)
+    S = np.uint64(seed_tokens)
+    j = np.arange(seed_tokens, dtype=np.uint64)
+    lo = (j * np.uint64(N)) // S
+    hi = ((j + np.uint64(1)) * np.uint64(N)) // S
+    r = (j * np.uint64(2654435769)) & np.uint64(0xFFFFFFFF)
+    return (lo + ((r * (hi - lo)) >> np.uint64(32))).astype(np.int64)
 
 
 def kmeans(X: np.ndarray, k: int, iters: int, u: Optional[np.ndarray] = None,
            C0: Optional[np.ndarray] = None, seed_tokens: int = 0):
-    """k-means++ seeding on the candidate tokens X[::stride] (or the given C0), then `iters` Lloyd
-    iterations over all tokens."""
+    """k-means++ seeding on the candidate tokens X[seed_candidates(N, seed_tokens)] (or the given
+    C0), then `iters` Lloyd iterations over all tokens."""
     if C0 is None:
-        _, C0 = kmeanspp(np.ascontiguousarray(X[::seed_stride(X.shape[0], seed_tokens)]), k, u)
+        _, C0 = kmeanspp(np.ascontiguousarray(X[seed_candidates(X.shape[0], seed_tokens)]), k, u)
     return lloyd(X, C0, iters)
 
 

@@ -98,16 +98,30 @@ void carve_layer(Carve& c, int BH, int N, int d, int nQ, int nK, const svg2_laye
   carve_attn(c, BH, N, nQ, L.attn);
 }
 
+// Bytes from the start of the permuted Q plane to the end of the permuted K plane: both are free
+// during the k-means (the gathers fill them afterwards), so the k-means++ candidate rows (at most
+// two bytes per element more than one bf16 plane, for float32 inputs) are copied there.
+size_t candidate_room(const LayerCarve& L, int BH, int N, int d) {
+  return static_cast<size_t>(reinterpret_cast<const char*>(L.Kp) - reinterpret_cast<const char*>(L.Qp)) +
+         static_cast<size_t>(BH) * N * d * sizeof(uint16_t);
+}
+
+// cand / cand_bytes: room for the compact copy of the k-means++ candidate rows (kmeanspp_candidate_bytes).
 cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int iters, int init, const double* u,
                        int seed_tokens, float* C, int32_t* labels, int32_t* counts, int32_t* perm, int32_t* offsets,
-                       const KmeansScratch& s, DeviceStatus* st, cudaStream_t stream) {
+                       const KmeansScratch& s, void* cand, size_t cand_bytes, DeviceStatus* st, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
   if (init == SVG2_INIT_KMEANSPP)
-    e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, s.c_hi, seed_tokens, st, stream);
+    e = launch_kmeanspp(X, f32, BH, N, d, k, u, C, s.pp_dist, s.pp_near, s.c_hi, seed_tokens, cand, cand_bytes, st,
+                        stream);
   if (e == cudaSuccess) e = launch_centroid_prep(C, BH, k, d, s.c_hi, s.c_lo, s.c_norm, stream);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-    e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, s.rr_list, s.rr_count, st,
-                      wait_budget_of(st), stream);
+    // after the first iteration, perm holds the stable sort of the previous labels: the pruned search
+    if (it > 0 && s.d2 != nullptr && !f32 && d == 128)
+      e = launch_assign_pruned(X, BH, N, k, C, perm, s.d2, labels, stream);
+    else
+      e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, s.rr_list, s.rr_count, st,
+                        wait_budget_of(st), stream);
     if (e == cudaSuccess) e = launch_sort(labels, BH, N, k, perm, offsets, counts, s.chunk_hist, st, stream);
     if (e == cudaSuccess) e = launch_update(X, f32, BH, N, d, k, perm, offsets, C, s.c_hi, s.c_lo, s.c_norm, stream);
   }
@@ -220,16 +234,18 @@ int svg2_kmeanspp(const void* X, int dtype, int B, int H, int N, int d, int k, c
     if (!valid_dtype(dtype) || X == nullptr || u == nullptr || centroids == nullptr || seed_tokens < 0)
       return SVG2_ERR_INVALID_ARG;
     if (!aligned(X, 16) || !aligned(centroids, 16)) return SVG2_ERR_INVALID_ARG;
-    if ((N + kmeanspp_stride(N, seed_tokens) - 1) / kmeanspp_stride(N, seed_tokens) < k) return SVG2_ERR_INVALID_ARG;
+    if (kmeanspp_candidates(N, seed_tokens) < k) return SVG2_ERR_INVALID_ARG;  // fewer candidates than seeds
     const int BH = B * H;
     Carve c(ws);
     DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
     KmeansScratch s;
     carve_kmeans(c, BH, N, d, k, s, false);
+    const size_t cand_bytes = kmeanspp_candidate_bytes(BH, N, d, dtype == SVG2_F32, seed_tokens);
+    void* cand = c.take<uint8_t>(cand_bytes);
     r = check_ws(ws, ws_bytes, c.off);
     if (r != SVG2_OK) return r;
     return to_status(launch_kmeanspp(X, dtype == SVG2_F32, BH, N, d, k, u, centroids, s.pp_dist, s.pp_near,
-                                     s.c_hi, seed_tokens, st, static_cast<cudaStream_t>(stream)));
+                                     s.c_hi, seed_tokens, cand, cand_bytes, st, static_cast<cudaStream_t>(stream)));
   } catch (...) {
     return SVG2_ERR_CUDA;
   }
@@ -250,17 +266,20 @@ int svg2_kmeans(const void* X, int dtype, int B, int H, int N, int d, int k, int
     const int BH = B * H;
     Carve c(ws);
     DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+    if (seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
+    if (init == SVG2_INIT_KMEANSPP && kmeanspp_candidates(N, seed_tokens) < k)
+      return SVG2_ERR_INVALID_ARG;  // fewer candidates than seeds
     KmeansScratch s;
     carve_kmeans(c, BH, N, d, k, s, perm == nullptr);
+    const size_t cand_bytes =
+        init == SVG2_INIT_KMEANSPP ? kmeanspp_candidate_bytes(BH, N, d, dtype == SVG2_F32, seed_tokens) : 0;
+    void* cand = c.take<uint8_t>(cand_bytes);
     r = check_ws(ws, ws_bytes, c.off);
     if (r != SVG2_OK) return r;
     if (perm == nullptr) perm = s.perm;
     if (offsets == nullptr) offsets = s.offsets;
-    if (seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
-    if (init == SVG2_INIT_KMEANSPP && (N + kmeanspp_stride(N, seed_tokens) - 1) / kmeanspp_stride(N, seed_tokens) < k)
-      return SVG2_ERR_INVALID_ARG;  // fewer candidates than seeds
     return to_status(run_kmeans(X, dtype == SVG2_F32, BH, N, d, k, iters, init, u, seed_tokens, centroids, labels, counts, perm,
-                                offsets, s, st, static_cast<cudaStream_t>(stream)));
+                                offsets, s, cand, cand_bytes, st, static_cast<cudaStream_t>(stream)));
   } catch (...) {
     return SVG2_ERR_CUDA;
   }
@@ -451,10 +470,8 @@ static int check_layer_params(const svg2_params* p, int dtype, int B, int H, int
   if (!valid_dtype(dtype) || p->iters < 1 || (p->init != SVG2_INIT_GIVEN && p->init != SVG2_INIT_KMEANSPP))
     return SVG2_ERR_INVALID_ARG;
   if (p->seed_tokens < 0) return SVG2_ERR_INVALID_ARG;
-  if (p->init == SVG2_INIT_KMEANSPP) {
-    const int stride = kmeanspp_stride(N, p->seed_tokens);
-    if ((N + stride - 1) / stride < (p->nQ > p->nK ? p->nQ : p->nK)) return SVG2_ERR_INVALID_ARG;
-  }
+  if (p->init == SVG2_INIT_KMEANSPP && kmeanspp_candidates(N, p->seed_tokens) < (p->nQ > p->nK ? p->nQ : p->nK))
+    return SVG2_ERR_INVALID_ARG;  // fewer candidates than seeds
   if (!(p->top_p > 0.f) || p->scale != p->scale) return SVG2_ERR_INVALID_ARG;
   if (cq == nullptr || ck == nullptr) return SVG2_ERR_INVALID_ARG;
   if (p->init == SVG2_INIT_KMEANSPP && (uq == nullptr || uk == nullptr)) return SVG2_ERR_INVALID_ARG;
@@ -479,11 +496,14 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
     if (r != SVG2_OK) return r;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f32 = dtype == SVG2_F32;
+    // the permuted planes are free until the gathers: the k-means++ candidates are copied there
+    void* cand = L.Qp;
+    const size_t cand_bytes = candidate_room(L, BH, N, d);
     cudaError_t e = run_kmeans(Q, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q, L.perm_q,
-                               L.q_off, L.kq, L.st, s);
+                               L.q_off, L.kq, cand, cand_bytes, L.st, s);
     if (e == cudaSuccess)
       e = run_kmeans(K, f32, BH, N, d, p->nK, p->iters, p->init, uk, p->seed_tokens, ck, L.labels_k, L.count_k, L.perm_k, L.k_off,
-                     L.kk, L.st, s);
+                     L.kk, cand, cand_bytes, L.st, s);
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, L.weights, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);
@@ -615,12 +635,12 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
         e = run_kmeans(static_cast<const char*>(Kd) + hb * plane_in, f32, hnc, N, d, p->nK, p->iters, p->init,
                        uk != nullptr ? uk + hb * p->nK : nullptr, p->seed_tokens, ck + hb * p->nK * d,
                        L.labels_k + hb * N, L.count_k + hb * p->nK, L.perm_k + hb * N, L.k_off + hb * (p->nK + 1),
-                       L.kk, L.st, s);
+                       L.kk, L.Qp, candidate_room(L, BH, N, d), L.st, s);
     }
     ok(cudaStreamWaitEvent(s, q_in, 0));
     if (e == cudaSuccess)
       e = run_kmeans(Qd, f32, BH, N, d, p->nQ, p->iters, p->init, uq, p->seed_tokens, cq, L.labels_q, L.count_q,
-                     L.perm_q, L.q_off, L.kq, L.st, s);
+                     L.perm_q, L.q_off, L.kq, L.Qp, candidate_room(L, BH, N, d), L.st, s);
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, nullptr, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);

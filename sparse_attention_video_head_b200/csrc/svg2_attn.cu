@@ -56,7 +56,8 @@ constexpr int kCubicPairs = 4;
 
 struct AttnBars {
   uint64_t q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], o_full, mma_done;
-  uint64_t s_full[2], p_full[2][2];  // per Q tile; P in two 64-key halves
+  uint64_t s_full[2], p_full[2][2];  // per Q tile (ring mode: per S slot); P in two 64-key halves
+  uint64_t pv_done;                  // ring mode: one phase per PV product
   uint32_t tmem_base;
   int32_t L;
   int32_t nranges;
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->mma_done), 1);
+    mbar_init(smem_u32(&bars->pv_done), 1);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -241,9 +243,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = sdesc_sw128(qa, 16, 1024), dq1 = sdesc_sw128(qb, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(kb, 16, 1024), dk1 = sdesc_sw128(kb + kTile, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(vb, 16384, 1024), dv1 = sdesc_sw128(vb + kTile, 16384, 1024);
-      // S_x = Q_x K(j)^T over the 128 keys of stage j%2 into Q tile x's 128 S columns
-      auto issue_s = [&](int x, int stage) {
-        const uint32_t d_tmem = tmem + x * 128;
+      // S = Q_x K(j)^T over the 128 keys of stage j%2 into the 128 S columns of slot `slot`
+      // (slot = x, or in ring mode the slot of tile j); announced on s_full[slot]
+      auto issue_s = [&](int x, int stage, int slot) {
+        const uint32_t d_tmem = tmem + slot * 128;
         const uint64_t aq = x == 0 ? dq0 : dq1;
         const uint64_t bk = stage == 0 ? dk0 : dk1;
 #pragma unroll
@@ -251,13 +254,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
           mma_ss(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
         }
-        mma_commit(smem_u32(&bars->s_full[x]));
+        mma_commit(smem_u32(&bars->s_full[slot]));
       };
-      // O_x += P_x(j) V(j) over keys 64h .. 64h+63: P is bf16 pair-packed in the first 64 columns
-      // of S_x, the keys of half h in columns 32h .. 32h+31
-      auto issue_pv = [&](int x, int stage, int h, bool acc) {
+      // O_x += P(j) V(j) over keys 64h .. 64h+63: P is bf16 pair-packed in the first 64 columns
+      // of its S slot, the keys of half h in columns 32h .. 32h+31
+      auto issue_pv = [&](int x, int slot, int stage, int h, bool acc) {
         const uint32_t d_tmem = tmem + 256 + x * 128;
-        const uint32_t p_tmem = tmem + x * 128;
+        const uint32_t p_tmem = tmem + slot * 128;
         const uint64_t bv = stage == 0 ? dv0 : dv1;
 #pragma unroll
         for (int ks = 4 * h; ks < 4 * h + 4; ++ks)
@@ -269,15 +272,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ok) {
           fence_proxy_async_smem();  // the key rows were written by cp.async (generic proxy)
           tc_fence_after();
-          issue_s(0, 0);
-          if (has_b) issue_s(1, 0);
+          issue_s(0, 0, 0);
+          if (has_b) issue_s(1, 0, 1);
           mma_commit(smem_u32(&bars->k_empty[0]));  // K(0) is not read again
+        }
+      }
+      if (!has_b) {
+        // Ring mode (one Q tile): S(j) goes to slot j%2, the unused tile's columns serving as the
+        // second slot, so S(j+1) is computed while the softmax of j runs.  Order: S(0), S(1), then
+        // per tile PV(j) in two halves and S(j+2) into the slot PV(j) has just read.  pv_done marks
+        // each PV product (the S commits no longer cover the latest one).
+        if (ok && T > 1) {
+          ok = mbar_wait(smem_u32(&bars->k_full[1]), 0, st, kWhereAttnMma, wb);
+          if (ok) {
+            fence_proxy_async_smem();
+            tc_fence_after();
+            issue_s(0, 1, 1);
+            mma_commit(smem_u32(&bars->k_empty[1]));
+          }
+        }
+        for (int j = 0; j < T && ok; ++j) {
+          const int stage = j & 1;
+          ok = mbar_wait(smem_u32(&bars->p_full[0][0]), j & 1, st, kWhereAttnMma, wb);
+          if (ok) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma, wb);
+          if (!ok) break;
+          fence_proxy_async_smem();
+          tc_fence_after();
+          issue_pv(0, stage, stage, 0, j > 0);
+          ok = mbar_wait(smem_u32(&bars->p_full[0][1]), j & 1, st, kWhereAttnMma, wb);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(0, stage, stage, 1, true);
+          mma_commit(smem_u32(&bars->pv_done));
+          mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
+          if (j + 2 < T) {
+            ok = mbar_wait(smem_u32(&bars->k_full[stage]), ((j + 2) >> 1) & 1, st, kWhereAttnMma, wb);
+            if (!ok) break;
+            fence_proxy_async_smem();
+            tc_fence_after();
+            issue_s(0, stage, stage);
+            mma_commit(smem_u32(&bars->k_empty[stage]));  // nor K(j+2)
+          }
         }
       }
       // Per tile j: PV_A(j) in two halves as the softmax hands them over, S_A(j+1), then the same
       // for B.  The commit after S_x(j+1) also covers PV_x(j), so when the softmax of x sees
       // S_x(j+1) it may rescale O_x and reuse its S columns.
-      for (int j = 0; j < T && ok; ++j) {
+      for (int j = 0; j < T && ok && has_b; ++j) {
         const int stage = j & 1, nstage = (j + 1) & 1;
         const bool more = j + 1 < T;
         ok = mbar_wait(smem_u32(&bars->p_full[0][0]), j & 1, st, kWhereAttnMma, wb);
@@ -285,31 +326,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_after();
-        issue_pv(0, stage, 0, j > 0);
+        issue_pv(0, 0, stage, 0, j > 0);
         ok = mbar_wait(smem_u32(&bars->p_full[0][1]), j & 1, st, kWhereAttnMma, wb);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(0, stage, 1, true);
+        issue_pv(0, 0, stage, 1, true);
         if (more) {
           ok = mbar_wait(smem_u32(&bars->k_full[nstage]), ((j + 1) >> 1) & 1, st, kWhereAttnMma, wb);
           if (!ok) break;
           fence_proxy_async_smem();
           tc_fence_after();
-          issue_s(0, nstage);
+          issue_s(0, nstage, 0);
         }
-        if (has_b) {
-          ok = mbar_wait(smem_u32(&bars->p_full[1][0]), j & 1, st, kWhereAttnMma, wb);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, stage, 0, j > 0);
-          ok = mbar_wait(smem_u32(&bars->p_full[1][1]), j & 1, st, kWhereAttnMma, wb);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, stage, 1, true);
-        }
+        ok = mbar_wait(smem_u32(&bars->p_full[1][0]), j & 1, st, kWhereAttnMma, wb);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, 1, stage, 0, j > 0);
+        ok = mbar_wait(smem_u32(&bars->p_full[1][1]), j & 1, st, kWhereAttnMma, wb);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, 1, stage, 1, true);
         mma_commit(smem_u32(&bars->v_empty[stage]));  // V(j) is not read again
         if (more) {
-          if (has_b) issue_s(1, nstage);
+          issue_s(1, nstage, 1);
           mma_commit(smem_u32(&bars->k_empty[nstage]));  // nor K(j+1)
         }
       }
@@ -380,22 +419,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // nothing to do
     } else {
       const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-      const uint32_t t_s = tmem + lane_off + x * 128;
       const uint32_t t_o = tmem + lane_off + 256 + x * 128;
       const float sl2 = scale * kLog2e;
       // Every tcgen05.ld/st below is a warp-collective (.sync.aligned) instruction, so all of it
       // runs under warp-uniform control flow; per-row decisions only select values.
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
+      // ring mode (no tile B): S(j) in slot j%2 (parity j/2 of that slot's barrier)
+      const bool ring = !has_b;
       for (int j = 0; j < T; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[x]), j & 1, st, kWhereAttnSoftmax, wb));
+        const int slot = ring ? (j & 1) : x;
+        const uint32_t par = ring ? ((j >> 1) & 1) : (j & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[slot]), par, st, kWhereAttnSoftmax, wb));
         if (!ok) break;
         tc_fence_after();
+        const uint32_t t_sj = tmem + lane_off + slot * 128;
         uint32_t sv[128];
-        tmem_ld32p(t_s, sv);
-        tmem_ld32p(t_s + 32, sv + 32);
-        tmem_ld32p(t_s + 64, sv + 64);
-        tmem_ld32p(t_s + 96, sv + 96);
+        tmem_ld32p(t_sj, sv);
+        tmem_ld32p(t_sj + 32, sv + 32);
+        tmem_ld32p(t_sj + 64, sv + 64);
+        tmem_ld32p(t_sj + 96, sv + 96);
         tmem_wait_ld();
         const int valid = L - j * 128;
         if (valid < 128) {  // the key stream's last tile: columns past its end become -inf (p = 0)
@@ -422,9 +465,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_used = m_new;
         }
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // S_x(j) has landed, and its commit covers PV_x(j-1): O_x holds every product up to
-          // j-1 and no MMA writes it until this warpgroup hands over P_x(j).  Rows that keep
-          // their max multiply by 1.
+          // O_x must hold every PV product up to j-1, and no MMA writes it until this warpgroup
+          // hands over P_x(j).  With two tiles the commit announcing S_x(j) covers PV_x(j-1); in
+          // ring mode S(j) was issued before PV(j-1), so that product is awaited on pv_done.
+          // Rows that keep their max multiply by 1.
+          if (ring) {
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&bars->pv_done), (j - 1) & 1, st, kWhereAttnSoftmax, wb));
+            if (!ok) break;
+            tc_fence_after();
+          }
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -456,7 +506,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pk[e] = pack_bf16x2(pe.x, pe.y);
             lsum4[e & 3] = add2(lsum4[e & 3], pe);
           }
-          tmem_st32(t_s + hh * 32, pk);
+          tmem_st32(t_sj + hh * 32, pk);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();

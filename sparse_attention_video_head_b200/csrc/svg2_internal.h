@@ -53,6 +53,10 @@ inline const uint64_t* wait_budget_of(const DeviceStatus* st) {
 constexpr int kSortChunks = 32;  // token chunks per (b,h) in the stable counting sort
 constexpr int kAssignTileM = 128;
 constexpr int kAssignChunkN = 128;  // centroids per MMA chunk
+constexpr int kMaxClustersAssign = 1024;  // == SVG2_MAX_CLUSTERS
+// From this many clusters on, the Lloyd iterations after the first use the pruned assignment
+// (centroid-to-centroid distances exclude most clusters per tile of label-ordered tokens).
+constexpr int kPrunedMinK = 256;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int kpad_of(int k) { return (k + kAssignChunkN - 1) / kAssignChunkN * kAssignChunkN; }
@@ -83,6 +87,7 @@ struct KmeansScratch {
   int32_t* offsets;   // [BH, k+1]
   uint4* rr_list;     // [BH * N] tokens whose assignment the exact re-rank decides: {bh, n, c0|c1, c2|c3}
   uint32_t* rr_count; // entries in rr_list
+  float* d2;          // [BH, k, k] centroid-to-centroid squared distances (k >= kPrunedMinK only)
 };
 
 inline void carve_kmeans(Carve& c, int BH, int N, int d, int k, KmeansScratch& s, bool need_perm) {
@@ -97,6 +102,7 @@ inline void carve_kmeans(Carve& c, int BH, int N, int d, int k, KmeansScratch& s
   s.offsets = c.take<int32_t>(static_cast<size_t>(BH) * (k + 1));
   s.rr_list = c.take<uint4>(static_cast<size_t>(BH) * N);
   s.rr_count = c.take<uint32_t>(1);
+  s.d2 = k >= kPrunedMinK ? c.take<float>(static_cast<size_t>(BH) * k * k) : nullptr;
 }
 
 // Attention work plan: one unit = up to two 128-row Q tiles of one Q cluster.
@@ -131,22 +137,31 @@ cudaError_t launch_gather2(const void* X0, const void* X1, bool x_f32, const int
 cudaError_t launch_unpermute(const void* Op, const int32_t* perm, int BH, int N, int d, void* O,
                              cudaStream_t s);
 
+// k-means++ seeding over the candidates kmeanspp_candidates() counts; when they are fewer than the
+// tokens, their rows are first copied into `cand` (at least kmeanspp_candidate_bytes() bytes).
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
                             float* centroids, double* dist, int32_t* near, uint16_t* seeds_bf16, int seed_tokens,
-                            DeviceStatus* st, cudaStream_t s);
+                            void* cand, size_t cand_bytes, DeviceStatus* st, cudaStream_t s);
 // k-means++ seeding on the tensor cores (bf16, d = 128); returns cudaErrorNotSupported for shapes
 // it does not take, so that the caller can use the CUDA-core kernels.
 // seeds_bf16: scratch of BH * k * d bf16 (the seeds' rows, for the seed-to-seed distances).
 cudaError_t launch_kmeanspp_tc(const void* X, int BH, int N, int stride, int S, int k, const double* u,
                                float* centroids, uint16_t* seeds_bf16, DeviceStatus* st, cudaStream_t s);
-// Spacing of the k-means++ candidates: every stride-th token, so that at most seed_tokens are used.
-int kmeanspp_stride(int N, int seed_tokens);
+// Number of k-means++ candidates: seed_tokens of the N tokens (one per stratum of the token order),
+// or all N when seed_tokens is 0 or at least N.
+int kmeanspp_candidates(int N, int seed_tokens);
+// Bytes of the compact candidate copy the seeding needs (0 when every token is a candidate).
+size_t kmeanspp_candidate_bytes(int BH, int N, int d, bool x_f32, int seed_tokens);
 cudaError_t launch_centroid_prep(const float* centroids, int BH, int k, int d, uint16_t* c_hi, uint16_t* c_lo,
                                  float* c_norm, cudaStream_t s);
 cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k, const float* centroids,
                           const uint16_t* c_hi, const uint16_t* c_lo, const float* c_norm, int32_t* labels,
                           uint4* rr_list, uint32_t* rr_count, DeviceStatus* st, const uint64_t* wait_budget,
                           cudaStream_t s);
+// Lloyd assignment from the previous iteration's stable sort `perm` (bf16 X, d = 128, k <= 1024):
+// the centroid-to-centroid table into d2 [BH, k, k], then the pruned exact search per tile.
+cudaError_t launch_assign_pruned(const void* X, int BH, int N, int k, const float* centroids, const int32_t* perm,
+                                 float* d2, int32_t* labels, cudaStream_t s);
 cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
                           const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
                           float* c_norm, cudaStream_t s);

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(1024, 1) kmeanspp_kernel(const void* __restric
                                                             int d, int k, const double* __restrict__ u,
                                                             float* __restrict__ C, double* __restrict__ Dg,
                                                             int32_t* __restrict__ Ag) {
-  const int N = (Ntok + stride - 1) / stride;  // candidates: every stride-th token
+  const int N = (Ntok + stride - 1) / stride;  // candidates: every stride-th row (the launcher passes 1)
   __shared__ float cs[128];
   __shared__ float ss[1024];
   __shared__ unsigned long long warp_buf[33];
@@ -1320,26 +1320,74 @@ cudaError_t launch_pp(const void* X, int BH, int N, int stride, int S, int k, co
   return cudaLaunchKernelEx(&L.cfg, kern, X, N, stride, S, k, u, C);
 }
 
-int kmeanspp_stride(int N, int seed_tokens) {
-  if (seed_tokens <= 0 || seed_tokens >= N) return 1;
-  return (N + seed_tokens - 1) / seed_tokens;
+int kmeanspp_candidates(int N, int seed_tokens) {
+  return (seed_tokens <= 0 || seed_tokens >= N) ? N : seed_tokens;
+}
+
+namespace {
+
+// Token of k-means++ candidate j of S < N: one candidate per stratum [floor(j N / S),
+// floor((j + 1) N / S)), at offset floor(r w / 2^32) inside it, w the stratum's width and
+// r = (j * 2654435769) mod 2^32, a multiplicative hash by the golden ratio.  The offsets vary from
+// stratum to stratum, so the candidates do not line up with the video grid's rows and columns.
+__device__ __forceinline__ int candidate_token(int j, int N, int S) {
+  const unsigned long long lo = static_cast<unsigned long long>(j) * N / S;
+  const unsigned long long hi = static_cast<unsigned long long>(j + 1) * N / S;
+  const unsigned long long r = static_cast<unsigned int>(static_cast<unsigned int>(j) * 2654435769u);
+  return static_cast<int>(lo + ((r * (hi - lo)) >> 32));
+}
+
+// Copies the candidate rows of every (b,h) plane into a compact [BH, S, row] buffer, 16 bytes per
+// thread and iteration.
+__global__ void gather_candidates_kernel(const uint4* __restrict__ X, int N, int S, int vec_per_row,
+                                         long long total_vecs, uint4* __restrict__ Xc) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total_vecs;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / vec_per_row;
+    const int v = static_cast<int>(i - r * vec_per_row);
+    const long long bh = r / S;
+    const int j = static_cast<int>(r - bh * S);
+    const int n = candidate_token(j, N, S);
+    Xc[i] = __ldg(X + (bh * N + n) * vec_per_row + v);
+  }
+}
+
+}  // namespace
+
+size_t kmeanspp_candidate_bytes(int BH, int N, int d, bool x_f32, int seed_tokens) {
+  const int S = kmeanspp_candidates(N, seed_tokens);
+  return S < N ? static_cast<size_t>(BH) * S * d * (x_f32 ? 4 : 2) : 0;
 }
 
 cudaError_t launch_kmeanspp(const void* X, bool x_f32, int BH, int N, int d, int k, const double* u,
                             float* centroids, double* dist, int32_t* near, uint16_t* seeds_bf16, int seed_tokens,
-                            DeviceStatus* st, cudaStream_t s) {
-  const int stride = kmeanspp_stride(N, seed_tokens);
-  const int S = (N + stride - 1) / stride;
+                            void* cand, size_t cand_bytes, DeviceStatus* st, cudaStream_t s) {
+  const int S = kmeanspp_candidates(N, seed_tokens);
+  const void* Xs = X;
+  int Ns = N;
+  if (S < N) {  // seed on the compact copy of the candidate rows
+    const size_t need = kmeanspp_candidate_bytes(BH, N, d, x_f32, seed_tokens);
+    if (cand == nullptr || cand_bytes < need) return cudaErrorInvalidValue;
+    const int vec_per_row = d * (x_f32 ? 4 : 2) / 16;
+    const long long total = static_cast<long long>(BH) * S * vec_per_row;
+    const long long blocks = (total + 255) / 256;
+    gather_candidates_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, s>>>(
+        static_cast<const uint4*>(X), N, S, vec_per_row, total, static_cast<uint4*>(cand));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    Xs = cand;
+    Ns = S;
+  }
   if (!x_f32 && d == 128) {
-    const cudaError_t e = launch_kmeanspp_tc(X, BH, N, stride, S, k, u, centroids, seeds_bf16, st, s);
+    const cudaError_t e = launch_kmeanspp_tc(Xs, BH, Ns, 1, S, k, u, centroids, seeds_bf16, st, s);
     if (e != cudaErrorNotSupported) return e;
   }
   if ((S + kPpMaxCluster - 1) / kPpMaxCluster <= kPpMaxPerCta && !(x_f32 && d == 128)) {
-    if (d == 128) return launch_pp<4, false>(X, BH, N, stride, S, k, u, centroids, s);
-    return x_f32 ? launch_pp<2, true>(X, BH, N, stride, S, k, u, centroids, s)
-                 : launch_pp<2, false>(X, BH, N, stride, S, k, u, centroids, s);
+    if (d == 128) return launch_pp<4, false>(Xs, BH, Ns, 1, S, k, u, centroids, s);
+    return x_f32 ? launch_pp<2, true>(Xs, BH, Ns, 1, S, k, u, centroids, s)
+                 : launch_pp<2, false>(Xs, BH, Ns, 1, S, k, u, centroids, s);
   }
-  kmeanspp_kernel<<<BH, 1024, 0, s>>>(X, x_f32, N, stride, d, k, u, centroids, dist, near);
+  kmeanspp_kernel<<<BH, 1024, 0, s>>>(Xs, x_f32, Ns, 1, d, k, u, centroids, dist, near);
   return cudaGetLastError();
 }
 
@@ -1383,6 +1431,211 @@ cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k
   }
   const dim3 grid((N + 127) / 128, BH);
   assign_exact_kernel<<<grid, 128, 0, s>>>(X, x_f32, N, d, k, centroids, labels);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------------
+// Pruned assignment for the Lloyd iterations after the first (bf16 X, d = 128)
+// ------------------------------------------------------------------------------------------------
+// The tokens are taken in the previous iteration's label order (its stable sort), 128 per CTA, so a
+// tile holds few distinct previous labels a.  For token x of label a, every centroid j with
+// ||c_a - c_j|| > 2 ||x - c_a|| is strictly farther from x than c_a (triangle inequality), so it
+// cannot be the argmin.  Per tile and label a, R_a = max ||x - c_a|| over the tile's tokens of that
+// label; the candidates of the tile are the union over its labels of {j : ||c_a - c_j||^2 <=
+// 4 R_a^2 (1 + margin)^2}, the margin covering the float32 rounding of both sides.  Every token then
+// takes the exact float32 argmin of ||x - c_j||^2 over the candidates (ascending j, ties to the lower
+// index): the label is the one the full search would give, at the cost of a few centroids per tile
+// instead of all k.  When the union is large the same loop simply runs over more chunks.
+constexpr int kPrThreads = 256;    // two threads per token, 64 coordinates each
+constexpr int kPrTile = 128;       // tokens per CTA
+constexpr int kPrChunk = 64;       // candidate centroid rows staged in shared memory at a time
+constexpr float kPrMargin = 1.001f;
+
+// D2[bh][a][j] = ||c_a - c_j||^2 in float32 (differences, not the expanded form, which would cancel).
+// Block = 32 x 32 pairs of one head; 256 threads, each 4 pairs sharing its row a.
+__global__ void __launch_bounds__(256) centroid_dist_kernel(const float* __restrict__ C, int k,
+                                                           float* __restrict__ D2) {
+  __shared__ float ca[32][129];
+  __shared__ float cj[32][129];
+  const int bh = blockIdx.z, a0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  const float* Ch = C + static_cast<size_t>(bh) * k * 128;
+  for (int i = threadIdx.x; i < 32 * 128; i += 256) {
+    const int r = i >> 7, c = i & 127;
+    ca[r][c] = a0 + r < k ? Ch[static_cast<size_t>(a0 + r) * 128 + c] : 0.f;
+    cj[r][c] = j0 + r < k ? Ch[static_cast<size_t>(j0 + r) * 128 + c] : 0.f;
+  }
+  __syncthreads();
+  const int ai = threadIdx.x >> 3, jb = threadIdx.x & 7;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int c = 0; c < 128; ++c) {
+    const float x = ca[ai][c];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float df = x - cj[jb + 8 * m][c];
+      acc[m] = fmaf(df, df, acc[m]);
+    }
+  }
+  if (a0 + ai < k) {
+    float* row = D2 + (static_cast<size_t>(bh) * k + a0 + ai) * k;
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      if (j0 + jb + 8 * m < k) row[j0 + jb + 8 * m] = acc[m];
+  }
+}
+
+__global__ void __launch_bounds__(kPrThreads) pruned_assign_kernel(const uint16_t* __restrict__ X, int N, int k,
+                                                                  const float* __restrict__ C,
+                                                                  const float* __restrict__ D2,
+                                                                  const int32_t* __restrict__ perm,
+                                                                  int32_t* __restrict__ labels) {
+  __shared__ __align__(16) float cs[kPrChunk][128];
+  __shared__ uint32_t rmax[kMaxClustersAssign];   // R_a^2 (float bits) of the labels in the tile
+  __shared__ uint32_t bits[kMaxClustersAssign / 32];
+  __shared__ int16_t cand[kMaxClustersAssign];
+  __shared__ int16_t tile_labels[kPrTile];
+  __shared__ int n_labels, n_cand;
+  const int bh = blockIdx.y;
+  const int p0 = blockIdx.x * kPrTile;
+  const int tok = threadIdx.x >> 1, half = threadIdx.x & 1;
+  const int p = p0 + tok;
+  const bool valid = p < N;
+  const size_t head = static_cast<size_t>(bh) * N;
+  const float* Ch = C + static_cast<size_t>(bh) * k * 128;
+
+  for (int i = threadIdx.x; i < (k + 31) / 32; i += kPrThreads) bits[i] = 0u;
+  if (threadIdx.x == 0) n_labels = 0;
+  int n = 0, a = 0;
+  if (valid) {
+    n = perm[head + p];
+    n = n < 0 ? 0 : (n >= N ? N - 1 : n);
+    a = labels[head + n];
+    a = a < 0 ? 0 : (a >= k ? k - 1 : a);
+  }
+  // this thread's 64 coordinates of x
+  float x[64];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(X + (head + n) * 128 + half * 64);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 w = valid ? __ldg(src + q) : make_uint4(0u, 0u, 0u, 0u);
+      x[8 * q + 0] = bf16lo_to_f32(w.x); x[8 * q + 1] = bf16hi_to_f32(w.x);
+      x[8 * q + 2] = bf16lo_to_f32(w.y); x[8 * q + 3] = bf16hi_to_f32(w.y);
+      x[8 * q + 4] = bf16lo_to_f32(w.z); x[8 * q + 5] = bf16hi_to_f32(w.z);
+      x[8 * q + 6] = bf16lo_to_f32(w.w); x[8 * q + 7] = bf16hi_to_f32(w.w);
+    }
+  }
+  // r^2 = ||x - c_a||^2 (the two halves summed across the thread pair)
+  float r2;
+  {
+    const float4* ca4 = reinterpret_cast<const float4*>(Ch + static_cast<size_t>(a) * 128 + half * 64);
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float4 c = __ldg(ca4 + q);
+      float df = x[4 * q] - c.x;
+      acc = fmaf(df, df, acc);
+      df = x[4 * q + 1] - c.y;
+      acc = fmaf(df, df, acc);
+      df = x[4 * q + 2] - c.z;
+      acc = fmaf(df, df, acc);
+      df = x[4 * q + 3] - c.w;
+      acc = fmaf(df, df, acc);
+    }
+    r2 = acc + __shfl_xor_sync(0xffffffffu, acc, 1);
+  }
+  __syncthreads();
+  // the distinct previous labels of the tile (consecutive runs: the tokens are in label order)
+  if (valid && half == 0) {
+    const int prev = tok > 0 ? labels[head + perm[head + p - 1]] : -1;
+    if (prev != a) {
+      rmax[a] = 0u;
+      tile_labels[atomicAdd(&n_labels, 1)] = static_cast<int16_t>(a);
+    }
+  }
+  __syncthreads();
+  if (valid && half == 0) atomicMax(&rmax[a], __float_as_uint(r2));  // r2 >= 0: bits order as values
+  __syncthreads();
+  // union of the labels' candidates
+  const int nl = n_labels;
+  for (int li = 0; li < nl; ++li) {
+    const int al = tile_labels[li];
+    const float lim = 4.f * __uint_as_float(rmax[al]) * (kPrMargin * kPrMargin);
+    const float* drow = D2 + (static_cast<size_t>(bh) * k + al) * k;
+    for (int j = threadIdx.x; j < k; j += kPrThreads)
+      if (j == al || __ldg(drow + j) <= lim) atomicOr(&bits[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // compact the bit set into an ascending list
+    int base = 0;
+    for (int w0 = 0; w0 < (k + 31) / 32; w0 += 32) {
+      const int w = w0 + threadIdx.x;
+      const uint32_t b = w < (k + 31) / 32 ? bits[w] : 0u;
+      const int cnt = __popc(b);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (static_cast<int>(threadIdx.x) >= o) incl += v;
+      }
+      int pos = base + incl - cnt;
+      uint32_t bb = b;
+      while (bb) {
+        const int e = __ffs(bb) - 1;
+        bb &= bb - 1;
+        cand[pos++] = static_cast<int16_t>(w * 32 + e);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (threadIdx.x == 0) n_cand = base;
+  }
+  __syncthreads();
+  const int nc = n_cand;
+  float best = INFINITY;
+  int best_j = 0;
+  for (int c0 = 0; c0 < nc; c0 += kPrChunk) {
+    const int m = nc - c0 < kPrChunk ? nc - c0 : kPrChunk;
+    for (int i = threadIdx.x; i < m * 32; i += kPrThreads) {
+      const int r = i >> 5, q = i & 31;
+      reinterpret_cast<float4*>(cs[r])[q] =
+          __ldg(reinterpret_cast<const float4*>(Ch + static_cast<size_t>(cand[c0 + r]) * 128) + q);
+    }
+    __syncthreads();
+    for (int r = 0; r < m; ++r) {
+      const float4* c4 = reinterpret_cast<const float4*>(cs[r] + half * 64);
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 c = c4[q];
+        float df = x[4 * q] - c.x;
+        acc = fmaf(df, df, acc);
+        df = x[4 * q + 1] - c.y;
+        acc = fmaf(df, df, acc);
+        df = x[4 * q + 2] - c.z;
+        acc = fmaf(df, df, acc);
+        df = x[4 * q + 3] - c.w;
+        acc = fmaf(df, df, acc);
+      }
+      const float d2 = acc + __shfl_xor_sync(0xffffffffu, acc, 1);
+      if (d2 < best) {  // ascending candidates: a tie keeps the lower index
+        best = d2;
+        best_j = cand[c0 + r];
+      }
+    }
+    __syncthreads();
+  }
+  if (valid && half == 0) labels[head + n] = best_j;
+}
+
+cudaError_t launch_assign_pruned(const void* X, int BH, int N, int k, const float* centroids, const int32_t* perm,
+                                 float* d2, int32_t* labels, cudaStream_t s) {
+  if (k > kMaxClustersAssign) return cudaErrorInvalidValue;
+  const dim3 gd((k + 31) / 32, (k + 31) / 32, BH);
+  centroid_dist_kernel<<<gd, 256, 0, s>>>(centroids, k, d2);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 ga((N + kPrTile - 1) / kPrTile, BH);
+  pruned_assign_kernel<<<ga, kPrThreads, 0, s>>>(static_cast<const uint16_t*>(X), N, k, centroids, d2, perm, labels);
   return cudaGetLastError();
 }
 

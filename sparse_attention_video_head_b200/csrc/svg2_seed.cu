@@ -7,8 +7,8 @@
 //
 //   * one (b,h) runs on the CTAs of one thread-block cluster, each owning a contiguous range of the
 //     candidates, cut into tiles of 128 consecutive candidates;
-//   * a tile is fetched by TMA (the candidates are every stride-th token: a row pitch of stride rows)
-//     and multiplied by the new seed on the tensor core (M = 128 candidates, N = 16 with the seed in
+//   * a tile is fetched by TMA (the candidates are contiguous rows: all tokens, or the compact copy
+//     of the candidate rows the launcher makes) and multiplied by the new seed on the tensor core (M = 128 candidates, N = 16 with the seed in
 //     column 0, K = 128), giving x . c in TMEM;
 //   * the epilogue forms f = ||x||^2 + ||c||^2 - 2 x.c and lists the candidates where f, widened by
 //     a rigorous error bound, does not rule out an improvement; after the stream the whole CTA

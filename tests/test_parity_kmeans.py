@@ -59,8 +59,8 @@ def _seeds(svg2, X, k, u, seed_tokens, dev_x):
 @pytest.mark.parametrize("cfg_name,heads,role,seed_tokens", [
     ("tiny", [0], "k", 0),                     # float32, d = 64 (CUDA-core seeding)
     ("small", [0, 3], "k", 0),                 # 12480 candidates, k = 256, clusters of several CTAs
-    ("small", [1], "q", 5000),                 # stride 3: 4160 candidates, ragged last tile
-    ("small", [2], "k", 300),                  # stride 42: 298 candidates for 256 seeds, one CTA
+    ("small", [1], "q", 5000),                 # 5000 candidates, ragged last tile
+    ("small", [2], "k", 300),                  # 300 candidates for 256 seeds, one CTA
     ("wan720p", [4], "q", 16384), ("wan720p", [9], "k", 16384),
     ("wan720p", [1], "k", 0),                  # all 75600 tokens: 13+ CTAs per head
     ("hunyuan720p", [6], "k", 16384)])         # k = 1000
@@ -72,9 +72,9 @@ def test_kmeanspp_seeds_bit_exact(oracle, cfg_name, heads, role, seed_tokens):
     X, u = data[role], data["u" + role]
     k = cfg.nQ if role == "q" else cfg.nK
     C = _seeds(svg2, X, k, u, seed_tokens, _xdev(cfg, X))
-    stride = oracle.seed_stride(X.shape[2], seed_tokens)
+    idx = oracle.seed_candidates(X.shape[2], seed_tokens)
     for h in range(len(heads)):
-        _, Cref = oracle.kmeanspp(np.ascontiguousarray(X[0, h][::stride]), k, u[0, h])
+        _, Cref = oracle.kmeanspp(np.ascontiguousarray(X[0, h][idx]), k, u[0, h])
         bad = np.nonzero((C[0, h] != Cref.astype(np.float32)).any(axis=1))[0]
         assert bad.size == 0, f"{cfg_name} head {heads[h]}: first differing seed {bad[:1]} of {k}"
 
@@ -107,8 +107,8 @@ def test_kmeanspp_then_lockstep_lloyd(oracle, cfg_name, heads, role, seed_tokens
     iters = cfg.iters
     # iteration 1 from k-means++ seeds (the seeds themselves are checked through it)
     C1, lab1, cnt1 = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_KMEANSPP, u=u, seed_tokens=seed_tokens)
-    stride = oracle.seed_stride(X.shape[2], seed_tokens)
-    seeds0 = lambda h: oracle.kmeanspp(np.ascontiguousarray(X[0, h][::stride]), k, u[0, h])[1]
+    idx = oracle.seed_candidates(X.shape[2], seed_tokens)
+    seeds0 = lambda h: oracle.kmeanspp(np.ascontiguousarray(X[0, h][idx]), k, u[0, h])[1]
     stats = []
     for h in range(len(heads)):
         C0 = seeds0(h)
@@ -222,3 +222,63 @@ def test_assign_candidate_list_overflow(oracle):
         assert not near_tie(d1, d2).any()
         bad = int((lab[0, h] != ref_lab).sum())
         assert bad == 0, f"head {h}: {bad} of {X.shape[2]} tokens not at their nearest centroid"
+
+
+def _pruned_iteration_check(oracle, svg2, cfg, X, C_in, what):
+    """Iteration 2 of a k-means run from C_in (the pruned search for k >= 256) against the oracle's
+    assignment to the centroids iteration 1 produced (exact given the GPU's own iteration-1 labels)."""
+    k = C_in.shape[2]
+    _, lab1, _ = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_GIVEN, C0=C_in)
+    C2, lab2, _ = _run(svg2, cfg, X, k, 2, svg2.SVG2_INIT_GIVEN, C0=C_in)
+    stats = []
+    for h in range(X.shape[1]):
+        C1, _ = oracle.update(X[0, h], lab1[0, h], C_in[0, h])
+        ref, d1, d2 = oracle.assign(X[0, h], C1)
+        stats.append(_check_assign(lab2[0, h], ref, d1, d2, f"{what} head {h} iteration 2"))
+        Cref, _ = oracle.update(X[0, h], lab2[0, h], C1)
+        np.testing.assert_array_equal(C2[0, h], Cref.astype(np.float32))
+    return stats
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg_name,heads,stage", [("small", [0, 3], 0), ("wan720p", [2], 0), ("wan720p", [5], 2),
+                                                 ("hunyuan720p", [1], 0)])
+def test_pruned_assignment_lockstep(oracle, cfg_name, heads, stage):
+    """The Lloyd iterations after the first use the pruned search on the K side (k >= 256): from the
+    k-means++ seeds (stage 0) or from centroids two oracle iterations later (stage 2)."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS[cfg_name]
+    data = pool_layer_inputs(cfg, heads)
+    X, u = data["k"], data["uk"]
+    k = cfg.nK
+    idx = oracle.seed_candidates(X.shape[2], svg2.DEFAULT_SEED_TOKENS)
+    C_in = []
+    for h in range(len(heads)):
+        C0 = oracle.kmeanspp(np.ascontiguousarray(X[0, h][idx]), k, u[0, h])[1]
+        if stage:
+            C0 = oracle.lloyd(X[0, h], C0, stage)[0]
+        C_in.append(C0.astype(np.float32).astype(np.float64))
+    stats = _pruned_iteration_check(oracle, svg2, cfg, X, np.stack(C_in)[None], cfg_name)
+    print(f"{cfg_name} stage {stage}: (near-tie mismatches, near-ties) {stats}")
+
+
+@pytest.mark.gpu
+def test_pruned_assignment_duplicate_centroids_and_far_tokens(oracle):
+    """Centroids given twice (distance 0 between them: neither may prune the other, and the first
+    iteration's ties go to the lower index), and a few tokens far from every centroid (a large
+    radius that keeps most clusters as candidates: the search then runs over several chunks of 64)."""
+    svg2 = require_gpu()
+    cfg = I.CONFIGS["small"]
+    rng = np.random.default_rng(33)
+    k, N = 300, 6000
+    centres = rng.standard_normal((k, 128))
+    centres[150:] = centres[:150]                       # clusters 150..299 duplicate 0..149
+    lab = rng.integers(0, 150, size=N)
+    X = centres[lab] + 0.3 * rng.standard_normal((N, 128))
+    X[:40] = 6.0 * rng.standard_normal((40, 128))       # far tokens
+    X = I.round_to_bf16(X.astype(np.float32))[None, None]
+    C_in = centres.astype(np.float32).astype(np.float64)[None, None]
+    _, lab1, _ = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_GIVEN, C0=C_in)
+    assert (lab1[0, 0] < 150).all()                     # a duplicate never beats the lower index
+    stats = _pruned_iteration_check(oracle, svg2, cfg, X, C_in, "duplicates")
+    print(stats)
