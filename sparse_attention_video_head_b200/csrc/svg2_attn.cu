@@ -360,8 +360,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
     // ---------------- key/value gather producer ----------------
     // Warp w fills rows 64w'..64w'+63 of each key tile (w' = w - first producer warp).  Each lane
-    // first finds the source rows of two stream positions; then every cp.async instruction moves
-    // whole rows (16 lanes x 16 bytes per row at d = 128), so one instruction touches 2 rows.
+    // follows the source rows of two stream positions from tile to tile with cursors over the range
+    // table (positions only grow, so each cursor crosses every range boundary once, where a search
+    // per tile would cost a chain of dependent shared-memory reads); then every cp.async instruction
+    // moves whole rows (16 lanes x 16 bytes per row at d = 128), so one instruction touches 2 rows.
     constexpr int CPR = D / 8;       // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;    // rows per warp instruction
     const int wr0 = (warp - kProducerWarp0) * 64;
@@ -369,20 +371,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const size_t head_row0 = static_cast<size_t>(bh) * N;
     const int my_chunk = lane % CPR, my_sub = lane / CPR;
     const int hf = my_chunk >> 3, cc = my_chunk & 7;
-    // source row of stream position p: the largest e with r_cum[e] <= p, then the offset inside it
-    auto src_row = [&](int p) {
+    int e0c = 0, e1c = 0;  // cursors of this lane's two stream positions: r_cum[e] <= p < r_cum[e + 1]
+    auto src_row = [&](int p, int& e) {
       if (p >= L) p = L - 1;
-      int lo = 0, hi = nranges - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (r_cum[mid] <= p) lo = mid; else hi = mid - 1;
-      }
-      const int r = r_start[lo] + (p - r_cum[lo]);
+      while (e + 1 < nranges && r_cum[e + 1] <= p) ++e;
+      const int r = r_start[e] + (p - r_cum[e]);
       return r < 0 ? 0 : (r >= N ? N - 1 : r);
     };
     for (int j = 0; j < T; ++j) {
       const int stage = j & 1;
-      const int krow0 = src_row(j * 128 + wr0 + lane), krow1 = src_row(j * 128 + wr0 + 32 + lane);
+      const int krow0 = src_row(j * 128 + wr0 + lane, e0c), krow1 = src_row(j * 128 + wr0 + 32 + lane, e1c);
       const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
       // K(j) may land as soon as both S products of K(j-2) are done, V(j) once both PV products of
       // V(j-2) are; each lands asynchronously and counts itself on its full barrier

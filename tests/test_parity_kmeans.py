@@ -225,7 +225,7 @@ def test_assign_candidate_list_overflow(oracle):
 
 
 def _pruned_iteration_check(oracle, svg2, cfg, X, C_in, what):
-    """Iteration 2 of a k-means run from C_in (the pruned search for k >= 256) against the oracle's
+    """Iteration 2 of a k-means run from C_in (the pruned search for k >= 500) against the oracle's
     assignment to the centroids iteration 1 produced (exact given the GPU's own iteration-1 labels)."""
     k = C_in.shape[2]
     _, lab1, _ = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_GIVEN, C0=C_in)
@@ -241,16 +241,17 @@ def _pruned_iteration_check(oracle, svg2, cfg, X, C_in, what):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("cfg_name,heads,stage", [("small", [0, 3], 0), ("wan720p", [2], 0), ("wan720p", [5], 2),
-                                                 ("hunyuan720p", [1], 0)])
-def test_pruned_assignment_lockstep(oracle, cfg_name, heads, stage):
-    """The Lloyd iterations after the first use the pruned search on the K side (k >= 256): from the
-    k-means++ seeds (stage 0) or from centroids two oracle iterations later (stage 2)."""
+@pytest.mark.parametrize("cfg_name,heads,stage,k", [("small", [0, 3], 0, 512), ("wan720p", [2], 0, 500),
+                                                   ("wan720p", [5], 2, 500), ("hunyuan720p", [1], 0, 1000)])
+def test_pruned_assignment_lockstep(oracle, cfg_name, heads, stage, k):
+    """The Lloyd iterations after the first use the pruned search when k >= 500 (the K side of the
+    Wan and Hunyuan layers): from the k-means++ seeds (stage 0) or from centroids two oracle
+    iterations later (stage 2); the small shape with k = 512 gives tiles of few tokens per cluster."""
     svg2 = require_gpu()
     cfg = I.CONFIGS[cfg_name]
     data = pool_layer_inputs(cfg, heads)
-    X, u = data["k"], data["uk"]
-    k = cfg.nK
+    X = data["k"]
+    u = np.random.default_rng(cfg.cfg_id + 77).random((1, len(heads), k))
     idx = oracle.seed_candidates(X.shape[2], svg2.DEFAULT_SEED_TOKENS)
     C_in = []
     for h in range(len(heads)):
@@ -270,15 +271,15 @@ def test_pruned_assignment_duplicate_centroids_and_far_tokens(oracle):
     svg2 = require_gpu()
     cfg = I.CONFIGS["small"]
     rng = np.random.default_rng(33)
-    k, N = 300, 6000
+    k, N = 600, 9000
     centres = rng.standard_normal((k, 128))
-    centres[150:] = centres[:150]                       # clusters 150..299 duplicate 0..149
-    lab = rng.integers(0, 150, size=N)
+    centres[300:] = centres[:300]                       # clusters 300..599 duplicate 0..299
+    lab = rng.integers(0, 300, size=N)
     X = centres[lab] + 0.3 * rng.standard_normal((N, 128))
     X[:40] = 6.0 * rng.standard_normal((40, 128))       # far tokens
     X = I.round_to_bf16(X.astype(np.float32))[None, None]
     C_in = centres.astype(np.float32).astype(np.float64)[None, None]
     _, lab1, _ = _run(svg2, cfg, X, k, 1, svg2.SVG2_INIT_GIVEN, C0=C_in)
-    assert (lab1[0, 0] < 150).all()                     # a duplicate never beats the lower index
+    assert (lab1[0, 0] < 300).all()                     # a duplicate never beats the lower index
     stats = _pruned_iteration_check(oracle, svg2, cfg, X, C_in, "duplicates")
     print(stats)
