@@ -86,10 +86,10 @@ def gen_inputs(cfg, step=0, heads=None):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 239.9 MB + 68.0 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 239.5 MB + 62.3 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "63ea0eeb193d63e8934ca4adae42c4976e0f0c7ac761c89790ffe9b393c0790e",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 239.936000e6 + 67.964672e6,
+ATTN_TRAFFIC = {"sha256": "929d4ecea5230bdbf26d7e174e2aaa22142e0ef2ef718326b9a0ccc1f696cbc7",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 239.534592e6 + 62.283008e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 
