@@ -12,6 +12,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsvg2.so")
+# The debug build (-DSVG2_DEBUG): every data-derived index the kernels clamp or skip is also reported
+# as SVG2_ERR_DEVICE_BOUNDS in the status word.  Same ABI, separate library.
+DEBUG_LIB = os.path.join(PKG, "libsvg2_debug.so")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
@@ -36,29 +39,32 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    """Compile libsvg2.so (or, with debug=True, libsvg2_debug.so) in-tree; returns the library's path."""
+    out_dir = os.path.join(BUILD_DIR, "debug") if debug else BUILD_DIR
+    lib = DEBUG_LIB if debug else LIB
+    os.makedirs(out_dir, exist_ok=True)
     headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src).replace(".cu", ".o"))
+        obj = os.path.join(out_dir, os.path.basename(src).replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [_nvcc(), *NVCC_FLAGS, "-c", src, "-o", obj]
+            cmd = [_nvcc(), *NVCC_FLAGS, *(["-DSVG2_DEBUG"] if debug else []), "-c", src, "-o", obj]
             if ptxas_verbose:
                 cmd += ["-Xptxas", "-v"]
             if verbose:
                 print(" ".join(cmd), file=sys.stderr)
             subprocess.check_call(cmd)
-    if force or _stale(LIB, objs):
-        cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs]
+    if force or _stale(lib, objs):
+        cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", lib, *objs]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.check_call(cmd)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_verbose="--ptxas" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_verbose="--ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

@@ -118,12 +118,13 @@ cudaError_t run_kmeans(const void* X, bool f32, int BH, int N, int d, int k, int
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
     // after the first iteration, perm holds the stable sort of the previous labels: the pruned search
     if (it > 0 && s.d2 != nullptr && !f32 && d == 128)
-      e = launch_assign_pruned(X, BH, N, k, C, perm, s.d2, labels, stream);
+      e = launch_assign_pruned(X, BH, N, k, C, perm, s.d2, labels, stream, st);
     else
       e = launch_assign(X, f32, BH, N, d, k, C, s.c_hi, s.c_lo, s.c_norm, labels, s.rr_list, s.rr_count, st,
                         wait_budget_of(st), stream);
     if (e == cudaSuccess) e = launch_sort(labels, BH, N, k, perm, offsets, counts, s.chunk_hist, st, stream);
-    if (e == cudaSuccess) e = launch_update(X, f32, BH, N, d, k, perm, offsets, C, s.c_hi, s.c_lo, s.c_norm, stream);
+    if (e == cudaSuccess)
+      e = launch_update(X, f32, BH, N, d, k, perm, offsets, C, s.c_hi, s.c_lo, s.c_norm, stream, st);
   }
   return e;
 }
@@ -507,8 +508,8 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, L.weights, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);
-    if (e == cudaSuccess) e = launch_gather(Q, f32, L.perm_q, BH, N, d, L.Qp, s);
-    if (e == cudaSuccess) e = launch_gather2(K, V, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s);
+    if (e == cudaSuccess) e = launch_gather(Q, f32, L.perm_q, BH, N, d, L.Qp, s, L.st);
+    if (e == cudaSuccess) e = launch_gather2(K, V, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s, L.st);
     if (e == cudaSuccess) {
       if (p->fuse_unpermute) {
         e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
@@ -516,7 +517,7 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
       } else {
         e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
                                p->scale, nullptr, L.Op, L.attn, L.st, wait_budget_of(L.st), s);
-        if (e == cudaSuccess) e = launch_unpermute(L.Op, L.perm_q, BH, N, d, O, s);
+        if (e == cudaSuccess) e = launch_unpermute(L.Op, L.perm_q, BH, N, d, O, s, L.st);
       }
     }
     return to_status(e);
@@ -644,7 +645,7 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, nullptr, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);
-    if (e == cudaSuccess) e = launch_gather(Qd, f32, L.perm_q, BH, N, d, L.Qp, s);
+    if (e == cudaSuccess) e = launch_gather(Qd, f32, L.perm_q, BH, N, d, L.Qp, s, L.st);
     // per head group: gather its K and V planes once its V has landed, attend, and copy the output
     // back while the next group runs
     const size_t plane_p = static_cast<size_t>(N) * d;  // elements of one permuted plane
@@ -655,7 +656,7 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
       if (e == cudaSuccess)
         e = launch_gather2(static_cast<const char*>(Kd) + h0 * plane_in, static_cast<const char*>(Vd) + h0 * plane_in,
                            f32, L.perm_k + h0 * N, hn, N, d, static_cast<uint16_t*>(L.Kp) + h0 * plane_p,
-                           static_cast<uint16_t*>(L.Vp) + h0 * plane_p, s);
+                           static_cast<uint16_t*>(L.Vp) + h0 * plane_p, s, L.st);
       if (e != cudaSuccess) break;
       e = launch_sparse_attn(static_cast<const uint16_t*>(L.Qp) + h0 * plane_p,
                              static_cast<const uint16_t*>(L.Kp) + h0 * plane_p,

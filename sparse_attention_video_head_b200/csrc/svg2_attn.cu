@@ -64,13 +64,14 @@ struct AttnBars {
 };
 
 __global__ void plan_count_kernel(const int32_t* __restrict__ q_off, int nQ, int N,
-                                  int32_t* __restrict__ head_units) {
+                                  int32_t* __restrict__ head_units, DeviceStatus* st) {
   __shared__ int32_t part[32];
   const int bh = blockIdx.x;
   int acc = 0;
   for (int i = threadIdx.x; i < nQ; i += blockDim.x) {
     const int r0 = q_off[static_cast<size_t>(bh) * (nQ + 1) + i];
     const int n = q_off[static_cast<size_t>(bh) * (nQ + 1) + i + 1] - r0;
+    SVG2_DEBUG_CHECK(r0 >= 0 && n >= 0 && r0 + n <= N, st, kWherePlan, i, r0);
     if (r0 < 0 || n <= 0 || r0 + n > N) continue;
     acc += (n + 255) / 256;
   }
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int pt = threadIdx.x - 32 * kProducerWarp0;
     const size_t row = static_cast<size_t>(bh) * nQ + un.cluster;
     int cnt = sel_count[row];
+    SVG2_DEBUG_CHECK(cnt >= 0 && cnt <= nK, st, kWherePlan, row, cnt);
     cnt = cnt < 0 ? 0 : (cnt > nK ? nK : cnt);
     const int32_t* ko = k_off + static_cast<size_t>(bh) * (nK + 1);
     // each thread handles a contiguous block of entries, then a scan over the block sums
@@ -179,8 +181,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int local = 0;
     for (int e = e0; e < e1; ++e) {
       int j = sel_idx[row * nK + e];
+      SVG2_DEBUG_CHECK(j >= 0 && j < nK, st, kWherePlan, row, j);
       j = j < 0 ? 0 : (j >= nK ? nK - 1 : j);
       const int s0 = ko[j], len = ko[j + 1] - s0;
+      SVG2_DEBUG_CHECK(s0 >= 0 && len >= 0 && s0 + len <= N, st, kWherePlan, j, s0);
       r_start[e] = s0;
       r_cum[e] = len;  // temporarily the length
       local += len;
@@ -376,6 +380,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (p >= L) p = L - 1;
       while (e + 1 < nranges && r_cum[e + 1] <= p) ++e;
       const int r = r_start[e] + (p - r_cum[e]);
+      SVG2_DEBUG_CHECK(r >= 0 && r < N, st, kWhereAttnProducer, p, r);
       return r < 0 ? 0 : (r >= N ? N - 1 : r);
     };
     for (int j = 0; j < T; ++j) {
@@ -521,6 +526,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         int tk = -1;
         if (row < nrows_x) {
           tk = perm_q != nullptr ? __ldg(perm_q + static_cast<size_t>(bh) * N + prow) : prow;
+          SVG2_DEBUG_CHECK(tk >= 0 && tk < N, st, kWhereAttnSoftmax, prow, tk);
           if (tk < 0 || tk >= N) tk = -1;  // an invalid permutation entry is skipped
         }
         uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<size_t>(bh) * N + (tk < 0 ? 0 : tk)) * D);
@@ -701,7 +707,7 @@ cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, c
                                int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
                                const AttnScratch& sc, DeviceStatus* st, const uint64_t* wait_budget,
                                cudaStream_t s) {
-  plan_count_kernel<<<BH, 256, 0, s>>>(q_off, nQ, N, sc.head_units);
+  plan_count_kernel<<<BH, 256, 0, s>>>(q_off, nQ, N, sc.head_units, st);
   plan_scan_kernel<<<1, 32, 0, s>>>(sc.head_units, BH, sc.head_base);
   plan_write_kernel<<<BH, 32, 0, s>>>(q_off, nQ, N, sc.head_base, sc.units);
   cudaError_t e = cudaGetLastError();

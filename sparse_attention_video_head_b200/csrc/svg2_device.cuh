@@ -30,6 +30,22 @@ __device__ __forceinline__ void raise_status(DeviceStatus* st, uint32_t code, ui
   }
 }
 
+// Index checks of the debug build (compiled with -DSVG2_DEBUG, library libsvg2_debug.so): where a kernel
+// clamps or skips a data-derived index that lies outside its buffer, the debug build also latches
+// SVG2_ERR_DEVICE_BOUNDS with the kernel tag and the offending values.  The access itself is clamped or
+// skipped in both builds, so a bad index is never dereferenced.
+#ifdef SVG2_DEBUG
+#define SVG2_DEBUG_CHECK(ok, st, where, a, b)                                                  \
+  do {                                                                                         \
+    if (!(ok)) ::svg2::raise_status((st), ::svg2::kStatusDeviceBounds, (where), static_cast<uint32_t>(a), \
+                                    static_cast<uint32_t>(b));                                 \
+  } while (0)
+#else
+#define SVG2_DEBUG_CHECK(ok, st, where, a, b) \
+  do {                                        \
+  } while (0)
+#endif
+
 __device__ __forceinline__ bool status_set(const DeviceStatus* st) {
   if (st == nullptr) return false;
   return *reinterpret_cast<const volatile uint32_t*>(&st->code) != 0u;

@@ -41,6 +41,10 @@ enum : uint32_t {
   kWhereSeedMma = 10,
   kWhereSeedEpilogue = 11,
   kWhereSeedDrain = 12,
+  kWhereGather = 13,     // row gathers and the inverse-permutation scatter (debug build)
+  kWhereUpdate = 14,     // centroid update (debug build)
+  kWherePlan = 15,       // attention work plan and range table (debug build)
+  kWherePruned = 16,     // pruned assignment (debug build)
 };
 
 constexpr int kStatusBytes = 256;
@@ -134,12 +138,13 @@ inline void carve_attn(Carve& c, int BH, int N, int nQ, AttnScratch& s) {
 // ---- launchers (host functions defined in the .cu files); all return cudaError_t ----
 cudaError_t launch_sort(const int32_t* labels, int BH, int N, int k, int32_t* perm, int32_t* offsets,
                         int32_t* counts, int32_t* chunk_hist, DeviceStatus* st, cudaStream_t s);
+// st (may be null) receives the debug build's index reports; the release build never writes it here.
 cudaError_t launch_gather(const void* X, bool x_f32, const int32_t* perm, int BH, int N, int d, void* Xp,
-                          cudaStream_t s);
+                          cudaStream_t s, DeviceStatus* st = nullptr);
 cudaError_t launch_gather2(const void* X0, const void* X1, bool x_f32, const int32_t* perm, int BH, int N,
-                           int d, void* Xp0, void* Xp1, cudaStream_t s);
+                           int d, void* Xp0, void* Xp1, cudaStream_t s, DeviceStatus* st = nullptr);
 cudaError_t launch_unpermute(const void* Op, const int32_t* perm, int BH, int N, int d, void* O,
-                             cudaStream_t s);
+                             cudaStream_t s, DeviceStatus* st = nullptr);
 
 // k-means++ seeding over the candidates kmeanspp_candidates() counts; when they are fewer than the
 // tokens, their rows are first copied into `cand` (at least kmeanspp_candidate_bytes() bytes).
@@ -165,10 +170,10 @@ cudaError_t launch_assign(const void* X, bool x_f32, int BH, int N, int d, int k
 // Lloyd assignment from the previous iteration's stable sort `perm` (bf16 X, d = 128, k <= 1024):
 // the centroid-to-centroid table into d2 [BH, k, k], then the pruned exact search per tile.
 cudaError_t launch_assign_pruned(const void* X, int BH, int N, int k, const float* centroids, const int32_t* perm,
-                                 float* d2, int32_t* labels, cudaStream_t s);
+                                 float* d2, int32_t* labels, cudaStream_t s, DeviceStatus* st = nullptr);
 cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
                           const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
-                          float* c_norm, cudaStream_t s);
+                          float* c_norm, cudaStream_t s, DeviceStatus* st = nullptr);
 
 cudaError_t launch_select(const float* cq, const float* ck, const float* weights_in, const int32_t* count_k,
                           int BH, int nQ, int nK, int d, float top_p, float scale, float* weights_out,

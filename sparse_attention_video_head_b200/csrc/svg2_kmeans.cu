@@ -1151,7 +1151,8 @@ __global__ void __launch_bounds__(kUpdThreads) update_kernel(const void* __restr
                                                               int kpad, const int32_t* __restrict__ perm,
                                                               const int32_t* __restrict__ offsets,
                                                               float* __restrict__ C, uint16_t* __restrict__ hi,
-                                                              uint16_t* __restrict__ lo, float* __restrict__ norm) {
+                                                              uint16_t* __restrict__ lo, float* __restrict__ norm,
+                                                              DeviceStatus* st) {
   constexpr int ESZ = F32 ? 4 : 2;
   constexpr int ROWB = D * ESZ;                 // bytes per row
   constexpr int CH = ROWB / 16;                 // 16-byte chunks per row
@@ -1159,8 +1160,11 @@ __global__ void __launch_bounds__(kUpdThreads) update_kernel(const void* __restr
   __shared__ __align__(16) uint8_t buf[2][kUpdBufBytes];
   __shared__ float red[kUpdThreads / 32];
   const int bh = blockIdx.x / k, j = blockIdx.x % k;
-  const int o0 = offsets[static_cast<size_t>(bh) * (k + 1) + j];
-  const int o1 = offsets[static_cast<size_t>(bh) * (k + 1) + j + 1];
+  int o0 = offsets[static_cast<size_t>(bh) * (k + 1) + j];
+  int o1 = offsets[static_cast<size_t>(bh) * (k + 1) + j + 1];
+  SVG2_DEBUG_CHECK(o0 >= 0 && o1 <= N && o0 <= o1, st, kWhereUpdate, o0, o1);
+  o0 = o0 < 0 ? 0 : (o0 > N ? N : o0);  // malformed offsets become an empty cluster
+  o1 = o1 < o0 ? o0 : (o1 > N ? N : o1);
   const int cnt = o1 - o0;
   const int tid = threadIdx.x;
   float* cj = C + (static_cast<size_t>(bh) * k + j) * D;
@@ -1186,6 +1190,7 @@ __global__ void __launch_bounds__(kUpdThreads) update_kernel(const void* __restr
       const int q = tid + i * kUpdThreads;
       const int r = q / CH, c = q - r * CH;
       if (r < nr) {
+        SVG2_DEBUG_CHECK(t[i] >= 0 && t[i] < N, st, kWhereUpdate, o0 + batch * kUpdRows + r, t[i]);
         const int tk = t[i] < 0 ? 0 : (t[i] >= N ? N - 1 : t[i]);
         cp_async16(smem_u32(&buf[b][r * ROWB + c * 16]), xb + static_cast<size_t>(tk) * ROWB + c * 16);
       }
@@ -1488,7 +1493,7 @@ __global__ void __launch_bounds__(kPrThreads) pruned_assign_kernel(const uint16_
                                                                   const float* __restrict__ C,
                                                                   const float* __restrict__ D2,
                                                                   const int32_t* __restrict__ perm,
-                                                                  int32_t* __restrict__ labels) {
+                                                                  int32_t* __restrict__ labels, DeviceStatus* st) {
   __shared__ __align__(16) float cs[kPrChunk][128];
   __shared__ uint32_t rmax[kMaxClustersAssign];   // R_a^2 (float bits) of the labels in the tile
   __shared__ uint32_t bits[kMaxClustersAssign / 32];
@@ -1508,8 +1513,10 @@ __global__ void __launch_bounds__(kPrThreads) pruned_assign_kernel(const uint16_
   int n = 0, a = 0;
   if (valid) {
     n = perm[head + p];
+    SVG2_DEBUG_CHECK(n >= 0 && n < N, st, kWherePruned, p, n);
     n = n < 0 ? 0 : (n >= N ? N - 1 : n);
     a = labels[head + n];
+    SVG2_DEBUG_CHECK(a >= 0 && a < k, st, kWherePruned, n, a);
     a = a < 0 ? 0 : (a >= k ? k - 1 : a);
   }
   // this thread's 64 coordinates of x
@@ -1547,7 +1554,13 @@ __global__ void __launch_bounds__(kPrThreads) pruned_assign_kernel(const uint16_
   __syncthreads();
   // the distinct previous labels of the tile (consecutive runs: the tokens are in label order)
   if (valid && half == 0) {
-    const int prev = tok > 0 ? labels[head + perm[head + p - 1]] : -1;
+    int prev = -1;
+    if (tok > 0) {
+      int np = perm[head + p - 1];
+      np = np < 0 ? 0 : (np >= N ? N - 1 : np);
+      prev = labels[head + np];
+      prev = prev < 0 ? 0 : (prev >= k ? k - 1 : prev);
+    }
     if (prev != a) {
       rmax[a] = 0u;
       tile_labels[atomicAdd(&n_labels, 1)] = static_cast<int16_t>(a);
@@ -1628,32 +1641,33 @@ __global__ void __launch_bounds__(kPrThreads) pruned_assign_kernel(const uint16_
 }
 
 cudaError_t launch_assign_pruned(const void* X, int BH, int N, int k, const float* centroids, const int32_t* perm,
-                                 float* d2, int32_t* labels, cudaStream_t s) {
+                                 float* d2, int32_t* labels, cudaStream_t s, DeviceStatus* st) {
   if (k > kMaxClustersAssign) return cudaErrorInvalidValue;
   const dim3 gd((k + 31) / 32, (k + 31) / 32, BH);
   centroid_dist_kernel<<<gd, 256, 0, s>>>(centroids, k, d2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 ga((N + kPrTile - 1) / kPrTile, BH);
-  pruned_assign_kernel<<<ga, kPrThreads, 0, s>>>(static_cast<const uint16_t*>(X), N, k, centroids, d2, perm, labels);
+  pruned_assign_kernel<<<ga, kPrThreads, 0, s>>>(static_cast<const uint16_t*>(X), N, k, centroids, d2, perm, labels,
+                                                  st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_update(const void* X, bool x_f32, int BH, int N, int d, int k, const int32_t* perm,
                           const int32_t* offsets, float* centroids, uint16_t* c_hi, uint16_t* c_lo,
-                          float* c_norm, cudaStream_t s) {
+                          float* c_norm, cudaStream_t s, DeviceStatus* st) {
   const int blocks = BH * k;
   const int kp = kpad_of(k);
   if (d == 128) {
     if (x_f32)
-      update_kernel<128, true><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+      update_kernel<128, true><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm, st);
     else
-      update_kernel<128, false><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+      update_kernel<128, false><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm, st);
   } else {
     if (x_f32)
-      update_kernel<64, true><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+      update_kernel<64, true><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm, st);
     else
-      update_kernel<64, false><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm);
+      update_kernel<64, false><<<blocks, kUpdThreads, 0, s>>>(X, BH, N, k, kp, perm, offsets, centroids, c_hi, c_lo, c_norm, st);
   }
   return cudaGetLastError();
 }

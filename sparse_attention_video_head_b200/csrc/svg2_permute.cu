@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict
                                                            bool f32, const int32_t* __restrict__ perm,
                                                            long long rows, int N, int d,
                                                            __nv_bfloat16* __restrict__ Y0,
-                                                           __nv_bfloat16* __restrict__ Y1) {
+                                                           __nv_bfloat16* __restrict__ Y1, DeviceStatus* st) {
   const int per_row = d / 8;  // threads per row
   const long long total = rows * per_row;
   const size_t esz = f32 ? 4 : 2;
@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict
     const int e = static_cast<int>(g - r * per_row) * 8;
     const long long bh = r / N;
     const int pr = __ldg(perm + r);
+    SVG2_DEBUG_CHECK(pr >= 0 && pr < N, st, kWhereGather, r, pr);
     if (pr < 0 || pr >= N) continue;  // an invalid permutation entry is skipped, never dereferenced
     const long long src = bh * N + pr;
     const uint4 v0 = load8_as_bf16(static_cast<const char*>(X0) + src * d * esz, e, f32);
@@ -163,7 +164,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict
 
 __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* __restrict__ Op,
                                                             const int32_t* __restrict__ perm, long long rows,
-                                                            int N, int d, __nv_bfloat16* __restrict__ O) {
+                                                            int N, int d, __nv_bfloat16* __restrict__ O,
+                                                            DeviceStatus* st) {
   const int per_row = d / 8;
   const long long total = rows * per_row;
   for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < total;
@@ -172,6 +174,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
     const int e = static_cast<int>(g - r * per_row) * 8;
     const long long bh = r / N;
     const int pr = __ldg(perm + r);
+    SVG2_DEBUG_CHECK(pr >= 0 && pr < N, st, kWhereGather, r, pr);
     if (pr < 0 || pr >= N) continue;
     const long long dst = bh * N + pr;
     *reinterpret_cast<uint4*>(O + dst * d + e) = __ldg(reinterpret_cast<const uint4*>(Op + r * d + e));
@@ -200,27 +203,27 @@ cudaError_t launch_sort(const int32_t* labels, int BH, int N, int k, int32_t* pe
 }
 
 cudaError_t launch_gather(const void* X, bool x_f32, const int32_t* perm, int BH, int N, int d, void* Xp,
-                          cudaStream_t s) {
+                          cudaStream_t s, DeviceStatus* st) {
   const long long rows = static_cast<long long>(BH) * N;
   gather_rows_kernel<<<copy_grid(rows * (d / 8)), 256, 0, s>>>(X, nullptr, x_f32, perm, rows, N, d,
-                                                                static_cast<__nv_bfloat16*>(Xp), nullptr);
+                                                                static_cast<__nv_bfloat16*>(Xp), nullptr, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather2(const void* X0, const void* X1, bool x_f32, const int32_t* perm, int BH, int N,
-                           int d, void* Xp0, void* Xp1, cudaStream_t s) {
+                           int d, void* Xp0, void* Xp1, cudaStream_t s, DeviceStatus* st) {
   const long long rows = static_cast<long long>(BH) * N;
   gather_rows_kernel<<<copy_grid(rows * (d / 8)), 256, 0, s>>>(X0, X1, x_f32, perm, rows, N, d,
                                                                 static_cast<__nv_bfloat16*>(Xp0),
-                                                                static_cast<__nv_bfloat16*>(Xp1));
+                                                                static_cast<__nv_bfloat16*>(Xp1), st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpermute(const void* Op, const int32_t* perm, int BH, int N, int d, void* O,
-                             cudaStream_t s) {
+                             cudaStream_t s, DeviceStatus* st) {
   const long long rows = static_cast<long long>(BH) * N;
   scatter_rows_kernel<<<copy_grid(rows * (d / 8)), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(Op), perm,
-                                                                 rows, N, d, static_cast<__nv_bfloat16*>(O));
+                                                                 rows, N, d, static_cast<__nv_bfloat16*>(O), st);
   return cudaGetLastError();
 }
 

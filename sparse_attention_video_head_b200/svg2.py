@@ -16,7 +16,11 @@ from typing import Dict, Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsvg2.so")
+RELEASE_LIB_PATH = os.path.join(_PKG, "libsvg2.so")
+# The debug build: the same ABI, and every data-derived index a kernel clamps or skips is also latched
+# as SVG2_ERR_DEVICE_BOUNDS in the status word (built by build.build(debug=True)).
+DEBUG_LIB_PATH = os.path.join(_PKG, "libsvg2_debug.so")
+LIB_PATH = RELEASE_LIB_PATH
 
 SVG2_BF16, SVG2_F32 = 0, 1
 SVG2_INIT_GIVEN, SVG2_INIT_KMEANSPP = 0, 1
@@ -189,6 +193,13 @@ def svg2_check_status(ws: torch.Tensor, stream=None):
     _check(lib().svg2_check_status(_p(ws), _stream(stream), ctypes.byref(code), ctypes.byref(where), info),
            "svg2_check_status")
     return int(code.value), int(where.value), (int(info[0]), int(info[1]))
+
+
+def use_debug_library(on: bool = True) -> None:
+    """Make the following calls go to libsvg2_debug.so (on) or back to libsvg2.so (off)."""
+    global LIB_PATH, _lib
+    LIB_PATH = DEBUG_LIB_PATH if on else RELEASE_LIB_PATH
+    _lib = None
 
 
 def svg2_set_wait_budget(ws: torch.Tensor, cycles: int, stream=None):
