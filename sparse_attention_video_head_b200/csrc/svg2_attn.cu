@@ -295,15 +295,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mma_commit(smem_u32(&bars->k_empty[1]));
           }
         }
+        // P(j) is announced on the barriers of its slot, phase j/2: while this thread waits for V(j)
+        // the softmax may finish P(j+1) too, which on one shared barrier pair would complete two
+        // phases before the wait for the second half of P(j) looks, and that wait would never end.
+        // P(j+2) needs S(j+2), issued only after both halves of P(j) were taken, so a slot's
+        // barriers are never two phases ahead.
         for (int j = 0; j < T && ok; ++j) {
           const int stage = j & 1;
-          ok = mbar_wait(smem_u32(&bars->p_full[0][0]), j & 1, st, kWhereAttnMma, wb);
+          const uint32_t ppar = (j >> 1) & 1;
+          ok = mbar_wait(smem_u32(&bars->p_full[stage][0]), ppar, st, kWhereAttnMma, wb);
           if (ok) ok = mbar_wait(smem_u32(&bars->v_full[stage]), (j >> 1) & 1, st, kWhereAttnMma, wb);
           if (!ok) break;
           fence_proxy_async_smem();
           tc_fence_after();
           issue_pv(0, stage, stage, 0, j > 0);
-          ok = mbar_wait(smem_u32(&bars->p_full[0][1]), j & 1, st, kWhereAttnMma, wb);
+          ok = mbar_wait(smem_u32(&bars->p_full[stage][1]), ppar, st, kWhereAttnMma, wb);
           if (!ok) break;
           tc_fence_after();
           issue_pv(0, stage, stage, 1, true);
@@ -428,7 +434,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // runs under warp-uniform control flow; per-row decisions only select values.
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
-      // ring mode (no tile B): S(j) in slot j%2 (parity j/2 of that slot's barrier)
+      // ring mode (no tile B): S(j) and P(j) in slot j%2 (parity j/2 of that slot's barriers)
       const bool ring = !has_b;
       for (int j = 0; j < T; ++j) {
         const int slot = ring ? (j & 1) : x;
@@ -513,7 +519,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x][hh]));
+          if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[slot][hh]));
         }
         const float2 ls = add2(add2(lsum4[0], lsum4[1]), add2(lsum4[2], lsum4[3]));
         l += ls.x + ls.y;
