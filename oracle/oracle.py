@@ -50,6 +50,11 @@ def lib():
         L.svg2o_unpermute.argtypes = [P, P, i64, i32, P]
         L.svg2o_sparse_attention_rows.argtypes = [P, P, P, i64, i32, P, P, i32, i32, P, f64, P, i64, P]
         L.svg2o_dense_attention_rows.argtypes = [P, P, P, i64, i32, f64, P, i64, P]
+        L.svg2o_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.svg2o_e4m3_value.restype = f64
+        L.svg2o_e4m3_round.argtypes = [f64]
+        L.svg2o_e4m3_round.restype = ctypes.c_uint8
+        L.svg2o_quantize_e4m3.argtypes = [P, i64, P, P]
         _lib = L
     return _lib
 
@@ -169,6 +174,47 @@ def dense_attention_rows(Q, K, V, scale, rows=None):
     out = np.zeros((rows.size, d), np.float64)
     lib().svg2o_dense_attention_rows(_p(Q), _p(K), _p(V), N, d, float(scale), _p(rows), rows.size, _p(out))
     return out
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """Values of E4M3 codes (svg2o_e4m3_value), float64, same shape."""
+    c = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib().svg2o_e4m3_value(i) for i in range(256)], np.float64)
+    return table[c]
+
+
+def e4m3_round(x) -> np.ndarray:
+    """E4M3 codes of values (svg2o_e4m3_round: nearest, ties to even, saturating), uint8."""
+    a = np.asarray(x, dtype=np.float64)
+    return np.array([lib().svg2o_e4m3_round(float(v)) for v in a.ravel()], np.uint8).reshape(a.shape)
+
+
+def quantize_e4m3(X: np.ndarray):
+    """Per-plane E4M3 quantisation (svg2o_quantize_e4m3) of X [..., n_plane]: the leading axes index
+    planes, each quantised with its own scale.  Returns (codes uint8 like X, scale float32 [planes])."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    planes = X.reshape(X.shape[0], -1) if X.ndim > 1 else X.reshape(1, -1)
+    codes = np.zeros(planes.shape, np.uint8)
+    scale = np.zeros(planes.shape[0], np.float32)
+    for b in range(planes.shape[0]):
+        row = np.ascontiguousarray(planes[b])
+        out = np.zeros(row.size, np.uint8)
+        sc = np.zeros(1, np.float32)
+        lib().svg2o_quantize_e4m3(_p(row), row.size, _p(out), _p(sc))
+        codes[b] = out
+        scale[b] = sc[0]
+    return codes.reshape(X.shape), scale
+
+
+def sparse_attention_fp8_rows(Q8, K8, V8, sq: float, sk: float, sv: float, q_off, k_off, mask, scale, rows=None):
+    """The FP8 attention's definition for one (b,h): sparse_attention_rows over the dequantised
+    values q = e4m3_value(Q8) * sq (likewise k, v).  The codes' values are exact in float32, and the
+    plane scales are factored out of the sums: scores scale * sq * sk * (q8 . k8), output sv * (P v8)."""
+    q = e4m3_value(Q8).astype(np.float32)
+    k = e4m3_value(K8).astype(np.float32)
+    v = e4m3_value(V8).astype(np.float32)
+    out = sparse_attention_rows(q, k, v, q_off, k_off, mask, float(scale) * float(sq) * float(sk), rows)
+    return out * float(sv)
 
 
 def seed_candidates(N: int, seed_tokens: int) -> np.ndarray:

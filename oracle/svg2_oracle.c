@@ -334,3 +334,63 @@ void svg2o_dense_attention_rows(const float *Q, const float *K, const float *V, 
         attend_row(Q + rows[n] * d, K, V, d, scale, &lo, &hi, 1, out + n * d);
     }
 }
+
+/*
+ * E4M3, the 8-bit floating point format of the FP8 attention variant (the project's roadmap item
+ * "Support FP8 attention", GitHub README, Open-source Plan; the format is OCP's 8-bit floating point
+ * E4M3): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits.  Exponent field 0 holds the
+ * subnormals m * 2^-9; there are no infinities; S.1111.111 is NaN, so the largest finite magnitude
+ * is 1.75 * 2^8 = 448.  Value of one code.
+ */
+double svg2o_e4m3_value(uint8_t code) {
+    int e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (code & 0x80) ? -v : v;
+}
+
+/*
+ * Rounding to E4M3 as the quantiser defines it: the nearest finite code, a tie going to the code
+ * with the even mantissa, magnitudes beyond 448 to 448 (saturation); the sign is kept (so a
+ * negative value that rounds to zero gives -0, code 0x80); NaN gives 0x7F.  Brute force over the
+ * 127 finite non-negative codes, which are ordered by value.
+ */
+uint8_t svg2o_e4m3_round(double x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs(x), bd = INFINITY;
+    int best = 0;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double dd = fabs(svg2o_e4m3_value((uint8_t)c) - a);
+        if (dd < bd || (dd == bd && (c & 1) == 0)) {
+            best = c;
+            bd = dd;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/*
+ * Per-plane E4M3 quantisation (reading: the pages give no scaling scheme for their FP8 attention;
+ * one scale per (batch, head) plane is the plainest).  amax = max |x| over the n values, NaN
+ * entries ignored; if amax > 0, inv = fl32(448 / amax) and scale = fl32(amax / 448), else inv =
+ * scale = 1; codes[i] = e4m3_round(fl32(x[i] * inv)).  A code c stands for e4m3_value(c) * scale.
+ * The float32 steps are float32 operations (round to nearest), as the definition states them.
+ */
+void svg2o_quantize_e4m3(const float *X, int64_t n, uint8_t *codes, float *scale_out) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(X[i]);
+        if (a > amax) amax = a;  /* false for NaN */
+    }
+    float inv = 1.0f, scale = 1.0f;
+    if (amax > 0.0f) {
+        inv = 448.0f / amax;
+        scale = amax / 448.0f;
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        float y = X[i] * inv;
+        codes[i] = svg2o_e4m3_round((double)y);
+    }
+    *scale_out = scale;
+}

@@ -446,3 +446,88 @@ def test_oracle_results_do_not_depend_on_the_thread_count(oracle, tmp_path):
     assert set(outs[0].files) == set(outs[1].files)
     for key in outs[0].files:
         np.testing.assert_array_equal(outs[0][key], outs[1][key])
+
+
+# ---------------------------------------------------------------- FP8 attention variant (E4M3)
+
+def _torch_e4m3(x32):
+    """torch's own float32 -> float8_e4m3fn rounding, as codes (a library routine independent of the oracle)."""
+    return torch.from_numpy(np.asarray(x32, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_value_of_every_code_matches_torch(oracle):
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_value(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and set(np.flatnonzero(nan)) == {0x7F, 0xFF}
+    assert np.array_equal(ours[~nan], ref[~nan])
+    # the format's landmarks: smallest subnormal, smallest normal, one, largest finite
+    assert (ours[0x01], ours[0x08], ours[0x38], ours[0x7E]) == (2.0 ** -9, 2.0 ** -6, 1.0, 448.0)
+
+
+def test_e4m3_round_matches_torch_including_every_tie(oracle):
+    rng = np.random.default_rng(40)
+    x = np.concatenate([rng.standard_normal(3000) * 40, rng.standard_normal(1000) * 0.01,
+                        rng.uniform(-448, 448, 1000)]).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_round(x), _torch_e4m3(x))
+    # every midpoint between adjacent finite codes (exact in float32) is a tie: it goes to the even code
+    vals = oracle.e4m3_value(np.arange(0x7F, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    got = oracle.e4m3_round(mids)
+    assert np.all(got % 2 == 0)
+    assert np.array_equal(got, _torch_e4m3(mids))
+    assert np.array_equal(oracle.e4m3_round(-mids), _torch_e4m3(-mids))
+
+
+def test_e4m3_round_saturates_keeps_the_sign_of_zero_and_maps_nan(oracle):
+    assert list(oracle.e4m3_round([448.0, 460.0, 1e6, np.inf, -1e6])) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+    assert list(oracle.e4m3_round([0.0, -0.0, -1e-9, 2.0 ** -10, 3 * 2.0 ** -11])) == [0x00, 0x80, 0x80, 0x00, 0x01]
+    assert oracle.e4m3_round([np.nan])[0] == 0x7F
+
+
+def test_quantize_e4m3_maps_the_plane_maximum_to_448_and_bounds_the_error(oracle):
+    rng = np.random.default_rng(41)
+    X = (rng.standard_normal((3, 4000)) * np.array([[0.02], [1.0], [300.0]])).astype(np.float32)
+    X[1, 17] = np.nan  # ignored by the maximum, quantised to the NaN code
+    codes, scale = oracle.quantize_e4m3(X)
+    for b in range(3):
+        x = X[b]
+        amax = np.float32(np.nanmax(np.abs(x)))
+        assert scale[b] == np.float32(amax / np.float32(448))
+        inv = np.float32(np.float32(448) / amax)
+        ok = ~np.isnan(x)
+        # the rounding step is torch's own rounding of the same float32 products
+        assert np.array_equal(codes[b][ok], _torch_e4m3((x * inv)[ok]))
+        assert codes[b][np.argmax(np.where(ok, np.abs(x), -1))] & 0x7F == 0x7E
+        # dequantised values are within half a step of E4M3 (2^-4 relative above 2^-6, else 2^-10 absolute)
+        deq = oracle.e4m3_value(codes[b][ok]) * np.float64(scale[b])
+        y = x[ok].astype(np.float64)
+        bound = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10 * np.float64(scale[b])) * 1.0001
+        assert np.all(np.abs(deq - y) <= bound)
+    assert codes[1][17] == 0x7F
+    zc, zs = oracle.quantize_e4m3(np.zeros((1, 64), np.float32))
+    assert zs[0] == 1.0 and not zc.any()
+
+
+def test_fp8_attention_is_attention_over_the_dequantised_values(oracle):
+    rng = np.random.default_rng(42)
+    N, d, nQ, nK = 500, 32, 5, 7
+    lq = I.random_labels(N, nQ, 43, 0.2)
+    lk = I.random_labels(N, nK, 44, 0.2)
+    q_off = np.concatenate([[0], np.cumsum(np.bincount(lq, minlength=nQ))]).astype(np.int32)
+    k_off = np.concatenate([[0], np.cumsum(np.bincount(lk, minlength=nK))]).astype(np.int32)
+    (Q8, sq), (K8, sk), (V8, sv) = (oracle.quantize_e4m3(rng.standard_normal((1, N, d)).astype(np.float32) * s)
+                                    for s in (1.0, 3.0, 0.5))
+    mask = (rng.random((nQ, nK)) < 0.5).astype(np.uint8)
+    count_k = np.diff(k_off)
+    for i in range(nQ):
+        if not (mask[i] * (count_k > 0)).any():
+            mask[i, int(np.argmax(count_k))] = 1
+    scale = 1 / np.sqrt(d)
+    out = oracle.sparse_attention_fp8_rows(Q8[0], K8[0], V8[0], sq[0], sk[0], sv[0], q_off, k_off, mask, scale)
+    deq = [oracle.e4m3_value(c[0]) * np.float64(s[0]) for c, s in ((Q8, sq), (K8, sk), (V8, sv))]
+    cq = np.repeat(np.arange(nQ), np.diff(q_off))
+    ck = np.repeat(np.arange(nK), np.diff(k_off))
+    tok = mask[cq][:, ck].astype(bool)
+    np.testing.assert_allclose(out, _sdpa64(*deq, scale, tok), rtol=1e-9, atol=1e-12)
