@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--no-warm", action="store_true", help="skip the warm-start denoising-sequence measurement")
     ap.add_argument("--warm-steps", type=int, default=10)
     ap.add_argument("--no-layer-call", action="store_true", help="skip the single svg2_layer call at top-p 0.5")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 attention variant's record")
     ap.add_argument("--second", default="hunyuan720p", choices=["none"] + sorted(I.CONFIGS),
                     help="a second configuration measured after the first (stages, top-p sweep, dense attention)")
     ap.add_argument("--seed-tokens", type=int, default=16384,
@@ -358,11 +359,12 @@ class LayerBench:
         return out
 
 
-def time_layer_call(svg2, torch, lb, top_p, dense_ms, reps=3):
+def time_layer_call(svg2, torch, lb, top_p, dense_ms, reps=3, attn_fp8=0):
     """The whole layer as one svg2_layer call (k-means++ and Lloyd on Q and K, selection,
     permutation, attention with the fused inverse permutation) at `top_p`, timed with CUDA events."""
     cfg = lb.cfg
-    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, top_p, lb.scale, 1, lb.seed_tokens)
+    prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP, top_p, lb.scale, 1, lb.seed_tokens,
+                           attn_fp8)
     cq, ck = torch.zeros_like(lb.cq), torch.zeros_like(lb.ck)
     outs = svg2.layer_output_buffers(1, cfg.H, cfg.N, cfg.nQ, cfg.nK, device=lb.dev)
     svg2.svg2_layer(lb.Q, lb.K, lb.V, prm, cq, ck, lb.O, lb.ws, lb.uq, lb.uk, outs)
@@ -378,10 +380,73 @@ def time_layer_call(svg2, torch, lb, top_p, dense_ms, reps=3):
     cnt_q = outs["count_q"].cpu().numpy().astype(np.float64)
     sl = outs["stream_len"].cpu().numpy().astype(np.float64)
     density = float((cnt_q * sl).sum()) / (cfg.N * cfg.N * cfg.B * cfg.H)
-    out = {"api": "svg2_layer", "top_p": top_p, "density": density, "ms": ms, "reps": reps}
+    out = {"api": "svg2_layer", "top_p": top_p, "attn_fp8": attn_fp8, "density": density, "ms": ms, "reps": reps}
     if isinstance(dense_ms, float):
         out["dense_sdpa_ms"] = dense_ms
         out["speedup_vs_dense"] = dense_ms / ms
+    return out
+
+
+def measure_fp8(svg2, torch, lb, P, reps=5):
+    """The FP8 attention variant on the step's own plan (clusters, selection, permutation): the three
+    quantising gathers (E4M3 codes with per-(b,h) scales), the FP8 attention, the relative L2 of its
+    output against the bf16 attention's on every element, and the whole layer as one svg2_layer call
+    with attn_fp8 = 1.  The FP8 peak is the measured bf16 sustained peak times 2 (the nominal dense
+    E4M3 / bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
+    cfg, dev = lb.cfg, lb.dev
+    shape = (1, cfg.H, cfg.N, cfg.d)
+    Q8, K8, V8 = (torch.empty(shape, dtype=torch.uint8, device=dev) for _ in range(3))
+    sq, sk, sv = (torch.empty(1, cfg.H, dtype=torch.float32, device=dev) for _ in range(3))
+    O8 = torch.empty_like(lb.O)
+
+    def quantize():
+        svg2.svg2_quantize_e4m3(lb.Q, Q8, sq, perm=lb.perm_q)
+        svg2.svg2_quantize_e4m3(lb.K, K8, sk, perm=lb.perm_k)
+        svg2.svg2_quantize_e4m3(lb.V, V8, sv, perm=lb.perm_k)
+
+    def attend():
+        svg2.svg2_sparse_attn_fp8(Q8, K8, V8, sq, sk, sv, lb.q_off, lb.k_off, lb.sel_count, lb.sel_idx, lb.scale,
+                                  O8, lb.ws, perm_q=lb.perm_q)
+
+    lb.step()  # the plan again: earlier records (the all-token seeding, the warm start) re-cluster in place
+    quantize()
+    attend()
+    lb.attend()  # the bf16 output on the same plan, for the comparison
+    torch.cuda.synchronize(dev)
+    svg2.raise_on_device_error(lb.ws)
+    diff = (O8.float() - lb.O.float()).norm() / lb.O.float().norm()
+    # quantisation, then the FP8 and the bf16 attention interleaved on the same plan
+    eq = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    eq[0].record(lb.stream)
+    for _ in range(reps):
+        quantize()
+    eq[1].record(lb.stream)
+    ea = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for e in ea:
+        e[0].record(lb.stream)
+        attend()
+        e[1].record(lb.stream)
+        lb.attend()
+        e[2].record(lb.stream)
+    torch.cuda.synchronize(dev)
+    svg2.raise_on_device_error(lb.ws)
+    q_ms = eq[0].elapsed_time(eq[1]) / reps
+    a_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ea)
+    b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ea)
+    actual, _, _ = lb.flops()
+    tflops = actual / (a_ms * 1e-3) / 1e12
+    # per tensor: the maximum pass reads the bf16 plane, the gather reads it again and writes one byte
+    # per value, and reads one permutation entry per row
+    quant_bytes = 3 * (lb.Q.numel() * (2 + 2 + 1) + lb.perm_q.numel() * 4)
+    out = {"kernel": "sparse_attn_kernel<128, F8> (tcgen05 kind::f8f6f4)", "top_p": lb.top_p,
+           "quantize_ms": q_ms, "quantize_bytes": quant_bytes,
+           "quantize_gbs": quant_bytes / (q_ms * 1e-3) / 1e9, "attn_ms": a_ms, "attn_tflops_actual": tflops,
+           "peak_tflops": 2 * P["bf16_sustained"], "frac_of_fp8_sustained_peak": tflops / (2 * P["bf16_sustained"]),
+           "bf16_attn_ms_same_plan": b_ms, "speedup_vs_bf16_attn": b_ms / a_ms,
+           "rel_l2_vs_bf16_output": float(diff)}
+    del Q8, K8, V8, O8
+    out["layer_call"] = time_layer_call(svg2, torch, lb, lb.top_p, None, attn_fp8=1)
+    out["layer_call_bf16"] = time_layer_call(svg2, torch, lb, lb.top_p, None)
     return out
 
 
@@ -550,6 +615,10 @@ def main():
     if not args.no_layer_call and rank == 0:
         layer_call = time_layer_call(svg2, torch, lb, 0.5, dense_ms)
 
+    fp8 = None
+    if not args.no_fp8 and rank == 0:
+        fp8 = measure_fp8(svg2, torch, lb, P)
+
     second = None
     if args.second not in ("none", cfg.name) and not args.heads and rank == 0 and world == 1:
         second = measure_second_config(svg2, torch, I.CONFIGS[args.second], args, dev, P)
@@ -585,7 +654,7 @@ def main():
         "hbm_stages": hbm_stages,
         "dense_sdpa_ms": dense_ms, "dense_sdpa_backends_enabled": sdpa_backends(torch) if dense_ms is not None else None,
         "dense_svg2_dense_attn": own_dense, "denoise_driver": denoise, "warm_start": warm, "kmeans_all_token_seeding": full_seed,
-        "top_p_sweep": sweep, "layer_call_low_density": layer_call, "second_config": second,
+        "top_p_sweep": sweep, "layer_call_low_density": layer_call, "fp8_attention": fp8, "second_config": second,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -189,6 +189,38 @@ SVG2_API int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, co
                      size_t ws_bytes, void* stream);
 
 /*
+ * Per-head E4M3 quantisation for the FP8 attention variant (the project's roadmap item "Support FP8
+ * attention", GitHub README, Open-source Plan; the pages fix no scaling scheme, this is the plainest:
+ * one scale per (b,h) plane).  E4M3 is the OCP 8-bit floating point format with 4 exponent bits
+ * (bias 7), 3 mantissa bits, no infinities and 448 as its largest finite magnitude.  Per plane:
+ *   amax = max |x| (NaN entries ignored); inv = fl32(448 / amax); scale[bh] = fl32(amax / 448)
+ *   (inv = scale = 1 when amax == 0); X8[bh, r, :] = E4M3(fl32(X[bh, perm[r], :] * inv)), rounded
+ *   to nearest even, saturating at +-448.
+ * A code c stands for E4M3(c) * scale[bh].
+ *   X      [B,H,N,d] bf16 or f32 (dtype), 16-byte aligned.
+ *   perm   optional int32 [B,H,N] (NULL: the identity); entries outside [0, N) leave their row unwritten.
+ *   X8     uint8 [B,H,N,d], out, 16-byte aligned.  scale  float [B,H], out.
+ * Three kernels on `stream`, no workspace.  Errors: SVG2_ERR_INVALID_ARG (null or unaligned
+ * pointers, bad dtype), SVG2_ERR_UNSUPPORTED (sizes), SVG2_ERR_CUDA (launch). */
+SVG2_API int svg2_quantize_e4m3(const void* X, int dtype, const int32_t* perm, int B, int H, int N, int d, void* X8,
+                                float* scale, void* stream);
+
+/*
+ * The FP8 variant of svg2_sparse_attn (project roadmap item "Support FP8 attention"): the same
+ * variable-block sparse attention on E4M3 codes, with the products on the tensor core's 8-bit path
+ * (tcgen05 kind::f8f6f4).  Computes softmax(scale * q.k) v over the dequantised values
+ * q = E4M3(Qp8) * scale_q[bh] (likewise k, v); P is handed to the PV product as E4M3 (its values
+ * stay within [0, 256] by the lazy rescale), accumulation is float32, O is bf16.
+ *   Qp8, Kp8, Vp8  uint8 E4M3 codes [B,H,N,d], d = 128, permuted as for svg2_sparse_attn (16-byte aligned).
+ *   scale_q, scale_k, scale_v  float [B,H]: the planes' dequantisation scales (svg2_quantize_e4m3).
+ *   Other arguments, workspace and errors as svg2_sparse_attn; d != 128 gives SVG2_ERR_UNSUPPORTED. */
+SVG2_API int svg2_sparse_attn_fp8(const void* Qp8, const void* Kp8, const void* Vp8, const float* scale_q,
+                                  const float* scale_k, const float* scale_v, const int32_t* q_off,
+                                  const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int B,
+                                  int H, int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Dense attention, O = softmax(scale * Q K^T) V per (b,h) over all N keys, on the same tcgen05
  * kernel as svg2_sparse_attn: the one-cluster case (one Q cluster and one K cluster holding every
  * token in its original order), so no permutation and no k-means.  This is the layer the pages run
@@ -216,6 +248,8 @@ typedef struct {
   int seed_tokens;     /* k-means++ candidates, as in svg2_kmeans (0 = all tokens) */
   int fuse_unpermute;  /* 1: write O in token order from the attention epilogue (default path);
                           0: write permuted rows, then run svg2_unpermute */
+  int attn_fp8;        /* 0: bf16 attention; 1: the FP8 variant (d = 128): the gathers write per-head
+                          E4M3 codes of Q, K, V (as svg2_quantize_e4m3) and svg2_sparse_attn_fp8 runs */
 } svg2_params;
 
 /* Optional device buffers for the layer's intermediate results.  Any NULL field is kept inside

@@ -70,6 +70,7 @@ struct LayerCarve {
   int32_t *sel_count, *sel_idx, *stream_len;
   void *Qp, *Kp, *Vp, *Op;
   AttnScratch attn;
+  uint32_t* f8;  // FP8 attention: per-plane maxima, then scales, of Q [BH], K [BH], V [BH]
 };
 
 void carve_layer(Carve& c, int BH, int N, int d, int nQ, int nK, const svg2_layer_outputs* o, LayerCarve& L) {
@@ -96,6 +97,7 @@ void carve_layer(Carve& c, int BH, int N, int d, int nQ, int nK, const svg2_laye
   L.Vp = c.take<uint16_t>(BHN * d);
   L.Op = c.take<uint16_t>(BHN * d);
   carve_attn(c, BH, N, nQ, L.attn);
+  L.f8 = c.take<uint32_t>(3 * static_cast<size_t>(BH));
 }
 
 // Bytes from the start of the permuted Q plane to the end of the permuted K plane: both are free
@@ -149,6 +151,20 @@ cudaError_t make_tmap_bf16_rows(void* map, const void* base, uint64_t rows, uint
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
                         dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_u8_rows(void* map, const void* base, uint64_t rows, uint32_t d, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  if (!aligned(base, 16) || rows == 0 || d != 128 || box_rows == 0 || box_rows > 256) return cudaErrorInvalidValue;
+  const cuuint64_t dims[2] = {d, rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d)};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -396,6 +412,59 @@ int svg2_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32
   }
 }
 
+int svg2_quantize_e4m3(const void* X, int dtype, const int32_t* perm, int B, int H, int N, int d, void* X8,
+                       float* scale, void* stream) {
+  try {
+    const int r = check_sizes(B, H, N, d);
+    if (r != SVG2_OK) return r;
+    if (!valid_dtype(dtype) || X == nullptr || X8 == nullptr || scale == nullptr) return SVG2_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(X8, 16) || !aligned(scale, 4)) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    const bool f32 = dtype == SVG2_F32;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* amax = reinterpret_cast<uint32_t*>(scale);  // the maxima live in `scale` until the last pass
+    cudaError_t e = launch_amax(X, nullptr, nullptr, 1, f32, BH, N, d, amax, s);
+    if (e == cudaSuccess) e = launch_gather_e4m3(X, nullptr, f32, perm, BH, N, d, amax, nullptr, X8, nullptr, s, nullptr);
+    if (e == cudaSuccess) e = launch_amax_to_scale(amax, BH, s);
+    return to_status(e);
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
+int svg2_sparse_attn_fp8(const void* Qp8, const void* Kp8, const void* Vp8, const float* scale_q, const float* scale_k,
+                         const float* scale_v, const int32_t* q_off, const int32_t* k_off, const int32_t* sel_count,
+                         const int32_t* sel_idx, int B, int H, int N, int d, int nQ, int nK, float scale,
+                         const int32_t* perm_q, void* O, void* ws, size_t ws_bytes, void* stream) {
+  try {
+    int r = check_sizes(B, H, N, d);
+    if (r == SVG2_OK) r = check_k(nQ, N);
+    if (r == SVG2_OK) r = check_k(nK, N);
+    if (r != SVG2_OK) return r;
+    if (d != 128) return SVG2_ERR_UNSUPPORTED;
+    if (Qp8 == nullptr || Kp8 == nullptr || Vp8 == nullptr || scale_q == nullptr || scale_k == nullptr ||
+        scale_v == nullptr || q_off == nullptr || k_off == nullptr || sel_count == nullptr || sel_idx == nullptr ||
+        O == nullptr)
+      return SVG2_ERR_INVALID_ARG;
+    if (!aligned(Qp8, 16) || !aligned(Kp8, 16) || !aligned(Vp8, 16) || !aligned(O, 16) || !aligned(scale_q, 4) ||
+        !aligned(scale_k, 4) || !aligned(scale_v, 4))
+      return SVG2_ERR_INVALID_ARG;
+    if (scale != scale) return SVG2_ERR_INVALID_ARG;
+    const int BH = B * H;
+    Carve c(ws);
+    DeviceStatus* st = c.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));
+    AttnScratch a;
+    carve_attn(c, BH, N, nQ, a);
+    r = check_ws(ws, ws_bytes, c.off);
+    if (r != SVG2_OK) return r;
+    return to_status(launch_sparse_attn_fp8(Qp8, Kp8, Vp8, F8Scales{scale_q, scale_k, scale_v}, q_off, k_off,
+                                            sel_count, sel_idx, BH, N, d, nQ, nK, scale, perm_q, O, a, st,
+                                            wait_budget_of(st), static_cast<cudaStream_t>(stream)));
+  } catch (...) {
+    return SVG2_ERR_CUDA;
+  }
+}
+
 namespace {
 struct DenseCarve {
   DeviceStatus* st;
@@ -476,6 +545,8 @@ static int check_layer_params(const svg2_params* p, int dtype, int B, int H, int
   if (!(p->top_p > 0.f) || p->scale != p->scale) return SVG2_ERR_INVALID_ARG;
   if (cq == nullptr || ck == nullptr) return SVG2_ERR_INVALID_ARG;
   if (p->init == SVG2_INIT_KMEANSPP && (uq == nullptr || uk == nullptr)) return SVG2_ERR_INVALID_ARG;
+  if (p->attn_fp8 != 0 && p->attn_fp8 != 1) return SVG2_ERR_INVALID_ARG;
+  if (p->attn_fp8 && d != 128) return SVG2_ERR_UNSUPPORTED;
   return SVG2_OK;
 }
 
@@ -508,9 +579,25 @@ int svg2_layer(const void* Q, const void* K, const void* V, int dtype, int B, in
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, L.weights, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);
-    if (e == cudaSuccess) e = launch_gather(Q, f32, L.perm_q, BH, N, d, L.Qp, s, L.st);
-    if (e == cudaSuccess) e = launch_gather2(K, V, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s, L.st);
-    if (e == cudaSuccess) {
+    const F8Scales f8{reinterpret_cast<const float*>(L.f8), reinterpret_cast<const float*>(L.f8 + BH),
+                      reinterpret_cast<const float*>(L.f8 + 2 * BH)};
+    if (p->attn_fp8) {
+      // E4M3 rows go to the first half of each permuted bf16 plane's room
+      if (e == cudaSuccess) e = launch_amax(Q, K, V, 3, f32, BH, N, d, L.f8, s);
+      if (e == cudaSuccess) e = launch_gather_e4m3(Q, nullptr, f32, L.perm_q, BH, N, d, L.f8, nullptr, L.Qp, nullptr, s, L.st);
+      if (e == cudaSuccess)
+        e = launch_gather_e4m3(K, V, f32, L.perm_k, BH, N, d, L.f8 + BH, L.f8 + 2 * BH, L.Kp, L.Vp, s, L.st);
+      if (e == cudaSuccess) e = launch_amax_to_scale(L.f8, 3 * BH, s);
+    } else {
+      if (e == cudaSuccess) e = launch_gather(Q, f32, L.perm_q, BH, N, d, L.Qp, s, L.st);
+      if (e == cudaSuccess) e = launch_gather2(K, V, f32, L.perm_k, BH, N, d, L.Kp, L.Vp, s, L.st);
+    }
+    if (e == cudaSuccess && p->attn_fp8) {
+      e = launch_sparse_attn_fp8(L.Qp, L.Kp, L.Vp, f8, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ,
+                                 p->nK, p->scale, p->fuse_unpermute ? L.perm_q : nullptr, p->fuse_unpermute ? O : L.Op,
+                                 L.attn, L.st, wait_budget_of(L.st), s);
+      if (e == cudaSuccess && !p->fuse_unpermute) e = launch_unpermute(L.Op, L.perm_q, BH, N, d, O, s, L.st);
+    } else if (e == cudaSuccess) {
       if (p->fuse_unpermute) {
         e = launch_sparse_attn(L.Qp, L.Kp, L.Vp, L.q_off, L.k_off, L.sel_count, L.sel_idx, BH, N, d, p->nQ, p->nK,
                                p->scale, L.perm_q, O, L.attn, L.st, wait_budget_of(L.st), s);
@@ -645,7 +732,14 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     if (e == cudaSuccess)
       e = launch_select(cq, ck, nullptr, L.count_k, BH, p->nQ, p->nK, d, p->top_p, p->scale, nullptr, L.mask,
                         L.sel_count, L.sel_idx, L.stream_len, s);
-    if (e == cudaSuccess) e = launch_gather(Qd, f32, L.perm_q, BH, N, d, L.Qp, s, L.st);
+    // FP8 attention: L.f8 holds Q's scales [BH], then per group its K scales and V scales [hn each]
+    if (p->attn_fp8) {
+      if (e == cudaSuccess) e = launch_amax(Qd, nullptr, nullptr, 1, f32, BH, N, d, L.f8, s);
+      if (e == cudaSuccess) e = launch_gather_e4m3(Qd, nullptr, f32, L.perm_q, BH, N, d, L.f8, nullptr, L.Qp, nullptr, s, L.st);
+      if (e == cudaSuccess) e = launch_amax_to_scale(L.f8, BH, s);
+    } else if (e == cudaSuccess) {
+      e = launch_gather(Qd, f32, L.perm_q, BH, N, d, L.Qp, s, L.st);
+    }
     // per head group: gather its K and V planes once its V has landed, attend, and copy the output
     // back while the next group runs
     const size_t plane_p = static_cast<size_t>(N) * d;  // elements of one permuted plane
@@ -653,18 +747,40 @@ int svg2_layer_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, vo
     for (int g = 0; g < ngroups && e == cudaSuccess; h0 += static_cast<size_t>(gsize[g]), ++g) {
       const int hn = gsize[g];
       ok(cudaStreamWaitEvent(s, v_in[g], 0));
-      if (e == cudaSuccess)
-        e = launch_gather2(static_cast<const char*>(Kd) + h0 * plane_in, static_cast<const char*>(Vd) + h0 * plane_in,
-                           f32, L.perm_k + h0 * N, hn, N, d, static_cast<uint16_t*>(L.Kp) + h0 * plane_p,
-                           static_cast<uint16_t*>(L.Vp) + h0 * plane_p, s, L.st);
-      if (e != cudaSuccess) break;
-      e = launch_sparse_attn(static_cast<const uint16_t*>(L.Qp) + h0 * plane_p,
-                             static_cast<const uint16_t*>(L.Kp) + h0 * plane_p,
-                             static_cast<const uint16_t*>(L.Vp) + h0 * plane_p, L.q_off + h0 * (p->nQ + 1),
-                             L.k_off + h0 * (p->nK + 1), L.sel_count + h0 * p->nQ,
-                             L.sel_idx + h0 * static_cast<size_t>(p->nQ) * p->nK, hn, N, d, p->nQ, p->nK, p->scale,
-                             L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st,
-                             wait_budget_of(L.st), s);
+      if (p->attn_fp8) {
+        const char* kg = static_cast<const char*>(Kd) + h0 * plane_in;
+        const char* vg = static_cast<const char*>(Vd) + h0 * plane_in;
+        uint32_t* fk = L.f8 + BH + 2 * h0;  // this group's K scales, then its V scales
+        if (e == cudaSuccess) e = launch_amax(kg, vg, nullptr, 2, f32, hn, N, d, fk, s);
+        if (e == cudaSuccess)
+          e = launch_gather_e4m3(kg, vg, f32, L.perm_k + h0 * N, hn, N, d, fk, fk + hn,
+                                 static_cast<uint8_t*>(L.Kp) + h0 * plane_p, static_cast<uint8_t*>(L.Vp) + h0 * plane_p,
+                                 s, L.st);
+        if (e == cudaSuccess) e = launch_amax_to_scale(fk, 2 * hn, s);
+        if (e != cudaSuccess) break;
+        const F8Scales f8{reinterpret_cast<const float*>(L.f8) + h0, reinterpret_cast<const float*>(fk),
+                          reinterpret_cast<const float*>(fk + hn)};
+        e = launch_sparse_attn_fp8(static_cast<const uint8_t*>(L.Qp) + h0 * plane_p,
+                                   static_cast<const uint8_t*>(L.Kp) + h0 * plane_p,
+                                   static_cast<const uint8_t*>(L.Vp) + h0 * plane_p, f8, L.q_off + h0 * (p->nQ + 1),
+                                   L.k_off + h0 * (p->nK + 1), L.sel_count + h0 * p->nQ,
+                                   L.sel_idx + h0 * static_cast<size_t>(p->nQ) * p->nK, hn, N, d, p->nQ, p->nK,
+                                   p->scale, L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st,
+                                   wait_budget_of(L.st), s);
+      } else {
+        if (e == cudaSuccess)
+          e = launch_gather2(static_cast<const char*>(Kd) + h0 * plane_in, static_cast<const char*>(Vd) + h0 * plane_in,
+                             f32, L.perm_k + h0 * N, hn, N, d, static_cast<uint16_t*>(L.Kp) + h0 * plane_p,
+                             static_cast<uint16_t*>(L.Vp) + h0 * plane_p, s, L.st);
+        if (e != cudaSuccess) break;
+        e = launch_sparse_attn(static_cast<const uint16_t*>(L.Qp) + h0 * plane_p,
+                               static_cast<const uint16_t*>(L.Kp) + h0 * plane_p,
+                               static_cast<const uint16_t*>(L.Vp) + h0 * plane_p, L.q_off + h0 * (p->nQ + 1),
+                               L.k_off + h0 * (p->nK + 1), L.sel_count + h0 * p->nQ,
+                               L.sel_idx + h0 * static_cast<size_t>(p->nQ) * p->nK, hn, N, d, p->nQ, p->nK, p->scale,
+                               L.perm_q + h0 * N, static_cast<char*>(Od) + h0 * plane_out, L.attn, L.st,
+                               wait_budget_of(L.st), s);
+      }
       ok(cudaEventRecord(o_out[g], s));
       ok(cudaStreamWaitEvent(cs, o_out[g], 0));
       ok(cudaMemcpyAsync(static_cast<char*>(Oh) + h0 * plane_out, static_cast<const char*>(Od) + h0 * plane_out,

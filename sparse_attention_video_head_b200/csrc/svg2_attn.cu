@@ -43,16 +43,21 @@ constexpr int kSoftmaxRegs = 184;
 constexpr int kOtherRegs = 120;
 static_assert(256 * kSoftmaxRegs + (kAttnThreads - 256) * kOtherRegs <= kAttnThreads * kLaunchRegs, "register split");
 constexpr int kMaxRanges = 1024;
-// bytes of one 128-row tile of d bf16 values (d/64 swizzled 16 KB halves)
-template <int D>
-constexpr uint32_t tile_bytes() { return 128u * D * 2u; }
-template <int D>
-constexpr uint32_t attn_smem() { return 6 * tile_bytes<D>() + 1024 /*align*/ + 4096 /*ranges*/ + 4096 + 64 /*cum*/ + 256; }
+// bytes of one 128-row tile of d values: bf16, or E4M3 codes in the FP8 variant (16 KB column blocks of
+// 128-byte swizzled rows)
+template <int D, bool F8>
+constexpr uint32_t tile_bytes() { return 128u * D * (F8 ? 1u : 2u); }
+template <int D, bool F8>
+constexpr uint32_t attn_smem() {
+  return 6 * tile_bytes<D, F8>() + 1024 /*align*/ + 4096 /*ranges*/ + 4096 + 64 /*cum*/ + 256;
+}
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 16 key pairs of a row, this many (the last ones) get 2^x from the cubic on the FMA pipe;
 // the rest use the MUFU, whose 16 exponentials per clock per SM would otherwise bound the softmax.
+// The FP8 instance's products take half the time, so more of its exponentials go to the FMA pipe.
 constexpr int kCubicPairs = 4;
+constexpr int kCubicPairsF8 = 4;
 
 struct AttnBars {
   uint64_t q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], o_full, mma_done;
@@ -117,23 +122,28 @@ __global__ void plan_write_kernel(const int32_t* __restrict__ q_off, int nQ, int
   }
 }
 
-template <int D>
+// F8: Q, K, V are E4M3 codes with one scale per (b,h) plane each (f8.q, f8.k, f8.v): the scores take
+// sq * sk into the softmax scale, the output sv into its normaliser, and P goes to the PV product as
+// E4M3.
+template <int D, bool F8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ Kp,
-                       const __nv_bfloat16* __restrict__ Vp, const int32_t* __restrict__ k_off,
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const uint8_t* __restrict__ Kp,
+                       const uint8_t* __restrict__ Vp, const int32_t* __restrict__ k_off,
                        const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_idx, int N, int nQ,
                        int nK, float scale, const int32_t* __restrict__ perm_q, __nv_bfloat16* __restrict__ O,
                        const AttnUnit* __restrict__ units, const int32_t* __restrict__ head_base, int BH,
-                       DeviceStatus* st, const uint64_t* __restrict__ wait_budget) {
+                       const F8Scales f8, DeviceStatus* st, const uint64_t* __restrict__ wait_budget) {
   const int total_units = head_base[BH];
   if (static_cast<int>(blockIdx.x) >= total_units) return;
   if (status_set(st)) return;
   const long long wb = effective_wait_budget(wait_budget);
   const AttnUnit un = units[blockIdx.x];
 
-  constexpr uint32_t kTile = tile_bytes<D>();
-  constexpr int kHalves = D / 64;   // 128-byte swizzle atoms across d
-  constexpr int kSteps = D / 16;    // K=16 MMA steps across d
+  constexpr uint32_t kTile = tile_bytes<D, F8>();
+  constexpr int kRowBytes = D * (F8 ? 1 : 2);
+  constexpr int kHalves = kRowBytes / 128;  // 128-byte swizzle atoms across a row
+  constexpr int kKStep = F8 ? 32 : 16;       // contraction elements (32 bytes) per MMA instruction
+  constexpr int kSteps = D / kKStep;         // instructions of one S product
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;                 // Q_A, Q_B
@@ -235,12 +245,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int y = bh * N + un.row0;
 #pragma unroll
       for (int hf = 0; hf < kHalves; ++hf) {
-        tma_load_2d(qa + hf * 16384, &tm_q, hf * 64, y, qbar);
-        if (has_b) tma_load_2d(qb + hf * 16384, &tm_q, hf * 64, y + 128, qbar);
+        tma_load_2d(qa + hf * 16384, &tm_q, hf * (128 / (kRowBytes / D)), y, qbar);
+        if (has_b) tma_load_2d(qb + hf * 16384, &tm_q, hf * (128 / (kRowBytes / D)), y + 128, qbar);
       }
       bool ok = mbar_wait(qbar, 0, st, kWhereAttnMma, wb);
-      const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
-      const uint32_t id_o = idesc_bf16_f32(128, D, 1);
+      const uint32_t id_s = F8 ? idesc_e4m3_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0);
+      const uint32_t id_o = F8 ? idesc_e4m3_f32(128, D, 1) : idesc_bf16_f32(128, D, 1);
       const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
       // Descriptors of every operand tile, built once: stepping along K only moves the start
       // address field (bits 0-13, in 16-byte units), which stays far below its 14-bit limit.
@@ -256,20 +266,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < kSteps; ++ks) {
           const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-          mma_ss(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
+          if constexpr (F8) mma_ss_f8(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
+          else mma_ss(d_tmem, aq + koff, bk + koff, id_s, ks > 0 ? 1u : 0u);
         }
         mma_commit(smem_u32(&bars->s_full[slot]));
       };
-      // O_x += P(j) V(j) over keys 64h .. 64h+63: P is bf16 pair-packed in the first 64 columns
-      // of its S slot, the keys of half h in columns 32h .. 32h+31
+      // O_x += P(j) V(j) over keys 64h .. 64h+63: P is packed in the first columns of its S slot,
+      // two bf16 or four E4M3 keys per 32-bit column, so each instruction's kKStep keys take 8
+      // columns and kKStep 128-byte rows of V
       auto issue_pv = [&](int x, int slot, int stage, int h, bool acc) {
+        constexpr int kPvSteps = 64 / kKStep;
         const uint32_t d_tmem = tmem + 256 + x * 128;
         const uint32_t p_tmem = tmem + slot * 128;
         const uint64_t bv = stage == 0 ? dv0 : dv1;
 #pragma unroll
-        for (int ks = 4 * h; ks < 4 * h + 4; ++ks)
-          mma_ts(d_tmem, p_tmem + ks * 8, bv + static_cast<uint64_t>((ks * 2048) >> 4), id_o,
-                 (acc || ks > 0) ? 1u : 0u);
+        for (int ks = kPvSteps * h; ks < kPvSteps * h + kPvSteps; ++ks) {
+          const uint64_t voff = static_cast<uint64_t>((ks * kKStep * 128) >> 4);
+          if constexpr (F8) mma_ts_f8(d_tmem, p_tmem + ks * 8, bv + voff, id_o, (acc || ks > 0) ? 1u : 0u);
+          else mma_ts(d_tmem, p_tmem + ks * 8, bv + voff, id_o, (acc || ks > 0) ? 1u : 0u);
+        }
       };
       if (ok && T > 0) {
         ok = mbar_wait(smem_u32(&bars->k_full[0]), 0, st, kWhereAttnMma, wb);
@@ -374,7 +389,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // table (positions only grow, so each cursor crosses every range boundary once, where a search
     // per tile would cost a chain of dependent shared-memory reads); then every cp.async instruction
     // moves whole rows (16 lanes x 16 bytes per row at d = 128), so one instruction touches 2 rows.
-    constexpr int CPR = D / 8;       // 16-byte chunks per row
+    constexpr int CPR = kRowBytes / 16;  // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;    // rows per warp instruction
     const int wr0 = (warp - kProducerWarp0) * 64;
     const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
@@ -402,7 +417,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int it = 0; it < 64 / RPI; ++it) {
         const int rr = it * RPI + my_sub;  // row within the warp's 64
         const int src = __shfl_sync(0xffffffffu, rr < 32 ? krow0 : krow1, rr & 31);
-        cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * D + my_chunk * 8);
+        cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * kRowBytes + my_chunk * 16);
       }
       cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->v_empty[stage]), ((j >> 1) - 1) & 1, st,
@@ -412,7 +427,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int it = 0; it < 64 / RPI; ++it) {
         const int rr = it * RPI + my_sub;
         const int src = __shfl_sync(0xffffffffu, rr < 32 ? krow0 : krow1, rr & 31);
-        cp_async16(vdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Vp + (head_row0 + src) * D + my_chunk * 8);
+        cp_async16(vdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Vp + (head_row0 + src) * kRowBytes + my_chunk * 16);
       }
       cp_async_mbar_arrive(smem_u32(&bars->v_full[stage]));
     }
@@ -429,7 +444,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else {
       const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
       const uint32_t t_o = tmem + lane_off + 256 + x * 128;
-      const float sl2 = scale * kLog2e;
+      const float sl2 = F8 ? scale * kLog2e * f8.q[bh] * f8.k[bh] : scale * kLog2e;
       // Every tcgen05.ld/st below is a warp-collective (.sync.aligned) instruction, so all of it
       // runs under warp-uniform control flow; per-row decisions only select values.
       float m_used = -INFINITY, l = 0.f;
@@ -504,18 +519,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // second half's exponentials are computed
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          auto p_pair = [&](int e) {  // p of keys 64hh + 2e, 64hh + 2e + 1
             const int col = hh * 64 + 2 * e;
             const float2 t = fma2(make_float2(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), scl, negm);
-            float2 pe;
-            if ((e & 15) >= 16 - kCubicPairs) pe = exp2_cubic2(t);
-            else pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-            pk[e] = pack_bf16x2(pe.x, pe.y);
+            const float2 pe = ((e & 15) >= 16 - (F8 ? kCubicPairsF8 : kCubicPairs)) ? exp2_cubic2(t)
+                                                             : make_float2(fast_exp2(t.x), fast_exp2(t.y));
             lsum4[e & 3] = add2(lsum4[e & 3], pe);
+            return pe;
+          };
+          if constexpr (F8) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 a = p_pair(2 * e), b = p_pair(2 * e + 1);
+              pk[e] = pack_e4m3x4(a.x, a.y, b.x, b.y);
+            }
+            tmem_st16(t_sj + hh * 16, pk);
+          } else {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float2 pe = p_pair(e);
+              pk[e] = pack_bf16x2(pe.x, pe.y);
+            }
+            tmem_st32(t_sj + hh * 32, pk);
           }
-          tmem_st32(t_sj + hh * 32, pk);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -536,7 +564,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (tk < 0 || tk >= N) tk = -1;  // an invalid permutation entry is skipped
         }
         uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<size_t>(bh) * N + (tk < 0 ? 0 : tk)) * D);
-        const float inv = (T > 0 && l > 0.f) ? 1.f / l : 0.f;
+        const float inv = (T > 0 && l > 0.f) ? (F8 ? f8.v[bh] : 1.f) / l : 0.f;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -708,34 +736,63 @@ cudaError_t launch_dense_plan(int BH, int N, int32_t* q_off, int32_t* k_off, int
   return cudaGetLastError();
 }
 
+namespace {
+
+template <int D, bool F8>
+cudaError_t launch_attn_kernel(const CUtensorMap& tq, const void* Kp, const void* Vp, const int32_t* k_off,
+                               const int32_t* sel_count, const int32_t* sel_idx, int BH, int N, int nQ, int nK,
+                               float scale, const int32_t* perm_q, void* O, const AttnScratch& sc,
+                               const F8Scales& f8, DeviceStatus* st, const uint64_t* wait_budget, cudaStream_t s) {
+  constexpr uint32_t smem = attn_smem<D, F8>();
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const long long grid = static_cast<long long>(BH) * attn_max_units_per_head(N, nQ);
+  sparse_attn_kernel<D, F8><<<static_cast<unsigned>(grid), kAttnThreads, smem, s>>>(
+      tq, static_cast<const uint8_t*>(Kp), static_cast<const uint8_t*>(Vp), k_off, sel_count, sel_idx, N, nQ, nK,
+      scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, f8, st, wait_budget);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_plan(const int32_t* q_off, int BH, int N, int nQ, const AttnScratch& sc, DeviceStatus* st,
+                             cudaStream_t s) {
+  plan_count_kernel<<<BH, 256, 0, s>>>(q_off, nQ, N, sc.head_units, st);
+  plan_scan_kernel<<<1, 32, 0, s>>>(sc.head_units, BH, sc.head_base);
+  plan_write_kernel<<<BH, 32, 0, s>>>(q_off, nQ, N, sc.head_base, sc.units);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
                                const int32_t* k_off, const int32_t* sel_count, const int32_t* sel_idx, int BH,
                                int N, int d, int nQ, int nK, float scale, const int32_t* perm_q, void* O,
                                const AttnScratch& sc, DeviceStatus* st, const uint64_t* wait_budget,
                                cudaStream_t s) {
-  plan_count_kernel<<<BH, 256, 0, s>>>(q_off, nQ, N, sc.head_units, st);
-  plan_scan_kernel<<<1, 32, 0, s>>>(sc.head_units, BH, sc.head_base);
-  plan_write_kernel<<<BH, 32, 0, s>>>(q_off, nQ, N, sc.head_base, sc.units);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_attn_plan(q_off, BH, N, nQ, sc, st, s);
   if (e != cudaSuccess) return e;
   alignas(64) CUtensorMap tq;
   e = make_tmap_bf16_rows(&tq, Qp, static_cast<uint64_t>(BH) * N, static_cast<uint32_t>(d), 128);
   if (e != cudaSuccess) return e;
-  const long long grid = static_cast<long long>(BH) * attn_max_units_per_head(N, nQ);
-  if (d == 128) {
-    e = cudaFuncSetAttribute(sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<128>());
-    if (e != cudaSuccess) return e;
-    sparse_attn_kernel<128><<<static_cast<unsigned>(grid), kAttnThreads, attn_smem<128>(), s>>>(
-        tq, static_cast<const __nv_bfloat16*>(Kp), static_cast<const __nv_bfloat16*>(Vp), k_off, sel_count, sel_idx,
-        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st, wait_budget);
-  } else {
-    e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<64>());
-    if (e != cudaSuccess) return e;
-    sparse_attn_kernel<64><<<static_cast<unsigned>(grid), kAttnThreads, attn_smem<64>(), s>>>(
-        tq, static_cast<const __nv_bfloat16*>(Kp), static_cast<const __nv_bfloat16*>(Vp), k_off, sel_count, sel_idx,
-        N, nQ, nK, scale, perm_q, static_cast<__nv_bfloat16*>(O), sc.units, sc.head_base, BH, st, wait_budget);
-  }
-  return cudaGetLastError();
+  if (d == 128)
+    return launch_attn_kernel<128, false>(tq, Kp, Vp, k_off, sel_count, sel_idx, BH, N, nQ, nK, scale, perm_q, O, sc,
+                                          F8Scales{}, st, wait_budget, s);
+  return launch_attn_kernel<64, false>(tq, Kp, Vp, k_off, sel_count, sel_idx, BH, N, nQ, nK, scale, perm_q, O, sc,
+                                       F8Scales{}, st, wait_budget, s);
+}
+
+cudaError_t launch_sparse_attn_fp8(const void* Qp8, const void* Kp8, const void* Vp8, const F8Scales& f8,
+                                   const int32_t* q_off, const int32_t* k_off, const int32_t* sel_count,
+                                   const int32_t* sel_idx, int BH, int N, int d, int nQ, int nK, float scale,
+                                   const int32_t* perm_q, void* O, const AttnScratch& sc, DeviceStatus* st,
+                                   const uint64_t* wait_budget, cudaStream_t s) {
+  if (d != 128) return cudaErrorInvalidValue;
+  cudaError_t e = launch_attn_plan(q_off, BH, N, nQ, sc, st, s);
+  if (e != cudaSuccess) return e;
+  alignas(64) CUtensorMap tq;
+  e = make_tmap_u8_rows(&tq, Qp8, static_cast<uint64_t>(BH) * N, static_cast<uint32_t>(d), 128);
+  if (e != cudaSuccess) return e;
+  return launch_attn_kernel<128, true>(tq, Kp8, Vp8, k_off, sel_count, sel_idx, BH, N, nQ, nK, scale, perm_q, O, sc,
+                                       f8, st, wait_budget, s);
 }
 
 cudaError_t launch_selftest_mma(const void* A, const void* Bm, int n, const void* V, float* C, float* O,

@@ -186,6 +186,28 @@ cudaError_t launch_sparse_attn(const void* Qp, const void* Kp, const void* Vp, c
                                const AttnScratch& scratch, DeviceStatus* st, const uint64_t* wait_budget,
                                cudaStream_t s);
 
+// Dequantisation scales of the FP8 attention: one float per (b,h) plane of Q, K and V.
+struct F8Scales {
+  const float* q = nullptr;
+  const float* k = nullptr;
+  const float* v = nullptr;
+};
+// FP8 variant (d = 128): Qp8, Kp8, Vp8 E4M3 codes [BH,N,d], value = E4M3(code) * scale of the plane.
+cudaError_t launch_sparse_attn_fp8(const void* Qp8, const void* Kp8, const void* Vp8, const F8Scales& f8,
+                                   const int32_t* q_off, const int32_t* k_off, const int32_t* sel_count,
+                                   const int32_t* sel_idx, int BH, int N, int d, int nQ, int nK, float scale,
+                                   const int32_t* perm_q, void* O, const AttnScratch& sc, DeviceStatus* st,
+                                   const uint64_t* wait_budget, cudaStream_t s);
+// Per-head E4M3 quantisation (svg2_fp8.cu).  launch_amax zeroes amax [tensors][BH] and writes the
+// float bits of max |x| per plane; launch_gather_e4m3 writes Y[r] = E4M3(X[bh, perm[r]] * 448 / amax)
+// (perm may be null: the identity; X1/Y1 may be null); launch_amax_to_scale turns each amax into
+// the dequantisation scale amax / 448 in place (1 for an all-zero plane).
+cudaError_t launch_amax(const void* X0, const void* X1, const void* X2, int tensors, bool f32, int BH, int N, int d,
+                        uint32_t* amax, cudaStream_t s);
+cudaError_t launch_gather_e4m3(const void* X0, const void* X1, bool f32, const int32_t* perm, int BH, int N, int d,
+                               const uint32_t* amax0, const uint32_t* amax1, void* Y0, void* Y1, cudaStream_t s,
+                               DeviceStatus* st);
+cudaError_t launch_amax_to_scale(uint32_t* amax, int n, cudaStream_t s);
 cudaError_t launch_dense_plan(int BH, int N, int32_t* q_off, int32_t* k_off, int32_t* sel_count, int32_t* sel_idx,
                               cudaStream_t s);
 
@@ -193,6 +215,9 @@ cudaError_t launch_selftest_mma(const void* A, const void* Bm, int n, const void
                                 DeviceStatus* st, cudaStream_t s);
 
 // Tensor map over a [rows, d] bf16 matrix with a box of 64 columns x box_rows rows, 128B swizzle.
+// 2D tensor map over rows of d one-byte codes (E4M3), box d x box_rows, 128-byte swizzle (d = 128).
+cudaError_t make_tmap_u8_rows(void* map /* CUtensorMap* */, const void* base, uint64_t rows, uint32_t d,
+                              uint32_t box_rows);
 cudaError_t make_tmap_bf16_rows(void* map /* CUtensorMap* */, const void* base, uint64_t rows, uint32_t d,
                                 uint32_t box_rows);
 

@@ -32,7 +32,8 @@ _EXPORTS = ("svg2_status_string", "svg2_workspace_size", "svg2_check_status", "s
             "svg2_unpermute", "svg2_layer", "svg2_layer_host", "svg2_selftest_mma", "svg2_sparse_attn_noalloc",
             "svg2_dense_attn_workspace_size", "svg2_dense_attn", "svg2_driver_create", "svg2_driver_destroy",
             "svg2_driver_cache_bytes", "svg2_driver_bind_cache", "svg2_driver_reset", "svg2_driver_workspace_size",
-            "svg2_driver_plan", "svg2_driver_layer", "svg2_set_wait_budget")
+            "svg2_driver_plan", "svg2_driver_layer", "svg2_set_wait_budget", "svg2_quantize_e4m3",
+            "svg2_sparse_attn_fp8")
 
 _lib = None
 
@@ -46,7 +47,7 @@ class Svg2Error(RuntimeError):
 class SvgParams(ctypes.Structure):
     _fields_ = [("nQ", ctypes.c_int), ("nK", ctypes.c_int), ("iters", ctypes.c_int), ("init", ctypes.c_int),
                 ("top_p", ctypes.c_float), ("scale", ctypes.c_float), ("seed_tokens", ctypes.c_int),
-                ("fuse_unpermute", ctypes.c_int)]
+                ("fuse_unpermute", ctypes.c_int), ("attn_fp8", ctypes.c_int)]
 
 
 class SvgDriverConfig(ctypes.Structure):
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.svg2_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
         L.svg2_dense_attn_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
         L.svg2_dense_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, S, P]
+        L.svg2_quantize_e4m3.argtypes = [P, I, P, I, I, I, I, P, P, P]
+        L.svg2_sparse_attn_fp8.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, S, P]
         L.svg2_driver_create.argtypes = [ctypes.POINTER(SvgDriverConfig), I, I, I, I, ctypes.POINTER(P)]
         L.svg2_driver_destroy.argtypes = [P]
         L.svg2_driver_cache_bytes.argtypes = [P, ctypes.POINTER(S)]
@@ -134,6 +137,7 @@ def _hp(t: torch.Tensor):
 
 _BF16, _F32, _F64, _I32, _U8 = (torch.bfloat16,), (torch.float32,), (torch.float64,), (torch.int32,), (torch.uint8,)
 _DATA = (torch.bfloat16, torch.float32)
+_E4M3 = (torch.uint8, torch.float8_e4m3fn)  # E4M3 codes, as raw bytes or as torch's own view of them
 
 
 def _arg(t: Optional[torch.Tensor], name: str, dtypes, numel: int, optional: bool = False, host: bool = False):
@@ -320,6 +324,36 @@ def svg2_sparse_attn(Qp: torch.Tensor, Kp: torch.Tensor, Vp: torch.Tensor, q_off
                                   _stream(stream)), "svg2_sparse_attn")
 
 
+def svg2_quantize_e4m3(X: torch.Tensor, X8: torch.Tensor, scale: torch.Tensor,
+                       perm: Optional[torch.Tensor] = None, stream=None):
+    """Per-(b,h) E4M3 codes of X (rows gathered through perm when given) and their scales."""
+    B, H, N, d = _dims(X, "X")
+    BH = B * H
+    _check(lib().svg2_quantize_e4m3(_arg(X, "X", _DATA, 0), _dtype(X), _arg(perm, "perm", _I32, BH * N, optional=True),
+                                    B, H, N, d, _arg(X8, "X8", _E4M3, BH * N * d), _arg(scale, "scale", _F32, BH),
+                                    _stream(stream)), "svg2_quantize_e4m3")
+
+
+def svg2_sparse_attn_fp8(Qp8: torch.Tensor, Kp8: torch.Tensor, Vp8: torch.Tensor, scale_q: torch.Tensor,
+                         scale_k: torch.Tensor, scale_v: torch.Tensor, q_off: torch.Tensor, k_off: torch.Tensor,
+                         sel_count: torch.Tensor, sel_idx: torch.Tensor, scale: float, O: torch.Tensor,
+                         ws: torch.Tensor, perm_q: Optional[torch.Tensor] = None, stream=None):
+    """svg2_sparse_attn on E4M3 codes with per-(b,h) dequantisation scales (d = 128)."""
+    B, H, N, d = _dims(Qp8, "Qp8")
+    if q_off is None or k_off is None or q_off.dim() < 1 or k_off.dim() < 1:
+        raise ValueError("q_off and k_off are required")
+    BH, n = B * H, B * H * N * d
+    nQ = int(q_off.shape[-1]) - 1
+    nK = int(k_off.shape[-1]) - 1
+    _check(lib().svg2_sparse_attn_fp8(
+        _arg(Qp8, "Qp8", _E4M3, 0), _arg(Kp8, "Kp8", _E4M3, n), _arg(Vp8, "Vp8", _E4M3, n),
+        _arg(scale_q, "scale_q", _F32, BH), _arg(scale_k, "scale_k", _F32, BH), _arg(scale_v, "scale_v", _F32, BH),
+        _arg(q_off, "q_off", _I32, BH * (nQ + 1)), _arg(k_off, "k_off", _I32, BH * (nK + 1)),
+        _arg(sel_count, "sel_count", _I32, BH * nQ), _arg(sel_idx, "sel_idx", _I32, BH * nQ * nK), B, H, N, d, nQ,
+        nK, float(scale), _arg(perm_q, "perm_q", _I32, BH * N, optional=True), _arg(O, "O", _BF16, n), _p(ws),
+        _nbytes(ws), _stream(stream)), "svg2_sparse_attn_fp8")
+
+
 def svg2_dense_attn_workspace_size(B: int, H: int, N: int, d: int) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().svg2_dense_attn_workspace_size(B, H, N, d, ctypes.byref(out)), "svg2_dense_attn_workspace_size")
@@ -368,10 +402,11 @@ class LayerParams:
     scale: float = 1.0 / 128 ** 0.5
     fuse_unpermute: int = 1
     seed_tokens: int = DEFAULT_SEED_TOKENS
+    attn_fp8: int = 0
 
     def c(self) -> SvgParams:
         return SvgParams(self.nQ, self.nK, self.iters, self.init, self.top_p, self.scale, self.seed_tokens,
-                         self.fuse_unpermute)
+                         self.fuse_unpermute, self.attn_fp8)
 
 
 def layer_output_buffers(B: int, H: int, N: int, nQ: int, nK: int, device="cuda") -> Dict[str, torch.Tensor]:

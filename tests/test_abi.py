@@ -209,3 +209,32 @@ def test_dense_attn_rejects_bad_arguments(L):
 def test_set_wait_budget_rejects_a_missing_or_misaligned_workspace(L):
     assert L.svg2_set_wait_budget(None, 100, None) == INVALID
     assert L.svg2_set_wait_budget(ctypes.c_void_p(0x10010), 100, None) == INVALID  # not 256-byte aligned
+
+
+def test_fp8_calls_reject_bad_arguments(L):
+    from sparse_attention_video_head_b200.svg2 import SvgParams
+    F = ctypes.c_float
+    q = lambda X=FAKE, dt=0, perm=None, d=128, X8=FAKE, sc=FAKE: L.svg2_quantize_e4m3(X, dt, perm, 1, 2, 100, d, X8, sc, None)
+    assert q(X=None) == INVALID
+    assert q(X8=None) == INVALID
+    assert q(sc=None) == INVALID
+    assert q(dt=7) == INVALID
+    assert q(d=96) == UNSUPPORTED
+    assert q(X8=ctypes.c_void_p(0x10008)) == INVALID          # not 16-byte aligned
+
+    def a(d=128, sq=FAKE, V8=FAKE, s=0.1, wsb=1 << 30):
+        return L.svg2_sparse_attn_fp8(FAKE, FAKE, V8, sq, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1000, d, 4, 4,
+                                      F(s), None, FAKE, FAKE, wsb, None)
+    assert a(d=64) == UNSUPPORTED                              # the FP8 kernel is built for d = 128
+    assert a(d=96) == UNSUPPORTED
+    assert a(sq=None) == INVALID
+    assert a(V8=None) == INVALID
+    assert a(s=float("nan")) == INVALID
+    assert a(wsb=64) == WORKSPACE
+
+    args = [FAKE, FAKE, FAKE, 0, 1, 1, 1000, 128, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 34, None]
+    bad = SvgParams(4, 8, 2, 1, 0.9, 0.1, 0, 1, 2)           # attn_fp8 is 0 or 1
+    assert L.svg2_layer(*args[:8], ctypes.byref(bad), *args[9:]) == INVALID
+    fp8 = SvgParams(4, 8, 2, 1, 0.9, 0.1, 0, 1, 1)
+    assert L.svg2_layer(*args[:7], 64, ctypes.byref(fp8), *args[9:]) == UNSUPPORTED
+

@@ -17,7 +17,7 @@ from tests.gpu_helpers import bf16_dev, host, pool_layer_inputs, require_gpu, to
 MAX_ABS, MEAN_ABS, REL_L2 = 2e-2, 2e-3, 1e-2
 
 
-def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1, seed_tokens=None):
+def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1, seed_tokens=None, attn_fp8=0):
     B, H, N, d = data["q"].shape
     conv = to_dev if cfg.dtype == "f32" else bf16_dev
     Q, K, V = conv(data["q"]), conv(data["k"]), conv(data["v"])
@@ -28,7 +28,7 @@ def run_layer(svg2, cfg, data, top_p, init=None, cq=None, ck=None, fuse=1, seed_
     ws = svg2.workspace(B, H, N, d, cfg.nQ, cfg.nK)
     prm = svg2.LayerParams(cfg.nQ, cfg.nK, cfg.iters, svg2.SVG2_INIT_KMEANSPP if init is None else init, top_p,
                            float(np.float32(cfg.scale)), fuse,
-                           svg2.DEFAULT_SEED_TOKENS if seed_tokens is None else seed_tokens)
+                           svg2.DEFAULT_SEED_TOKENS if seed_tokens is None else seed_tokens, attn_fp8)
     svg2.svg2_layer(Q, K, V, prm, cq, ck, O, ws, to_dev(data["uq"]), to_dev(data["uk"]), outs)
     torch.cuda.synchronize()
     svg2.raise_on_device_error(ws)
