@@ -82,11 +82,13 @@ def test_call_validation(svg2):
 
 
 @pytest.mark.gpu
-def test_driver_calls_equal_the_layer_calls_they_stand_for():
+@pytest.mark.parametrize("attn_fp8", [0, 1])
+def test_driver_calls_equal_the_layer_calls_they_stand_for(attn_fp8):
     svg2 = require_gpu()
     cfg = I.CONFIGS["small"]
     H, N, d = 2, cfg.N, cfg.d
-    params = svg2.LayerParams(nQ=cfg.nQ, nK=cfg.nK, iters=cfg.iters, top_p=0.9, scale=float(np.float32(cfg.scale)))
+    params = svg2.LayerParams(nQ=cfg.nQ, nK=cfg.nK, iters=cfg.iters, top_p=0.9, scale=float(np.float32(cfg.scale)),
+                              attn_fp8=attn_fp8)
     steps, layers = 4, 2
     drv = svg2.Driver(1, H, N, d, num_steps=steps, num_layers=layers, dense_steps=1, warm_iters=2, params=params)
     rng = np.random.default_rng(3)

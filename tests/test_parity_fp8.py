@@ -245,3 +245,39 @@ def test_fp8_rejects_other_head_dims():
     with pytest.raises(svg2.Svg2Error) as e:
         svg2.svg2_sparse_attn_fp8(x, x, x, s, s, s, off, off, cnt, idx, 0.125, O, ws)
     assert e.value.code == 2  # SVG2_ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+def test_fp8_layer_from_float32_inputs(oracle):
+    """The FP8 layer on float32 inputs: the quantiser reads the float32 values themselves (not a bf16
+    rounding of them), so the oracle quantises the float32 planes."""
+    from types import SimpleNamespace
+    from tests.test_layer import run_layer
+    svg2 = require_gpu()
+    rng = np.random.default_rng(90)
+    H, N, d, nQ, nK = 2, 1500, 128, 10, 30
+
+    def mixture(comps=6, sigma=0.3):
+        out = np.empty((1, H, N, d), np.float32)
+        for h in range(H):
+            centres = rng.standard_normal((comps, d), dtype=np.float32)
+            out[0, h] = centres[rng.integers(0, comps, N)] + sigma * rng.standard_normal((N, d), dtype=np.float32)
+        return out
+
+    data = {"q": mixture(), "k": mixture(), "v": rng.standard_normal((1, H, N, d), dtype=np.float32),
+            "uq": rng.random((1, H, nQ)), "uk": rng.random((1, H, nK))}
+    assert not np.array_equal(data["q"], I.round_to_bf16(data["q"]))
+    cfg = SimpleNamespace(nQ=nQ, nK=nK, iters=3, scale=float(np.float32(1 / np.sqrt(d))), dtype="f32")
+    res = run_layer(svg2, cfg, data, 0.9, seed_tokens=0, attn_fp8=1)
+    rels = []
+    for h in range(H):
+        (Q8, sq), (K8, sk), (V8, sv) = (_quantize_oracle(oracle, data[x][:, h:h + 1]) for x in ("q", "k", "v"))
+        pq, pk = res["perm_q"][0, h], res["perm_k"][0, h]
+        inv = np.empty_like(pq)
+        inv[pq] = np.arange(pq.size, dtype=np.int32)
+        ref = oracle.sparse_attention_fp8_rows(Q8[0, 0][pq], K8[0, 0][pk], V8[0, 0][pk], sq[0, 0], sk[0, 0],
+                                               sv[0, 0], res["q_off"][0, h], res["k_off"][0, h], res["mask"][0, h],
+                                               cfg.scale, inv)
+        rels.append(rel_l2(res["o"][0, h], ref))
+    print("relative L2 per head", rels)
+    assert max(rels) <= REL_L2, rels
