@@ -87,10 +87,10 @@ def gen_inputs(cfg, step=0, heads=None):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 238.9 MB + 61.6 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 237.9 MB + 62.3 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "b338eb4f9b8fdff3be62ab0bd058c02e3e9cfb5dbc952483d05e4e046e59e59a",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 238.888448e6 + 61.553152e6,
+ATTN_TRAFFIC = {"sha256": "a680326d9280a5135cd8673d8dd045419125b040aedbef24837f14cc9c9c6a17",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 237.852672e6 + 62.337536e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 
