@@ -87,10 +87,10 @@ def gen_inputs(cfg, step=0, heads=None):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 237.9 MB + 62.3 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 241.7 MB + 66.9 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "a680326d9280a5135cd8673d8dd045419125b040aedbef24837f14cc9c9c6a17",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 237.852672e6 + 62.337536e6,
+ATTN_TRAFFIC = {"sha256": "2272645a4c4d9484d3493dcdeca04f2d1a1f2e15d70ecc6d941d63c5f58da12e",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 241.663232e6 + 66.939648e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 

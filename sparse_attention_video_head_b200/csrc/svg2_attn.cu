@@ -401,12 +401,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // per tile would cost a chain of dependent shared-memory reads); then every cp.async instruction
     // moves whole rows (16 lanes x 16 bytes per row at d = 128), so one instruction touches 2 rows.
     constexpr int CPR = kRowBytes / 16;  // 16-byte chunks per row
-    constexpr int RPI = 32 / CPR;    // rows per warp instruction
+    constexpr int RPI = 32 / CPR;        // rows per warp instruction
+    constexpr int kIters = 64 / RPI;     // instructions per tile and operand
+    constexpr int kPeriod = 8 / RPI;     // the row's place in its 8-row swizzle group repeats this often
     const int wr0 = (warp - kProducerWarp0) * 64;
     const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
-    const size_t head_row0 = static_cast<size_t>(bh) * N;
+    const uint32_t head_row0 = static_cast<uint32_t>(bh) * static_cast<uint32_t>(N);  // B*H*N < 2^31
     const int my_chunk = lane % CPR, my_sub = lane / CPR;
     const int hf = my_chunk >> 3, cc = my_chunk & 7;
+    // This thread's byte offset within a tile for instruction it is xo[it % kPeriod] + it * RPI * 128
+    // (row rr = it * RPI + my_sub, 128-byte swizzle: chunk cc lands at cc ^ (rr & 7)).
+    uint32_t xo[kPeriod];
+#pragma unroll
+    for (int k = 0; k < kPeriod; ++k)
+      xo[k] = hf * 16384 + (wr0 + my_sub) * 128 + ((cc ^ ((k * RPI + my_sub) & 7)) << 4);
+    const AttnElem<F8>* kbase = Kp + my_chunk * (16 / sizeof(AttnElem<F8>));
+    const AttnElem<F8>* vbase = Vp + my_chunk * (16 / sizeof(AttnElem<F8>));
     int e0c = 0, e1c = 0;  // cursors of this lane's two stream positions: r_cum[e] <= p < r_cum[e + 1]
     auto src_row = [&](int p, int& e) {
       if (p >= L) p = L - 1;
@@ -417,7 +427,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     };
     for (int j = 0; j < T; ++j) {
       const int stage = j & 1;
-      const int krow0 = src_row(j * 128 + wr0 + lane, e0c), krow1 = src_row(j * 128 + wr0 + 32 + lane, e1c);
+      // global rows of this lane's two stream positions; a K row and its V row share the index
+      const uint32_t g0 = head_row0 + static_cast<uint32_t>(src_row(j * 128 + wr0 + lane, e0c));
+      const uint32_t g1 = head_row0 + static_cast<uint32_t>(src_row(j * 128 + wr0 + 32 + lane, e1c));
       const uint32_t kdst = kb + stage * kTile, vdst = vb + stage * kTile;
       // K(j) may land as soon as both S products of K(j-2) are done, V(j) once both PV products of
       // V(j-2) are; each lands asynchronously and counts itself on its full barrier
@@ -425,20 +437,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                                              kWhereAttnProducer, 128, wb)))
         break;
 #pragma unroll
-      for (int it = 0; it < 64 / RPI; ++it) {
-        const int rr = it * RPI + my_sub;  // row within the warp's 64
-        const int src = __shfl_sync(0xffffffffu, rr < 32 ? krow0 : krow1, rr & 31);
-        cp_async16(kdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Kp + (head_row0 + src) * D + my_chunk * (16 / sizeof(AttnElem<F8>)));
+      for (int it = 0; it < kIters; ++it) {
+        // row it * RPI + my_sub of the warp's 64: below 32 exactly when it < kIters / 2
+        const uint32_t g = __shfl_sync(0xffffffffu, it < kIters / 2 ? g0 : g1, (it * RPI + my_sub) & 31);
+        cp_async16(kdst + xo[it % kPeriod] + it * RPI * 128, kbase + static_cast<size_t>(g) * D);
       }
       cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_sleep(smem_u32(&bars->v_empty[stage]), ((j >> 1) - 1) & 1, st,
                                                              kWhereAttnProducer, 128, wb)))
         break;
 #pragma unroll
-      for (int it = 0; it < 64 / RPI; ++it) {
-        const int rr = it * RPI + my_sub;
-        const int src = __shfl_sync(0xffffffffu, rr < 32 ? krow0 : krow1, rr & 31);
-        cp_async16(vdst + hf * 16384 + sw128_offset(wr0 + rr, cc), Vp + (head_row0 + src) * D + my_chunk * (16 / sizeof(AttnElem<F8>)));
+      for (int it = 0; it < kIters; ++it) {
+        const uint32_t g = __shfl_sync(0xffffffffu, it < kIters / 2 ? g0 : g1, (it * RPI + my_sub) & 31);
+        cp_async16(vdst + xo[it % kPeriod] + it * RPI * 128, vbase + static_cast<size_t>(g) * D);
       }
       cp_async_mbar_arrive(smem_u32(&bars->v_full[stage]));
     }
