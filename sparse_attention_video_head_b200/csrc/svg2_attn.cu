@@ -7,10 +7,12 @@
 // Blackwell execution model rather than the pages' FlashInfer-derived kernel:
 //   warps 0-3   softmax + lazy O rescale + epilogue for Q tile A (TMEM lanes = query rows)
 //   warps 4-7   the same for Q tile B
-//   warps 8-9   key/value producer: each thread gathers two rows of each key tile with cp.async
-//               into the 128-byte-swizzled layout the tensor core reads (two stages)
+//   warps 8, 9, 11  key/value producers (rows 0-47, 48-87, 88-127 of each key tile; warps 8-9 also
+//               build the kept clusters' range table): cp.async gathers into the 128-byte-swizzled
+//               layout the tensor core reads (two stages).  Three warps on three SMSPs, because each
+//               SMSP also runs two softmax warps and the slowest of those sets the pace.
 //   warp 10     TMEM allocator (512 columns: S_A, S_B, O_A, O_B), Q tiles by TMA, then the
-//               single-thread MMA issuer; warp 11 idles (setmaxnreg acts on whole warpgroups)
+//               single-thread MMA issuer
 // After set-up the softmax warps take 184 registers per thread and the rest 120.  Each Q tile has one
 // 128-column S slot: S = Q K^T is one N = 128 product per key tile (full rate; a 64-key product is
 // bound by the shared-memory reads of its operands), and P (bf16) overwrites the slot's first 64
@@ -32,11 +34,11 @@ namespace svg2 {
 
 namespace {
 
-// 12 warps in three warpgroups: 8 softmax warps, 2 key/value producer warps, the MMA issuer and
-// one idle warp (setmaxnreg acts on whole warpgroups).
+// 12 warps in three warpgroups: 8 softmax warps, then 3 key/value producer warps and the MMA issuer.
 constexpr int kAttnThreads = 384;
-constexpr int kProducerWarp0 = 8, kProducerWarps = 2;
+constexpr int kProducerWarp0 = 8, kProducerWarps = 2;  // the warps that build the range table
 constexpr int kProducerThreads = 32 * kProducerWarps;
+constexpr int kGatherThreads = 96;                      // warps 8, 9 and 11 gather K and V
 constexpr int kMmaWarp = 10;
 // Register split after set-up (setmaxnreg): 256 x 184 + 128 x 120 = 62464 <= 384 x 168, the launch's
 // allocation under __launch_bounds__(384, 1) (ptxas gives 168 registers per thread).
@@ -171,8 +173,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars->k_full[i]), kProducerThreads);
-      mbar_init(smem_u32(&bars->v_full[i]), kProducerThreads);
+      mbar_init(smem_u32(&bars->k_full[i]), kGatherThreads);
+      mbar_init(smem_u32(&bars->v_full[i]), kGatherThreads);
       mbar_init(smem_u32(&bars->k_empty[i]), 1);
       mbar_init(smem_u32(&bars->v_empty[i]), 1);
       mbar_init(smem_u32(&bars->s_full[i]), 1);
@@ -393,18 +395,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(smem_u32(&bars->mma_done), 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
       if (!ok) mbar_wait(qbar, 0, nullptr, kWhereAttnDrain, kWaitBudgetCycles / 8);
     }
-  } else if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducerWarps) {
+  } else if (warp == 8 || warp == 9 || warp == 11) {
     // ---------------- key/value gather producer ----------------
-    // Warp w fills rows 64w'..64w'+63 of each key tile (w' = w - first producer warp).  Each lane
+    // Warps 8, 9 and 11 fill rows 0-47, 48-87 and 88-127 of each key tile.  Each lane
     // follows the source rows of two stream positions from tile to tile with cursors over the range
     // table (positions only grow, so each cursor crosses every range boundary once, where a search
     // per tile would cost a chain of dependent shared-memory reads); then every cp.async instruction
     // moves whole rows (16 lanes x 16 bytes per row at d = 128), so one instruction touches 2 rows.
     constexpr int CPR = kRowBytes / 16;  // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;        // rows per warp instruction
-    constexpr int kIters = 64 / RPI;     // instructions per tile and operand
+    constexpr int kIters = 48 / RPI;     // at most this many instructions per tile and operand
     constexpr int kPeriod = 8 / RPI;     // the row's place in its 8-row swizzle group repeats this often
-    const int wr0 = (warp - kProducerWarp0) * 64;
+    const int pw = warp == 11 ? 2 : warp - 8;
+    const int wr0 = pw == 0 ? 0 : (pw == 1 ? 48 : 88);   // rows 0-47, 48-87, 88-127 (multiples of 8)
+    const int nrw = pw == 0 ? 48 : 40;
     const uint32_t kb = smem_u32(k_s), vb = smem_u32(v_s);
     const uint32_t head_row0 = static_cast<uint32_t>(bh) * static_cast<uint32_t>(N);  // B*H*N < 2^31
     const int my_chunk = lane % CPR, my_sub = lane / CPR;
@@ -438,8 +442,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
 #pragma unroll
       for (int it = 0; it < kIters; ++it) {
-        // row it * RPI + my_sub of the warp's 64: below 32 exactly when it < kIters / 2
-        const uint32_t g = __shfl_sync(0xffffffffu, it < kIters / 2 ? g0 : g1, (it * RPI + my_sub) & 31);
+        if (it * RPI >= nrw) break;
+        // row it * RPI + my_sub of the warp's rows: below 32 exactly when it * RPI < 32
+        const uint32_t g = __shfl_sync(0xffffffffu, it * RPI < 32 ? g0 : g1, (it * RPI + my_sub) & 31);
         cp_async16(kdst + xo[it % kPeriod] + it * RPI * 128, kbase + static_cast<size_t>(g) * D);
       }
       cp_async_mbar_arrive(smem_u32(&bars->k_full[stage]));
@@ -448,7 +453,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
 #pragma unroll
       for (int it = 0; it < kIters; ++it) {
-        const uint32_t g = __shfl_sync(0xffffffffu, it < kIters / 2 ? g0 : g1, (it * RPI + my_sub) & 31);
+        if (it * RPI >= nrw) break;
+        const uint32_t g = __shfl_sync(0xffffffffu, it * RPI < 32 ? g0 : g1, (it * RPI + my_sub) & 31);
         cp_async16(vdst + xo[it % kPeriod] + it * RPI * 128, vbase + static_cast<size_t>(g) * D);
       }
       cp_async_mbar_arrive(smem_u32(&bars->v_full[stage]));
