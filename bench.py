@@ -87,10 +87,10 @@ def gen_inputs(cfg, step=0, heads=None):
 
 
 # DRAM traffic of one sparse-attention launch from an ncu capture of a 4-head cut of the Wan-720p
-# layer (dram__bytes_read.sum + dram__bytes_write.sum = 242.1 MB + 67.4 MB), scaled by heads; valid
+# layer (dram__bytes_read.sum + dram__bytes_write.sum = 242.6 MB + 62.9 MB), scaled by heads; valid
 # only for the kernel source it was taken on (sha256 of svg2_attn.cu), else reported as null.
-ATTN_TRAFFIC = {"sha256": "7e5ad927a2d5ab7ae8473860f73f5be6a5c31357bcdd87c8a4f03d24ac2950a5",
-                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 242.093824e6 + 67.359232e6,
+ATTN_TRAFFIC = {"sha256": "5d676feb5bb9696a0912839103b85c5bd59af583faf74c082eb38fb0c5d484f9",
+                "workload": "wan720p", "heads_captured": 4, "bytes_captured": 242.608128e6 + 62.930688e6,
                 "summary": "profiles/sparse_attn_kernel_wan720p_4heads.md"}
 
 

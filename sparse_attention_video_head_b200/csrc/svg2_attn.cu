@@ -13,7 +13,7 @@
 //               SMSP also runs two softmax warps and the slowest of those sets the pace.
 //   warp 10     TMEM allocator (512 columns: S_A, S_B, O_A, O_B), Q tiles by TMA, then the
 //               single-thread MMA issuer
-// After set-up the softmax warps take 184 registers per thread and the rest 120.  Each Q tile has one
+// After set-up the softmax warps take 176 registers per thread and the rest 136.  Each Q tile has one
 // 128-column S slot: S = Q K^T is one N = 128 product per key tile (full rate; a 64-key product is
 // bound by the shared-memory reads of its operands), and P (bf16) overwrites the slot's first 64
 // columns as the A operand of the PV product.  MMA order per key tile j: PV_A(j), S_A(j+1),
@@ -40,11 +40,11 @@ constexpr int kProducerWarp0 = 8, kProducerWarps = 2;  // the warps that build t
 constexpr int kProducerThreads = 32 * kProducerWarps;
 constexpr int kGatherThreads = 96;                      // warps 8, 9 and 11 gather K and V
 constexpr int kMmaWarp = 10;
-// Register split after set-up (setmaxnreg): 256 x 184 + 128 x 120 = 62464 <= 384 x 168, the launch's
+// Register split after set-up (setmaxnreg): 256 x 176 + 128 x 136 = 62464 <= 384 x 168, the launch's
 // allocation under __launch_bounds__(384, 1) (ptxas gives 168 registers per thread).
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 184;
-constexpr int kOtherRegs = 120;
+constexpr int kSoftmaxRegs = 176;  // in steps of 8, the split at which neither side spills (168: softmax; 184: the rest)
+constexpr int kOtherRegs = 136;
 static_assert(256 * kSoftmaxRegs + (kAttnThreads - 256) * kOtherRegs <= kAttnThreads * kLaunchRegs, "register split");
 constexpr int kMaxRanges = 1024;
 // bytes of one 128-row tile of d values: bf16, or E4M3 codes in the FP8 variant (16 KB column blocks of
