@@ -66,8 +66,9 @@ typedef enum { SVG2_INIT_GIVEN = 0, SVG2_INIT_KMEANSPP = 1 } svg2_init;
  * the seeding cheap on video-length layers. */
 #define SVG2_DEFAULT_SEED_TOKENS 16384
 
-/* Largest sizes the library supports.  Besides these, B*H <= 2^20 and B*H*N < 2^31 (token rows
- * across all planes are indexed with 32-bit integers); larger sizes return SVG2_ERR_UNSUPPORTED. */
+/* Largest sizes the library supports.  Besides these, B*H <= 65535 (several kernels give the (b,h)
+ * planes a grid dimension of their own) and B*H*N < 2^31 (token rows across all planes are indexed
+ * with 32-bit integers); larger sizes return SVG2_ERR_UNSUPPORTED. */
 #define SVG2_MAX_CLUSTERS 1024
 #define SVG2_MAX_TOKENS (1 << 24)
 

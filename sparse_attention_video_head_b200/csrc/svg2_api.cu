@@ -41,7 +41,8 @@ bool valid_dtype(int dt) { return dt == SVG2_BF16 || dt == SVG2_F32; }
 int check_sizes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1) return SVG2_ERR_INVALID_ARG;
   if (N > SVG2_MAX_TOKENS) return SVG2_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H > (1 << 20)) return SVG2_ERR_UNSUPPORTED;
+  // the (b,h) planes are a grid dimension of their own in several kernels (at most 65535)
+  if (static_cast<long long>(B) * H > 65535) return SVG2_ERR_UNSUPPORTED;
   // token rows across all planes are indexed (and addressed by TMA) with 32-bit integers
   if (static_cast<long long>(B) * H * N >= (1LL << 31)) return SVG2_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return SVG2_ERR_UNSUPPORTED;

@@ -56,7 +56,7 @@ extern "C" SVG2_API int svg2_sparse_attn_noalloc(const void* Qp, const void* Kp,
     if ((mis & 15u) != 0 || scale != scale) return SVG2_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(device_status) & 15u) != 0) return SVG2_ERR_INVALID_ARG;
     const long long BH = static_cast<long long>(B) * H;
-    if (BH > (1 << 20) || BH * N >= (1LL << 31)) return SVG2_ERR_UNSUPPORTED;
+    if (BH > 65535 || BH * N >= (1LL << 31)) return SVG2_ERR_UNSUPPORTED;
     // the same layout the workspace path uses: status word, then the work plan
     Carve measure(nullptr);
     measure.take<DeviceStatus>(kStatusBytes / sizeof(DeviceStatus));

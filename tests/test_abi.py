@@ -67,10 +67,12 @@ def test_workspace_size_is_monotone_and_validates(L):
     assert L.svg2_workspace_size(1, 1, 5000, 128, 2000, 4, ctypes.byref(out)) == UNSUPPORTED
     assert L.svg2_workspace_size(0, 1, 100, 128, 4, 4, ctypes.byref(out)) == INVALID
     assert L.svg2_workspace_size(1, 1, 100, 128, 4, 4, None) == INVALID
-    # B*H*N must stay below 2^31 rows; B*H at most 2^20
+    # B*H*N must stay below 2^31 rows; B*H at most 65535 (a grid dimension in several kernels)
     assert L.svg2_workspace_size(1, 256, 1 << 23, 128, 4, 4, ctypes.byref(out)) == UNSUPPORTED
     assert L.svg2_workspace_size(2, 128, (1 << 23) - 1, 128, 4, 4, ctypes.byref(out)) == OK
     assert L.svg2_workspace_size(1, (1 << 20) + 1, 4, 128, 4, 4, ctypes.byref(out)) == UNSUPPORTED
+    assert L.svg2_workspace_size(1, 65536, 4, 128, 4, 4, ctypes.byref(out)) == UNSUPPORTED
+    assert L.svg2_workspace_size(3, 21845, 4, 128, 4, 4, ctypes.byref(out)) == OK
 
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation first
