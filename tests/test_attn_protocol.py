@@ -3,8 +3,9 @@
 The attention kernel (svg2_attn.cu) hands its work from agent to agent through mbarriers that are
 waited on by phase parity:
 
-* the producer warps gather K(j) and V(j) into shared-memory stage j % 2 with cp.async. Each
-  copy lands asynchronously and arrives on k_full / v_full. The producer waits on k_empty / v_empty
+* the producer warps (three, each writing its own rows of a tile) gather K(j) and V(j) into
+  shared-memory stage j % 2 with cp.async. Each warp's copies land asynchronously and arrive on
+  k_full / v_full, which complete once every warp has arrived. Each warp waits on k_empty / v_empty
   before it reuses a stage.
 * the MMA thread issues S = Q K^T into a tensor-memory slot, and PV in two 64-key halves. Its
   commits arrive on s_full, k_empty, v_empty, pv_done and o_full once every earlier product has
@@ -22,7 +23,8 @@ against what the schedule intends, which catches a stage or slot overwritten too
 The model restates the protocol, not the code. A change to the kernel's barrier scheme must be
 made here too. ``test_shared_p_barriers_in_ring_mode_deadlock`` plants the single P barrier pair
 that ring mode once shared between consecutive tiles. It checks that the model finds the resulting
-hang, which the device reported as a bounded-wait timeout in the MMA thread.
+hang, which the device reported as a bounded-wait timeout in the MMA thread, and the early reads
+the same sharing allows.
 """
 import random
 
@@ -59,16 +61,18 @@ def check(cond, what):
 class Kernel:
     """One CTA of the attention kernel: one unit of one or two Q tiles over T key tiles."""
 
-    def __init__(self, T, has_b, rng, shared_p=False):
-        self.T, self.has_b, self.rng, self.shared_p = T, has_b, rng, shared_p
-        self.k_full = [Bar(1), Bar(1)]
-        self.v_full = [Bar(1), Bar(1)]
+    def __init__(self, T, has_b, rng, shared_p=False, producers=3):
+        self.T, self.has_b, self.rng, self.shared_p, self.producers = T, has_b, rng, shared_p, producers
+        self.k_full = [Bar(producers), Bar(producers)]
+        self.v_full = [Bar(producers), Bar(producers)]
         self.k_empty = [Bar(1), Bar(1)]
         self.v_empty = [Bar(1), Bar(1)]
         self.s_full = [Bar(1), Bar(1)]
         self.p_full = [[Bar(4), Bar(4)], [Bar(4), Bar(4)]]
         self.pv_done, self.o_full = Bar(1), Bar(1)
-        self.k_smem, self.v_smem = [None, None], [None, None]
+        # shared memory: per stage, the tile each producer's rows hold
+        self.k_smem = [[None] * producers for _ in range(2)]
+        self.v_smem = [[None] * producers for _ in range(2)]
         # tensor memory: per slot and warp quarter, the S tile held and the P halves written over it
         self.s_tm = [[None] * 4 for _ in range(2)]
         self.p_tm = [[[None, None] for _ in range(4)] for _ in range(2)]
@@ -82,13 +86,13 @@ class Kernel:
         kind = op[0]
         if kind == "S":
             _, x, j, stage, slot = op
-            check(self.k_smem[stage] == ("K", j), f"S_{x}({j}) read stage {stage} holding {self.k_smem[stage]}")
+            check(all(r == ("K", j) for r in self.k_smem[stage]), f"S_{x}({j}) read stage {stage} holding {self.k_smem[stage]}")
             for q in range(4):
                 self.s_tm[slot][q] = (x, j)
                 self.p_tm[slot][q] = [None, None]
         elif kind == "PV":
             _, x, j, slot, stage, h = op
-            check(self.v_smem[stage] == ("V", j), f"PV_{x}({j}) read stage {stage} holding {self.v_smem[stage]}")
+            check(all(r == ("V", j) for r in self.v_smem[stage]), f"PV_{x}({j}) read stage {stage} holding {self.v_smem[stage]}")
             for q in range(4):
                 check(self.p_tm[slot][q][h] == (x, j), f"PV_{x}({j}) half {h} read {self.p_tm[slot][q][h]}")
                 check(not self.in_rescale[x][q], f"PV_{x}({j}) ran during a rescale of O_{x}")
@@ -99,26 +103,26 @@ class Kernel:
 
     def run_copy(self):
         i = self.rng.randrange(len(self.copies))
-        smem, stage, val, bar = self.copies.pop(i)
-        smem[stage] = val
+        rows, w, val, bar = self.copies.pop(i)
+        rows[w] = val
         bar.arrive()
 
     # ---- agents: each yields a wait condition (or None for a plain step) ----
     def wait(self, bar, parity):
         return lambda: bar.done(parity)
 
-    def producer(self):
+    def producer(self, w):
         for j in range(self.T):
             st = j & 1
             if j >= 2:
                 yield self.wait(self.k_empty[st], ((j >> 1) - 1) & 1)
-            self.k_smem[st] = ("landing", j)
-            self.copies.append((self.k_smem, st, ("K", j), self.k_full[st]))
+            self.k_smem[st][w] = ("landing", j)
+            self.copies.append((self.k_smem[st], w, ("K", j), self.k_full[st]))
             yield None
             if j >= 2:
                 yield self.wait(self.v_empty[st], ((j >> 1) - 1) & 1)
-            self.v_smem[st] = ("landing", j)
-            self.copies.append((self.v_smem, st, ("V", j), self.v_full[st]))
+            self.v_smem[st][w] = ("landing", j)
+            self.copies.append((self.v_smem[st], w, ("V", j), self.v_full[st]))
             yield None
 
     def mma(self):
@@ -209,7 +213,8 @@ def run_schedule(T, has_b, seed, shared_p=False, max_steps=100000):
     """Run one random interleaving; raise ProtocolError on a hazard or a deadlock."""
     rng = random.Random(seed)
     k = Kernel(T, has_b, rng, shared_p)
-    agents = {"producer": k.producer(), "mma": k.mma()}
+    agents = {f"producer{w}": k.producer(w) for w in range(k.producers)}
+    agents["mma"] = k.mma()
     for x in range(2 if has_b else 1):
         for w in range(4):
             agents[f"softmax{x}.{w}"] = k.softmax(x, w)
@@ -248,9 +253,10 @@ def test_protocol_has_no_deadlock_or_hazard(T, has_b):
 @pytest.mark.parametrize("T", [2, 3, 5])
 def test_shared_p_barriers_in_ring_mode_deadlock(T):
     """One P barrier pair shared by consecutive ring-mode tiles lets the softmax complete two
-    phases before the MMA thread waits for the first. Some interleavings then hang. From three
-    tiles on, others let a wait pass on the wrong phase, so a PV product reads P before it is
-    written."""
+    phases before the MMA thread waits for the first, so some interleavings hang. Others let a
+    phase complete on arrivals meant for two different tiles (one softmax warp a tile ahead of
+    another), or let a wait pass on the wrong phase, so a PV product reads P before it is written.
+    Every tile count shows the fault; from three tiles on, 400 schedules show both forms."""
     deadlocks = hazards = 0
     for seed in range(400):
         try:
@@ -260,6 +266,6 @@ def test_shared_p_barriers_in_ring_mode_deadlock(T):
                 deadlocks += 1
             else:
                 hazards += 1
-    assert deadlocks > 0
+    assert deadlocks + hazards > 0
     if T >= 3:
-        assert hazards > 0
+        assert deadlocks > 0 and hazards > 0
