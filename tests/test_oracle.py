@@ -531,3 +531,20 @@ def test_fp8_attention_is_attention_over_the_dequantised_values(oracle):
     ck = np.repeat(np.arange(nK), np.diff(k_off))
     tok = mask[cq][:, ck].astype(bool)
     np.testing.assert_allclose(out, _sdpa64(*deq, scale, tok), rtol=1e-9, atol=1e-12)
+
+
+def test_e4m3_handworked_golden(oracle):
+    """Hand-worked E4M3 cases from the format's definition (tests/golden/e4m3_handworked.json)."""
+    g = json.load(open(os.path.join(GOLDEN, "e4m3_handworked.json")))
+    for c in g["round"]:
+        assert oracle.e4m3_round([c["x"]])[0] == int(c["code"], 16), c["note"]
+    for c in g["value"]:
+        v = oracle.e4m3_value(np.array([int(c["code"], 16)], np.uint8))[0]
+        if c["x"] == "nan":
+            assert np.isnan(v)
+        else:
+            assert v == c["x"] and np.signbit(v) == np.signbit(c["x"]), c
+    q = g["quantize"]
+    codes, scale = oracle.quantize_e4m3(np.array([q["x"]], np.float32))
+    assert [int(c) for c in codes[0]] == [int(c, 16) for c in q["codes"]], q["note"]
+    assert scale[0] == np.float32(np.float32(q["scale_times_448"]) / np.float32(448.0))
