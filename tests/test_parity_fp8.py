@@ -281,3 +281,24 @@ def test_fp8_layer_from_float32_inputs(oracle):
         rels.append(rel_l2(res["o"][0, h], ref))
     print("relative L2 per head", rels)
     assert max(rels) <= REL_L2, rels
+
+
+def test_exact_p_bound_catches_misordered_keys(oracle):
+    """On the CPU: the exact-P bound has the power the GPU test relies on.  A wrong byte order in the
+    packed P (keys of a 4-key group multiplied by each other's V rows) is planted in the oracle's inputs
+    as V rows swapped pairwise inside every group of 4; the output then leaves the bound almost
+    everywhere, while the unplanted reference stays inside it."""
+    c = _exact_p_case(60, 1500, 10, 20, 0.5, 1)
+    scale = float(np.float32(np.log(2.0)))
+    ref = _reference(oracle, c, scale, 0)
+    planted = dict(c)
+    v = c["V8"].copy()
+    n4 = v.shape[2] // 4 * 4
+    g = v[0, 0, :n4].reshape(-1, 4, v.shape[3])
+    v[0, 0, :n4] = g[:, [2, 3, 0, 1]].reshape(n4, v.shape[3])
+    planted["V8"] = v
+    wrong = _reference(oracle, planted, scale, 0)
+    bound = (2.0 ** -8 + 2e-4) * np.abs(ref) + 1e-6 * np.abs(ref).max()
+    outside = float((np.abs(wrong - ref) > bound).mean())
+    assert outside > 0.9, outside
+    assert rel_l2(wrong, ref) > 100 * EXACT_REL_L2
