@@ -240,3 +240,19 @@ def test_fp8_calls_reject_bad_arguments(L):
     fp8 = SvgParams(4, 8, 2, 1, 0.9, 0.1, 0, 1, 1)
     assert L.svg2_layer(*args[:7], 64, ctypes.byref(fp8), *args[9:]) == UNSUPPORTED
 
+
+
+def test_noalloc_checks_sizes_before_any_cuda_call(L):
+    F = ctypes.c_float
+
+    def call(B=1, H=1, N=1000, d=128, nQ=4, nK=4, Q=FAKE):
+        return L.svg2_sparse_attn_noalloc(Q, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, H, N, d, nQ, nK, F(0.1), None,
+                                          FAKE, None, None)
+    assert call(H=65536) == UNSUPPORTED        # the (b,h) planes are a grid dimension of their own
+    assert call(B=2, H=32768) == UNSUPPORTED
+    assert call(d=96) == UNSUPPORTED
+    assert call(nQ=2000, N=5000) == UNSUPPORTED
+    assert call(B=0) == INVALID
+    assert call(nQ=1001) == INVALID            # more clusters than tokens
+    assert call(Q=None) == INVALID
+    assert call(Q=ctypes.c_void_p(0x10008)) == INVALID
